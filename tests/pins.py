@@ -1,0 +1,359 @@
+"""Pins for the CPU oracle: checks against facts fixed by the pages and by mathematics.
+
+Each pin takes an ``oracle.Oracle`` and raises AssertionError when the oracle disagrees
+with something other than itself: the hand-worked golden example, a closed form, a
+special case that reduces to a library routine (numpy matmul / lexsort, torch's
+scaled-dot-product attention), or an invariant.  They are chosen so that a plausible
+mistake anywhere in the oracle (a dropped term, a wrong sign or index, a transposed
+operand, an off-by-one in the mask) fails at least one of them; the planted-mistake test
+checks exactly that.
+"""
+from __future__ import annotations
+
+import math
+import os
+
+import numpy as np
+
+import synth
+from synth import configs as C
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def bf(x) -> np.ndarray:
+    """float values that are exact in bf16 -> bf16 bit patterns."""
+    x = np.asarray(x, dtype=np.float32)
+    bits = synth.f32_to_bf16_bits(x)
+    assert np.array_equal(synth.bf16_bits_to_f32(bits), x), "value not exact in bf16"
+    return bits
+
+
+def f(bits) -> np.ndarray:
+    return synth.bf16_bits_to_f32(bits).astype(np.float64)
+
+
+def load_golden(name: str) -> dict:
+    out = {}
+    with open(os.path.join(GOLDEN, name)) as fh:
+        for line in fh:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, *vals = line.split()
+            out[key] = vals
+    return out
+
+
+def _rng(seed: int) -> np.random.Generator:
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------------------- indexer
+
+def pin_indexer_golden(o):
+    g = load_golden("indexer_worked_example.txt")
+    nh, hd = int(g["heads"][0]), int(g["head_dim"][0])
+    q = bf(np.array(g["q"], dtype=np.float32).reshape(1, 1, nh, hd))
+    w = np.array(g["w"], dtype=np.float32).reshape(1, 1, nh)
+    keys = [g[f"k{i}"] for i in range(4)]
+    k = bf(np.array(keys, dtype=np.float32).reshape(1, 4, hd))
+    q_pos0 = int(g["q_pos0"][0])
+    s = o.index_score(q, w, k, q_pos0)
+    want = np.array([float(x) for x in g["score"]])
+    assert np.array_equal(s[0, 0], want), (s[0, 0], want)
+    sf = s.astype(np.float32)
+    assert o.topk(sf, q_pos0, 2)[0, 0].tolist() == [int(x) for x in g["top2"]]
+    assert o.topk(sf, q_pos0, 5)[0, 0].tolist() == [int(x) for x in g["top5"]]
+
+
+def pin_indexer_nonnegative_is_matmul(o):
+    """With q >= 0 and k >= 0 no dot product is negative, ReLU is the identity, and
+    I(t,s) = (sum_h w[t,h] q[t,h]) . k[s]: one matrix product."""
+    r = _rng(1)
+    B, T, nh, hd, N = 2, 3, 5, 16, 40
+    qv = r.integers(0, 9, size=(B, T, nh, hd)).astype(np.float32)
+    kv = r.integers(0, 9, size=(B, N, hd)).astype(np.float32)
+    w = np.ldexp(1.0, -r.integers(1, 7, size=(B, T, nh))).astype(np.float32)
+    s = o.index_score(bf(qv), w, bf(kv), q_pos0=N - 1)
+    qsum = np.einsum("bth,bthd->btd", w.astype(np.float64), qv.astype(np.float64))
+    want = np.matmul(qsum, np.swapaxes(kv.astype(np.float64), 1, 2))
+    assert np.array_equal(s, want)
+
+
+def pin_indexer_relu_zero(o):
+    """q >= 0 and k <= 0: every dot product is <= 0, so every visible score is 0."""
+    r = _rng(2)
+    qv = r.integers(0, 9, size=(1, 2, 4, 8)).astype(np.float32)
+    kv = -r.integers(0, 9, size=(1, 30, 8)).astype(np.float32)
+    w = np.full((1, 2, 4), 0.5, dtype=np.float32)
+    s = o.index_score(bf(qv), w, bf(kv), q_pos0=29)
+    assert np.array_equal(s[0, 0], np.zeros(30))
+
+
+def pin_indexer_one_hot(o):
+    """q[t,h] = a_h e_{i_h}, k[s] = b_s e_{j_s}: I(t,s) = sum_h w_h max(0, a_h b_s)[i_h = j_s]."""
+    r = _rng(3)
+    nh, hd, N = 6, 8, 25
+    a = r.integers(-8, 9, size=nh)
+    ih = r.integers(0, hd, size=nh)
+    bs = r.integers(-8, 9, size=N)
+    js = r.integers(0, hd, size=N)
+    qv = np.zeros((1, 1, nh, hd), np.float32)
+    qv[0, 0, np.arange(nh), ih] = a
+    kv = np.zeros((1, N, hd), np.float32)
+    kv[0, np.arange(N), js] = bs
+    w = np.ldexp(1.0, -r.integers(1, 7, size=(1, 1, nh))).astype(np.float32)
+    s = o.index_score(bf(qv), w, bf(kv), q_pos0=N - 1)
+    for sidx in range(N):
+        want = sum(float(w[0, 0, h]) * max(0, int(a[h]) * int(bs[sidx])) * (ih[h] == js[sidx])
+                   for h in range(nh))
+        assert s[0, 0, sidx] == want, (sidx, s[0, 0, sidx], want)
+
+
+def pin_indexer_causal(o):
+    """Query t sees exactly the positions s <= q_pos0 + t (and s < N)."""
+    r = _rng(4)
+    B, T, nh, hd, N, q_pos0 = 1, 5, 2, 8, 12, 6
+    qv = r.integers(-8, 9, size=(B, T, nh, hd)).astype(np.float32)
+    kv = r.integers(-8, 9, size=(B, N, hd)).astype(np.float32)
+    w = np.full((B, T, nh), 0.25, np.float32)
+    s = o.index_score(bf(qv), w, bf(kv), q_pos0)
+    for t in range(T):
+        vis = min(N, q_pos0 + t + 1)
+        assert np.all(np.isfinite(s[0, t, :vis])) and np.all(s[0, t, vis:] == -np.inf), t
+    full = o.index_score(bf(qv), w, bf(kv), q_pos0=N - 1)
+    for t in range(T):
+        vis = min(N, q_pos0 + t + 1)
+        assert np.array_equal(s[0, t, :vis], full[0, t, :vis])
+
+
+def pin_indexer_head_and_weight_structure(o):
+    """Permuting heads (with their weights) changes nothing; doubling w doubles I;
+    swapping batch items swaps the score rows."""
+    r = _rng(5)
+    B, T, nh, hd, N = 2, 2, 6, 16, 50
+    qv = r.integers(-8, 9, size=(B, T, nh, hd)).astype(np.float32)
+    kv = r.integers(-8, 9, size=(B, N, hd)).astype(np.float32)
+    w = np.ldexp(1.0, -r.integers(1, 7, size=(B, T, nh))).astype(np.float32)
+    base = o.index_score(bf(qv), w, bf(kv), N - 1)
+    perm = r.permutation(nh)
+    assert np.array_equal(o.index_score(bf(qv[:, :, perm]), w[:, :, perm], bf(kv), N - 1), base)
+    assert np.array_equal(o.index_score(bf(qv), 2 * w, bf(kv), N - 1), 2 * base)
+    sw = o.index_score(bf(qv[::-1].copy()), w[::-1].copy(), bf(kv[::-1].copy()), N - 1)
+    assert np.array_equal(sw, base[::-1])
+
+
+def pin_indexer_exact_on_workload_inputs(o):
+    """On the workloads' inputs (integers in [-8,8], w in {2^-1..2^-6}) every score is a
+    multiple of 2^-6 below 2^17, so it is exact in float32 (24-bit significand)."""
+    w = C.scaled(C.WORKLOADS["tiny"], N=300, q_pos0=299)
+    iq, wt, ik, _, _ = C.host_group_inputs(w, with_attention=False)
+    s = o.index_score(iq, wt, ik, w.q_pos0)
+    m = s * 64.0
+    assert np.array_equal(m, np.round(m)) and np.all(s >= 0) and np.all(s < 2 ** 17)
+    assert np.array_equal(s.astype(np.float32).astype(np.float64), s)
+
+
+# ----------------------------------------------------------------------------- top-k
+
+def _lexsort_topk(row: np.ndarray, vis: int, k: int) -> list:
+    """Library reference: numpy lexsort by (score descending, index ascending)."""
+    sc = row[:vis].astype(np.float64)
+    key = np.where(np.isnan(sc), -np.inf, sc)
+    nanrank = np.isnan(sc).astype(np.int64)          # numbers before NaN
+    order = np.lexsort((np.arange(vis), -key, nanrank))
+    take = sorted(order[:k].tolist())
+    return take + [-1] * (k - len(take))
+
+
+def pin_topk_matches_lexsort(o):
+    r = _rng(6)
+    for N, k, spread in [(1, 1, 5), (7, 3, 3), (100, 10, 1000), (257, 64, 4), (1000, 999, 50),
+                         (1000, 1000, 50), (1000, 1500, 50), (4096, 256, 7)]:
+        sc = (r.integers(0, spread, size=(2, 3, N)) * 0.015625).astype(np.float32)
+        idx = o.topk(sc, N - 1, k)
+        for b in range(2):
+            for t in range(3):
+                assert idx[b, t].tolist() == _lexsort_topk(sc[b, t], N, k), (N, k, b, t)
+
+
+def pin_topk_ties(o):
+    N, k = 500, 37
+    sc = np.full((1, 1, N), 3.5, np.float32)
+    assert o.topk(sc, N - 1, k)[0, 0].tolist() == list(range(k))
+    # two-valued row: every 1.0 is taken before any 0.0; among equals the lower index
+    r = _rng(7)
+    row = (r.random(N) < 0.05).astype(np.float32)
+    ones = np.flatnonzero(row == 1.0).tolist()
+    zeros = np.flatnonzero(row == 0.0).tolist()
+    want = ones[:k] if len(ones) >= k else ones + zeros[: k - len(ones)]
+    assert o.topk(row[None, None], N - 1, k)[0, 0].tolist() == sorted(want)
+    # -0 and +0 are equal scores: the lower index wins
+    row = np.array([-0.0, 0.0, -0.0, 0.0, -1.0], np.float32)
+    assert o.topk(row[None, None], 4, 2)[0, 0].tolist() == [0, 1]
+    # a NaN ranks below every number
+    row = np.array([np.nan, -5.0, np.nan, 2.0], np.float32)
+    assert o.topk(row[None, None], 3, 3)[0, 0].tolist() == [0, 1, 3]
+
+
+def pin_topk_causal_and_padding(o):
+    r = _rng(8)
+    T, N, q_pos0, k = 6, 40, 20, 24
+    sc = r.random((1, T, N)).astype(np.float32)
+    idx = o.topk(sc, q_pos0, k)
+    for t in range(T):
+        vis = min(N, q_pos0 + t + 1)
+        row = idx[0, t]
+        valid = row[row >= 0]
+        assert len(valid) == min(k, vis) and np.all(row[len(valid):] == -1)
+        assert np.all(valid <= q_pos0 + t) and np.all(np.diff(valid) > 0)
+        if vis <= k:
+            assert valid.tolist() == list(range(vis))
+        assert row.tolist() == _lexsort_topk(sc[0, t], vis, k)
+
+
+def pin_topk_selection_invariant(o):
+    """Every selected score >= every unselected visible score; equal scores split by index."""
+    r = _rng(9)
+    N, k = 3000, 200
+    sc = (r.integers(0, 300, size=(4, 1, N)) * 0.5).astype(np.float32)
+    idx = o.topk(sc, N - 1, k)
+    for b in range(4):
+        sel = idx[b, 0]
+        mask = np.zeros(N, bool)
+        mask[sel] = True
+        lo = sc[b, 0][mask].min()
+        assert sc[b, 0][~mask].max() <= lo
+        tied_out = np.flatnonzero((~mask) & (sc[b, 0] == lo))
+        tied_in = np.flatnonzero(mask & (sc[b, 0] == lo))
+        if len(tied_out):
+            assert tied_in.max() < tied_out.min()
+
+
+# ----------------------------------------------------------------------------- attention
+
+def _attn_inputs(seed, B=1, T=2, H=3, N=60, k=20, dqk=576):
+    r = _rng(seed)
+    q = bf((r.integers(-64, 65, size=(B, T, H, dqk)) / 64.0).astype(np.float32))
+    kv = bf((r.integers(-64, 65, size=(B, N, dqk)) / 64.0).astype(np.float32))
+    idx = np.stack([np.stack([np.sort(r.choice(N, size=k, replace=False)) for _ in range(T)])
+                    for _ in range(B)]).astype(np.int32)
+    return q, kv, idx
+
+
+def pin_attn_single_row(o):
+    """One valid index: the softmax weight is 1 and the output is that row's value part."""
+    q, kv, _ = _attn_inputs(10)
+    idx = np.full((1, 2, 5), -1, np.int32)
+    idx[0, 0, 3] = 17
+    idx[0, 1, 0] = 42
+    out = o.sparse_attn(q, kv, idx, C.SCALE)
+    for t, row in ((0, 17), (1, 42)):
+        for h in range(3):
+            assert np.array_equal(out[0, t, h], f(kv[0, row, :512]))
+
+
+def pin_attn_uniform_logits(o):
+    """q = 0: all logits equal, the output is the plain mean of the selected value rows."""
+    q, kv, idx = _attn_inputs(11)
+    q[:] = 0
+    out = o.sparse_attn(q, kv, idx, C.SCALE)
+    for t in range(2):
+        want = f(kv[0, idx[0, t], :512]).mean(axis=0)
+        for h in range(3):
+            assert np.allclose(out[0, t, h], want, rtol=0, atol=1e-13)
+
+
+def pin_attn_matches_torch_sdpa(o):
+    """The selected-row attention equals torch's scaled_dot_product_attention (float64)
+    over the gathered rows, with the value = the first 512 columns."""
+    import torch
+    q, kv, idx = _attn_inputs(12, B=2, T=2, H=4, N=80, k=33)
+    out = o.sparse_attn(q, kv, idx, C.SCALE)
+    for b in range(2):
+        for t in range(2):
+            rows = torch.from_numpy(f(kv[b, idx[b, t]]))            # [k, 576]
+            qq = torch.from_numpy(f(q[b, t]))                        # [H, 576]
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                qq[None], rows[None], rows[None, :, :512], scale=C.SCALE)[0]
+            assert np.allclose(out[b, t], ref.numpy(), rtol=1e-12, atol=1e-13)
+
+
+def pin_attn_dense_masked(o):
+    """Sparse attention == dense softmax over all N positions with -inf outside the set."""
+    q, kv, idx = _attn_inputs(13, B=2, T=3, H=2, N=90, k=31)
+    idx[1, 2, 5:9] = -1
+    a = o.sparse_attn(q, kv, idx, C.SCALE)
+    d = o.sparse_attn(q, kv, idx, C.SCALE, dense_masked=True)
+    assert np.allclose(a, d, rtol=1e-12, atol=1e-13)
+
+
+def pin_attn_order_and_padding_invariance(o):
+    q, kv, idx = _attn_inputs(14)
+    base = o.sparse_attn(q, kv, idx, C.SCALE)
+    r = _rng(15)
+    shuffled = idx.copy()
+    for t in range(2):
+        shuffled[0, t] = r.permutation(shuffled[0, t])
+    assert np.allclose(o.sparse_attn(q, kv, shuffled, C.SCALE), base, rtol=1e-12, atol=1e-13)
+    padded = np.concatenate([idx, np.full((1, 2, 7), -1, np.int32)], axis=2)
+    assert np.allclose(o.sparse_attn(q, kv, padded, C.SCALE), base, rtol=1e-12, atol=1e-13)
+    # the output is a convex combination of the selected value rows
+    for t in range(2):
+        vals = f(kv[0, idx[0, t], :512])
+        assert np.all(base[0, t] <= vals.max(0) + 1e-12) and np.all(base[0, t] >= vals.min(0) - 1e-12)
+
+
+def pin_attn_empty_selection_is_zero(o):
+    q, kv, _ = _attn_inputs(16)
+    idx = np.full((1, 2, 4), -1, np.int32)
+    assert np.array_equal(o.sparse_attn(q, kv, idx, C.SCALE), np.zeros((1, 2, 3, 512)))
+
+
+# ----------------------------------------------------------------------------- group
+
+def pin_group_shares_one_index_list(o):
+    """Indexer + top-k once, then every layer attends over the same, unchanged list."""
+    w = C.scaled(C.WORKLOADS["tiny"], N=200, q_pos0=199, k=32, H=2, L=4)
+    iq, wt, ik, qs, kvs = C.host_group_inputs(w)
+    idx, outs = o.group_forward(iq, wt, ik, qs, kvs, w.q_pos0, w.k, C.SCALE)
+    sc = o.index_score(iq, wt, ik, w.q_pos0).astype(np.float32)
+    assert np.array_equal(idx, o.topk(sc, w.q_pos0, w.k))
+    for l in range(4):
+        assert np.array_equal(outs[l], o.sparse_attn(qs[l], kvs[l], idx, C.SCALE))
+    # reuse: with compute_indices off the caller's list is used unchanged
+    mine = np.sort(_rng(17).choice(w.N, size=(1, 1, w.k), replace=False), axis=-1).astype(np.int32)
+    idx2, outs2 = o.group_forward(iq, wt, ik, qs, kvs, w.q_pos0, w.k, C.SCALE,
+                                  compute_indices=False, idx_shared=mine.copy())
+    assert np.array_equal(idx2, mine)
+    assert np.array_equal(outs2[2], o.sparse_attn(qs[2], kvs[2], mine, C.SCALE))
+
+
+def pin_mtp_draft_rows_never_attended(o):
+    """MTP reuse: the step-1 query sits at the last target position, so the draft rows
+    appended after it are never selected, and steps 2.. reuse that list: changing the
+    draft rows changes no output."""
+    w = C.scaled(C.WORKLOADS["mtp"], B=2, N=150 + 3, q_pos0=149, k=40, H=2, L=1, steps=3)
+    iq, wt, ik, _, kvs = C.host_group_inputs(w)
+    kv = kvs[0].copy()
+    idx = None
+    outs_a, outs_b = [], []
+    kv_b = kv.copy()
+    kv_b[:, 150:, :] = bf(np.full((2, 3, 576), 8.0, np.float32))  # loud draft rows
+    ik_b = ik.copy()
+    ik_b[:, 150:, :] = bf(np.full((2, 3, 128), 8.0, np.float32))
+    for step in range(w.steps):
+        q = synth.normal_bf16(w.key(synth.KIND_Q, 0, 0, step), (w.B, 1, w.H, 576))
+        ia, oa = o.group_forward(iq, wt, ik, [q], [kv], w.q_pos0, w.k, C.SCALE,
+                                 compute_indices=(step == 0), idx_shared=idx)
+        ib, ob = o.group_forward(iq, wt, ik_b, [q], [kv_b], w.q_pos0, w.k, C.SCALE,
+                                 compute_indices=(step == 0), idx_shared=None if step == 0 else idx)
+        if step == 0:
+            idx = ia.copy()
+        assert np.array_equal(ia, idx) and np.array_equal(ib, idx)
+        assert np.all(idx < 150)
+        assert np.array_equal(oa[0], ob[0])
+
+
+ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]
