@@ -1,0 +1,140 @@
+/*
+ * dsa.h -- C ABI of libdsa: the DSA (DeepSeek-style Sparse Attention) hot path with
+ * IndexShare for one NVIDIA B200 (sm_100a).
+ *
+ * The path has three steps and a driver:
+ *   1. lightweight indexer score      I(t,s) = sum_h w[t,h] * ReLU(q[t,h] . k[s])
+ *   2. per-query top-k select         the k best-scoring visible tokens
+ *   3. sparse MLA attention           softmax attention over the selected compressed rows
+ *   4. IndexShare group driver        1 x (1+2), then L x (3) with the same index list
+ * Sources (page title, section): "GLM-5.2 1M architecture teardown" (clawlihai.cn),
+ * Cut 1: DSA (an indexer coarse-screens 2048 of the history tokens; full attention runs
+ * over those only; index_topk 2048, index_head_dim 128, index_n_heads 32), Cut 2:
+ * IndexShare (the indexer sits in the first of every 4 layers and its top-k list is used
+ * by all 4; index_topk_freq 4), Cut 3: MLA (a 512-wide compressed KV row per token);
+ * "GLM-5.2 MTP IndexShare inference" (4sapi.ai), Indexer Share and its use in the MTP
+ * layer (draft steps reuse the step-1 mask, so draft-token KV is never attended), KV
+ * Share (the MTP layer reads the target model's cache); "Le contexte d'un million de
+ * tokens" (glmmodel.cn), Attention sparse IndexShare and MTP avec IndexShare et KVShare.
+ * The pages print no formula for the indexer score or the attention; the forms above
+ * (and a 576-wide compressed row = 512 latent + 64 rope, value = first 512 entries) are
+ * the readings this library implements.
+ *
+ * Conventions for every entry point
+ *   - Tensors are caller-owned DEVICE pointers, dense row-major, in the layouts given.
+ *     bf16 tensors are passed as uint16_t bit patterns.  bf16 tensors and the score,
+ *     output and workspace buffers must be 16-byte aligned; float/int tensors 4-byte.
+ *   - Calls are asynchronous: work is enqueued on `stream` and the call returns.  The
+ *     library allocates no memory and keeps no per-call state; scratch memory is the
+ *     caller's `workspace` (size from dsa_workspace_size).
+ *   - Invalid arguments return an error before anything is enqueued.  DSA_ERR_CUDA
+ *     reports a launch failure (cudaGetLastError after the launch).
+ *   - Query t of a sequence sits at position q_pos0 + t and sees cached positions
+ *     s <= q_pos0 + t, s < N (causal mask).  For decode, q_pos0 = N - 1.
+ */
+#ifndef DSA_H
+#define DSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSA_OK = 0,
+    DSA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misaligned pointer          */
+    DSA_ERR_UNSUPPORTED = -2,  /* a shape the kernels do not implement                */
+    DSA_ERR_WORKSPACE = -3,    /* workspace missing or smaller than dsa_workspace_size */
+    DSA_ERR_CUDA = -4,         /* a CUDA launch or runtime call failed                 */
+    DSA_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up (see status word) */
+    DSA_ERR_DEVICE = -6        /* a kernel recorded a device-side error                */
+} dsa_status;
+
+/* Fixed sizes of the path (GLM-5.2 configuration as quoted on the pages). */
+#define DSA_INDEX_HEADS 32   /* index_n_heads                                          */
+#define DSA_INDEX_DIM 128    /* index_head_dim                                         */
+#define DSA_DQK 576          /* compressed row width: 512 latent + 64 rope             */
+#define DSA_DV 512           /* value width: the first 512 entries of the row          */
+#define DSA_MAX_TOPK 2048    /* index_topk                                             */
+#define DSA_MAX_LAYERS 8     /* layers per dsa_group_forward call                      */
+
+/* Human-readable name of a dsa_status value. */
+const char *dsa_status_string(int status);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int dsa_version(void);
+
+/*
+ * Bytes of workspace needed by dsa_topk, dsa_sparse_attn and dsa_group_forward for these
+ * sizes (the largest of the three; one workspace serves all calls of that size).
+ * B sequences, T queries per sequence, N cached rows, k top-k, H attention heads,
+ * L layers per group.  Returns 0 for invalid sizes.
+ */
+size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L);
+
+/*
+ * Step 1 -- indexer score.
+ *   q      [B, T, 32, 128]  bf16   indexer queries
+ *   w      [B, T, 32]       f32    per-query head weights
+ *   k      [B, N, 128]      bf16   index-key cache (one key per cached token)
+ *   scores [B, T, N]        f32    out: I(t,s) for every visible s; entries with
+ *                                  s > q_pos0 + t are unspecified
+ * Products are bf16 x bf16, accumulated in f32 on the tensor cores.
+ */
+dsa_status dsa_index_score(const uint16_t *q, const float *w, const uint16_t *k,
+                           int B, int T, int N, long long q_pos0, float *scores,
+                           cudaStream_t stream);
+
+/*
+ * Step 2 -- top-k select.
+ *   scores [B, T, N] f32 (only s <= q_pos0 + t is read)
+ *   idx    [B, T, k] i32 out: the selected token positions in ascending order; when
+ *                       fewer than k positions are visible all are kept and the rest
+ *                       of the row is -1.
+ * Order: higher score first; equal scores (-0 == +0) go to the lower token index; a NaN
+ * ranks below every number.  Deterministic and bit-exact.  1 <= k <= 2048.
+ */
+dsa_status dsa_topk(const float *scores, int B, int T, int N, long long q_pos0, int k,
+                    int32_t *idx, void *workspace, size_t workspace_bytes,
+                    cudaStream_t stream);
+
+/*
+ * Step 3 -- sparse MLA attention over the selected rows.
+ *   q    [B, T, H, 576] bf16   attention queries (absorbed form)
+ *   kv   [B, N, 576]    bf16   compressed cache; value = first 512 entries of a row
+ *   idx  [B, T, k]      i32    selected rows (entries < 0 are skipped; all must be < N)
+ *   out  [B, T, H, 512] f32    softmax_j(scale * q . kv[idx_j]) weighted sum of values;
+ *                              zero when a row selects nothing
+ * bf16 operands, f32 accumulation and softmax.  H in {16, 32, 48, 64}.
+ */
+dsa_status dsa_sparse_attn(const uint16_t *q, const uint16_t *kv, const int32_t *idx,
+                           int B, int T, int N, int H, int k, float scale, float *out,
+                           void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Step 4 -- one IndexShare group (also one MTP draft step).
+ *   iq, w, ik          indexer inputs as in dsa_index_score
+ *   q[l], kv[l], out[l] for l < L: HOST arrays of L device pointers, one per layer, with
+ *                       the layouts of dsa_sparse_attn
+ *   compute_indices     1: run the indexer and top-k and write idx_shared;
+ *                       0: use idx_shared as given (IndexShare layers 2..4 of a group,
+ *                          MTP draft steps 2..7); iq, w, ik may then be NULL
+ *   idx_shared [B,T,k]  the shared index list; never written when compute_indices = 0,
+ *                       and read unchanged by all L layers
+ * 1 <= L <= DSA_MAX_LAYERS.
+ */
+dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t *ik,
+                             const uint16_t *const *q, const uint16_t *const *kv, int L,
+                             int B, int T, int N, long long q_pos0, int H, int k, float scale,
+                             int compute_indices, int32_t *idx_shared, float *const *out,
+                             void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DSA_H */

@@ -1,0 +1,201 @@
+"""Python binding of libdsa (argument marshalling only).
+
+Every step of the DSA hot path runs in the CUDA kernels of ``libdsa.so``; this module
+checks tensor dtypes, shapes and devices, passes raw device pointers and the current
+CUDA stream through ctypes, and raises ``DsaError`` on a non-OK status.  PyTorch is used
+only for device memory and streams.  There is no fallback: if ``libdsa.so`` is missing
+or no CUDA device is present, the calls raise.
+
+Names and argument order follow the C ABI in ``include/dsa.h``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdsa.so")
+
+INDEX_HEADS = 32
+INDEX_DIM = 128
+DQK = 576
+DV = 512
+MAX_TOPK = 2048
+MAX_LAYERS = 8
+
+DSA_OK = 0
+STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3: "DSA_ERR_WORKSPACE",
+          -4: "DSA_ERR_CUDA", -5: "DSA_ERR_TIMEOUT", -6: "DSA_ERR_DEVICE"}
+
+# every symbol include/dsa.h declares
+EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_topk",
+           "dsa_sparse_attn", "dsa_group_forward")
+
+
+class DsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libdsa.so (built in-tree by ``python -m sparse_long_context_score_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is not built; run python -m sparse_long_context_score_b200.build")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, LL, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+        L.dsa_status_string.argtypes = [I]
+        L.dsa_status_string.restype = ctypes.c_char_p
+        L.dsa_version.argtypes = []
+        L.dsa_version.restype = I
+        L.dsa_workspace_size.argtypes = [I, I, I, I, I, I]
+        L.dsa_workspace_size.restype = S
+        L.dsa_index_score.argtypes = [P, P, P, I, I, I, LL, P, P]
+        L.dsa_topk.argtypes = [P, I, I, I, LL, I, P, P, S, P]
+        L.dsa_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, F, P, P, S, P]
+        L.dsa_group_forward.argtypes = [P, P, P, P, P, I, I, I, I, LL, I, I, F, I, P, P, P, S, P]
+        for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward"):
+            getattr(L, f).restype = I
+        _lib = L
+    return _lib
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream) -> int:
+    torch = _torch()
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t, dtypes, name, shape=None):
+    torch = _torch()
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (there is no CPU path)")
+    if t.dtype not in dtypes:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    return t.data_ptr()
+
+
+def _bf16_types():
+    torch = _torch()
+    return (torch.bfloat16, torch.int16, torch.uint16)
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != DSA_OK:
+        raise DsaError(rc, where)
+
+
+def dsa_workspace_size(B: int, T: int, N: int, k: int, H: int, L: int) -> int:
+    return int(lib().dsa_workspace_size(B, T, N, k, H, L))
+
+
+def workspace(B: int, T: int, N: int, k: int, H: int, L: int, device=None):
+    """Allocate a workspace tensor of dsa_workspace_size bytes (torch allocation)."""
+    torch = _torch()
+    n = dsa_workspace_size(B, T, N, k, H, L)
+    if n == 0:
+        raise ValueError("invalid sizes for dsa_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def dsa_index_score(q, w, k, q_pos0: int, scores=None, stream=None):
+    """q [B,T,32,128] bf16, w [B,T,32] f32, k [B,N,128] bf16 -> scores [B,T,N] f32."""
+    torch = _torch()
+    B, T = q.shape[0], q.shape[1]
+    N = k.shape[1]
+    if scores is None:
+        scores = torch.empty((B, T, N), dtype=torch.float32, device=q.device)
+    rc = lib().dsa_index_score(_ptr(q, _bf16_types(), "q", (B, T, INDEX_HEADS, INDEX_DIM)),
+                               _ptr(w, (torch.float32,), "w", (B, T, INDEX_HEADS)),
+                               _ptr(k, _bf16_types(), "k", (B, N, INDEX_DIM)), B, T, N, int(q_pos0),
+                               _ptr(scores, (torch.float32,), "scores", (B, T, N)), _stream(stream))
+    _check(rc, "dsa_index_score")
+    return scores
+
+
+def dsa_topk(scores, q_pos0: int, k: int, idx=None, ws=None, stream=None):
+    """scores [B,T,N] f32 -> idx [B,T,k] int32 (ascending, -1 padding)."""
+    torch = _torch()
+    B, T, N = scores.shape
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=scores.device)
+    if ws is None:
+        ws = workspace(B, T, N, k, 16, 1, scores.device)
+    rc = lib().dsa_topk(_ptr(scores, (torch.float32,), "scores"), B, T, N, int(q_pos0), int(k),
+                        _ptr(idx, (torch.int32,), "idx", (B, T, k)), _ptr(ws, (torch.uint8,), "workspace"),
+                        ws.numel(), _stream(stream))
+    _check(rc, "dsa_topk")
+    return idx
+
+
+def dsa_sparse_attn(q, kv, idx, scale: float, out=None, ws=None, stream=None):
+    """q [B,T,H,576] bf16, kv [B,N,576] bf16, idx [B,T,k] int32 -> out [B,T,H,512] f32."""
+    torch = _torch()
+    B, T, H, _ = q.shape
+    N = kv.shape[1]
+    k = idx.shape[2]
+    if out is None:
+        out = torch.empty((B, T, H, DV), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(B, T, N, k, H, 1, q.device)
+    rc = lib().dsa_sparse_attn(_ptr(q, _bf16_types(), "q", (B, T, H, DQK)),
+                               _ptr(kv, _bf16_types(), "kv", (B, N, DQK)),
+                               _ptr(idx, (torch.int32,), "idx", (B, T, k)), B, T, N, H, k, float(scale),
+                               _ptr(out, (torch.float32,), "out", (B, T, H, DV)),
+                               _ptr(ws, (torch.uint8,), "workspace"), ws.numel(), _stream(stream))
+    _check(rc, "dsa_sparse_attn")
+    return out
+
+
+def dsa_group_forward(iq, w, ik, qs, kvs, q_pos0: int, k: int, scale: float, compute_indices: bool = True,
+                      idx_shared=None, outs=None, ws=None, stream=None):
+    """One IndexShare group (or MTP draft step): indexer + top-k once when
+    compute_indices, then sparse attention for each of the L layers with the same index
+    list.  Returns (idx_shared, [out_l])."""
+    torch = _torch()
+    L = len(qs)
+    if L < 1 or L > MAX_LAYERS or len(kvs) != L:
+        raise ValueError("need 1..8 layers with one q and one kv each")
+    B, T, H, _ = qs[0].shape
+    N = kvs[0].shape[1]
+    dev = qs[0].device
+    if idx_shared is None:
+        if not compute_indices:
+            raise ValueError("idx_shared is required when compute_indices is False")
+        idx_shared = torch.empty((B, T, k), dtype=torch.int32, device=dev)
+    if outs is None:
+        outs = [torch.empty((B, T, H, DV), dtype=torch.float32, device=dev) for _ in range(L)]
+    if ws is None:
+        ws = workspace(B, T, N, k, H, L, dev)
+    qp = (ctypes.c_void_p * L)(*[_ptr(x, _bf16_types(), "q[l]", (B, T, H, DQK)) for x in qs])
+    kp = (ctypes.c_void_p * L)(*[_ptr(x, _bf16_types(), "kv[l]", (B, N, DQK)) for x in kvs])
+    op = (ctypes.c_void_p * L)(*[_ptr(x, (torch.float32,), "out[l]", (B, T, H, DV)) for x in outs])
+    ci = bool(compute_indices)
+    rc = lib().dsa_group_forward(
+        _ptr(iq, _bf16_types(), "iq", (B, T, INDEX_HEADS, INDEX_DIM)) if ci else None,
+        _ptr(w, (torch.float32,), "w", (B, T, INDEX_HEADS)) if ci else None,
+        _ptr(ik, _bf16_types(), "ik", (B, N, INDEX_DIM)) if ci else None,
+        ctypes.addressof(qp), ctypes.addressof(kp), L, B, T, N, int(q_pos0), H, int(k), float(scale), int(ci),
+        _ptr(idx_shared, (torch.int32,), "idx_shared", (B, T, k)), ctypes.addressof(op),
+        _ptr(ws, (torch.uint8,), "workspace"), ws.numel(), _stream(stream))
+    _check(rc, "dsa_group_forward")
+    return idx_shared, outs

@@ -1,0 +1,56 @@
+// dsa_internal.h -- constants and launch entry points shared by the libdsa sources.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace dsa {
+
+constexpr int kIndexHeads = 32;   // index_n_heads
+constexpr int kIndexDim = 128;    // index_head_dim
+constexpr int kDqk = 576;         // compressed row: 512 latent + 64 rope
+constexpr int kDv = 512;          // value = first 512 entries
+constexpr int kMaxTopk = 2048;    // index_topk
+constexpr int kMaxLayers = 8;
+
+// top-k: first radix digit = the top 12 bits of the order key
+constexpr int kHistBits = 12;
+constexpr int kHistBins = 1 << kHistBits;
+constexpr int kHistShift = 32 - kHistBits;
+constexpr int kTopkChunk = 8192;       // scores per CTA in the scan kernels
+constexpr int kCandCap = 8192;         // candidates kept per row for the in-SMEM resolve
+constexpr int kRowStateWords = 16;
+
+struct TopkWorkspace {
+  uint32_t* hist;        // [rows][kHistBins]
+  uint32_t* row_state;   // [rows][kRowStateWords]
+  uint32_t* chunk_sel;   // [rows][nchunks]  selected threshold-bin candidates per chunk
+  uint32_t* chunk_above; // [rows][nchunks]  elements above the threshold bin per chunk
+  uint32_t* chunk_off;   // [rows][nchunks]  output offset of each chunk
+  uint64_t* cand;        // [rows][kCandCap] composite keys of threshold-bin elements
+  size_t zero_bytes;     // bytes from hist that must be zero before a select
+};
+
+size_t topk_workspace_bytes(long long rows, int N);
+TopkWorkspace topk_workspace(void* base, long long rows, int N);
+
+struct AttnLayers {
+  const uint16_t* q[kMaxLayers];
+  const uint16_t* kv[kMaxLayers];
+  float* out[kMaxLayers];
+};
+
+int attn_num_splits(long long rows, int L, int k);
+size_t attn_workspace_bytes(long long rows, int L, int H, int k);
+
+cudaError_t launch_index_score(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
+                               long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream);
+
+cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
+                        const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream);
+
+cudaError_t launch_sparse_attn(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
+                               int k, float scale, void* ws, cudaStream_t stream);
+
+}  // namespace dsa

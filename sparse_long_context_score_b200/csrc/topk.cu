@@ -1,0 +1,391 @@
+// topk.cu -- per-query top-k select over the indexer scores.
+//
+// "GLM-5.2 1M architecture teardown", Cut 1: DSA -- keep the index_topk (2048) best
+// history tokens per query; Cut 2: IndexShare -- the top-k list is computed once per
+// group of 4 layers.
+//
+// Order: higher score first, ties to the lower token index, a NaN below every number,
+// -0 == +0.  Every visible element s gets the 64-bit composite
+//     C(s) = order_key(score[s]) << 32 | (0xFFFFFFFF - s)
+// which is distinct per element and orders exactly as required, so the selection is
+// "the k largest composites" and the answer is unique: bit-exact and deterministic.
+//
+// Radix select over C, most significant digit first:
+//   1. histogram of the top 12 bits (4096 bins) per row -- built here, or folded into
+//      the indexer epilogue;
+//   2. select kernel, grid (rows, chunks of 8192): every CTA finds the threshold bin b*
+//      from the histogram, counts its elements above b*, and appends the elements of
+//      bin b* to a per-row candidate list; the last CTA of a row (atomic ticket, no
+//      waiting) resolves the remaining 52 bits by 8-bit radix passes over the
+//      candidates in shared memory (or, if the bin holds more than kCandCap elements,
+//      over the row itself), giving the exact threshold composite, and turns per-chunk
+//      counts into output offsets;
+//   3. compact kernel, grid (rows, chunks): every element with C(s) >= threshold is
+//      written at its chunk offset plus its warp-ballot rank, so the output comes out
+//      in ascending token order.
+// When a row has no more than k visible positions all of them are kept (0..V-1) and the
+// row is padded with -1.
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+
+namespace dsa {
+
+namespace {
+
+constexpr int kHistThreads = 256;
+constexpr int kSelThreads = 512;
+constexpr int kCmpThreads = 256;
+constexpr uint64_t kLow52 = (1ull << 52) - 1;
+
+// row_state words
+constexpr int RS_CAND = 0;    // candidates appended (atomic)
+constexpr int RS_TICKET = 1;  // select CTAs finished (atomic)
+constexpr int RS_BSTAR = 2;
+constexpr int RS_ABOVE = 3;
+constexpr int RS_THR_LO = 4;
+constexpr int RS_THR_HI = 5;
+
+__device__ __forceinline__ uint64_t composite(uint32_t key, uint32_t s) {
+  return ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - s);
+}
+
+__device__ __forceinline__ int row_t(int row, int T) { return row % T; }
+
+__global__ void __launch_bounds__(kHistThreads)
+topk_hist_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, uint32_t* __restrict__ hist) {
+  const int row = blockIdx.x;
+  const long long V = visible_count(N, q_pos0, row_t(row, T));
+  const long long s0 = (long long)blockIdx.y * kTopkChunk;
+  if (s0 >= V) return;
+  const long long s1 = min(s0 + (long long)kTopkChunk, V);
+  __shared__ uint32_t sh[kHistBins];
+  for (int i = threadIdx.x; i < kHistBins; i += kHistThreads) sh[i] = 0;
+  __syncthreads();
+  const float* sr = scores + (size_t)row * N;
+  for (long long s = s0 + threadIdx.x; s < s1; s += kHistThreads) atomicAdd(&sh[order_key(sr[s]) >> kHistShift], 1u);
+  __syncthreads();
+  uint32_t* gh = hist + (size_t)row * kHistBins;
+  for (int i = threadIdx.x; i < kHistBins; i += kHistThreads)
+    if (sh[i]) atomicAdd(&gh[i], sh[i]);
+}
+
+// Block-wide exclusive scan of one value per thread (kSelThreads threads).
+__device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t wv = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0u;
+    uint32_t z = wv;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      uint32_t y = __shfl_up_sync(0xFFFFFFFFu, z, o);
+      if (lane >= o) z += y;
+    }
+    if (lane < (int)(blockDim.x >> 5)) s_warp[lane] = z - wv;
+    if (lane == 31) *total = z;
+  }
+  __syncthreads();
+  const uint32_t r = s_warp[warp] + x - v;
+  __syncthreads();
+  return r;
+}
+
+struct SelectSmem {
+  uint32_t radix[256];
+  uint32_t warp_tmp[32];
+  uint32_t total;
+  uint32_t bstar, above, remaining, digit, digit_count, is_last;
+  unsigned long long prefix;
+  uint64_t cand[kCandCap];
+};
+
+// Radix passes over the low 52 bits of the threshold-bin composites.  `get(i, c)` yields
+// element i's composite (returns false if element i is not in the threshold bin).
+template <class Get>
+__device__ uint64_t resolve_threshold(SelectSmem& sm, long long count, uint32_t remaining, Get get) {
+  unsigned long long prefix = 0;
+  int shift = 52;
+  while (true) {
+    const int width = shift >= 8 ? 8 : shift;
+    shift -= width;
+    const uint32_t mask = (1u << width) - 1u;
+    for (int i = threadIdx.x; i < 256; i += kSelThreads) sm.radix[i] = 0;
+    __syncthreads();
+    const int hi_shift = shift + width;
+    for (long long i = threadIdx.x; i < count; i += kSelThreads) {
+      uint64_t c;
+      if (!get(i, c)) continue;
+      c &= kLow52;
+      if (hi_shift >= 52 || (c >> hi_shift) == (prefix >> hi_shift))
+        atomicAdd(&sm.radix[(uint32_t)(c >> shift) & mask], 1u);
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      uint32_t cum = 0;
+      int d = (int)mask;
+      for (; d > 0; --d) {
+        if (cum + sm.radix[d] >= remaining) break;
+        cum += sm.radix[d];
+      }
+      sm.digit = (uint32_t)d;
+      sm.digit_count = sm.radix[d];
+      sm.remaining = remaining - cum;
+    }
+    __syncthreads();
+    remaining = sm.remaining;
+    prefix |= (unsigned long long)sm.digit << shift;
+    const bool done = (sm.digit_count == remaining) || shift == 0;
+    __syncthreads();
+    if (done) break;
+  }
+  return prefix;
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, int k, TopkWorkspace ws,
+                   int32_t* __restrict__ idx_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
+  const int row = blockIdx.x;
+  const int chunk = blockIdx.y;
+  const int nchunks = gridDim.y;
+  const long long V = visible_count(N, q_pos0, row_t(row, T));
+  uint32_t* state = ws.row_state + (size_t)row * kRowStateWords;
+
+  if (V <= k) {
+    // every visible position is kept; pad the rest of the row
+    if (chunk == 0)
+      for (long long j = V + threadIdx.x; j < k; j += kSelThreads) idx_out[(size_t)row * k + j] = -1;
+    return;
+  }
+
+  // 1. threshold bin b*: the bin where the count from the top reaches k
+  const uint32_t* gh = ws.hist + (size_t)row * kHistBins;
+  constexpr int kPer = kHistBins / kSelThreads;  // 8 bins per thread
+  const int rt = kSelThreads - 1 - threadIdx.x;   // thread 0 owns the highest bins
+  uint32_t local[kPer];
+  uint32_t lsum = 0;
+#pragma unroll
+  for (int i = 0; i < kPer; ++i) {
+    local[i] = __ldcg(&gh[rt * kPer + i]);
+    lsum += local[i];
+  }
+  if (threadIdx.x == 0) {
+    sm.bstar = 0;
+    sm.above = 0;
+  }
+  // suffix sums over threads ordered from the top bin down
+  const uint32_t above_mine = block_excl_scan(lsum, sm.warp_tmp, &sm.total);
+  {
+    uint32_t run = above_mine;
+    for (int i = kPer - 1; i >= 0; --i) {
+      if (run < (uint32_t)k && run + local[i] >= (uint32_t)k) {
+        sm.bstar = (uint32_t)(rt * kPer + i);
+        sm.above = run;
+      }
+      run += local[i];
+    }
+  }
+  __syncthreads();
+  const uint32_t bstar = sm.bstar;
+  const uint32_t above = sm.above;
+  const uint32_t bcount = __ldcg(&gh[bstar]);
+  const bool use_cand = bcount <= (uint32_t)kCandCap;
+
+  // 2. scan this chunk
+  const float* sr = scores + (size_t)row * N;
+  const long long s0 = (long long)chunk * kTopkChunk;
+  const long long s1 = min(s0 + (long long)kTopkChunk, V);
+  uint64_t* cand = ws.cand + (size_t)row * kCandCap;
+  uint32_t n_above = 0;
+  for (long long s = s0 + threadIdx.x; s < s1; s += kSelThreads) {
+    const uint32_t key = order_key(sr[s]);
+    const uint32_t bin = key >> kHistShift;
+    if (bin > bstar) ++n_above;
+    else if (bin == bstar && use_cand) {
+      const uint32_t pos = atomicAdd(&state[RS_CAND], 1u);
+      if (pos < (uint32_t)kCandCap) cand[pos] = composite(key, (uint32_t)s);
+    }
+  }
+  (void)block_excl_scan(n_above, sm.warp_tmp, &sm.total);
+  if (threadIdx.x == 0) ws.chunk_above[(size_t)row * nchunks + chunk] = sm.total;
+
+  // 3. the last CTA of the row resolves the threshold
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) sm.is_last = atomicAdd(&state[RS_TICKET], 1u) == (uint32_t)(nchunks - 1);
+  __syncthreads();
+  if (!sm.is_last) return;
+  __threadfence();
+
+  const uint32_t remaining = (uint32_t)k - above;  // 1 <= remaining <= bcount
+  uint64_t thr52;
+  if (use_cand) {
+    for (long long i = threadIdx.x; i < bcount; i += kSelThreads) sm.cand[i] = __ldcg(&cand[i]);
+    __syncthreads();
+    thr52 = resolve_threshold(sm, bcount, remaining, [&](long long i, uint64_t& c) {
+      c = sm.cand[i];
+      return true;
+    });
+  } else {
+    thr52 = resolve_threshold(sm, V, remaining, [&](long long s, uint64_t& c) {
+      const uint32_t key = order_key(sr[s]);
+      if ((key >> kHistShift) != bstar) return false;
+      c = composite(key, (uint32_t)s);
+      return true;
+    });
+  }
+  const uint64_t thr = ((uint64_t)bstar << 52) | thr52;
+
+  // 4. threshold-bin elements selected per chunk
+  uint32_t* csel = ws.chunk_sel + (size_t)row * nchunks;
+  if (use_cand) {
+    for (long long i = threadIdx.x; i < bcount; i += kSelThreads) {
+      const uint64_t c = sm.cand[i];
+      if (c >= thr) atomicAdd(&csel[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+    }
+  } else {
+    for (long long s = threadIdx.x; s < V; s += kSelThreads) {
+      const uint32_t key = order_key(sr[s]);
+      if ((key >> kHistShift) == bstar && composite(key, (uint32_t)s) >= thr) atomicAdd(&csel[s / kTopkChunk], 1u);
+    }
+  }
+  __threadfence();
+  __syncthreads();
+
+  // 5. output offset of every chunk
+  uint32_t carry = 0;
+  for (int c0 = 0; c0 < nchunks; c0 += kSelThreads) {
+    const int c = c0 + threadIdx.x;
+    const uint32_t v = c < nchunks ? __ldcg(&ws.chunk_above[(size_t)row * nchunks + c]) + __ldcg(&csel[c]) : 0u;
+    const uint32_t off = block_excl_scan(v, sm.warp_tmp, &sm.total);
+    if (c < nchunks) ws.chunk_off[(size_t)row * nchunks + c] = carry + off;
+    carry += sm.total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    state[RS_THR_LO] = (uint32_t)thr;
+    state[RS_THR_HI] = (uint32_t)(thr >> 32);
+    state[RS_BSTAR] = bstar;
+    state[RS_ABOVE] = above;
+  }
+}
+
+__global__ void __launch_bounds__(kCmpThreads)
+topk_compact_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, int k, TopkWorkspace ws,
+                    int32_t* __restrict__ idx_out) {
+  const int row = blockIdx.x;
+  const int chunk = blockIdx.y;
+  const int nchunks = gridDim.y;
+  const long long V = visible_count(N, q_pos0, row_t(row, T));
+  const long long s0 = (long long)chunk * kTopkChunk;
+  if (s0 >= V) return;
+  const long long s1 = min(s0 + (long long)kTopkChunk, V);
+  const bool take_all = V <= k;
+  uint64_t thr = 0;
+  long long base = s0;
+  if (!take_all) {
+    const uint32_t* state = ws.row_state + (size_t)row * kRowStateWords;
+    thr = ((uint64_t)__ldcg(&state[RS_THR_HI]) << 32) | __ldcg(&state[RS_THR_LO]);
+    base = __ldcg(&ws.chunk_off[(size_t)row * nchunks + chunk]);
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kSeg = kTopkChunk / (kCmpThreads / 32);
+  const long long g0 = s0 + (long long)warp * kSeg;
+  const long long g1 = min(g0 + kSeg, s1);
+  const float* sr = scores + (size_t)row * N;
+  __shared__ uint32_t s_cnt[kCmpThreads / 32];
+
+  uint32_t cnt = 0;
+  for (long long s = g0; s < g1; s += 32) {
+    const long long e = s + lane;
+    bool sel = false;
+    if (e < g1) sel = take_all || composite(order_key(sr[e]), (uint32_t)e) >= thr;
+    cnt += __popc(__ballot_sync(0xFFFFFFFFu, sel));
+  }
+  if (lane == 0) s_cnt[warp] = cnt;
+  __syncthreads();
+  long long off = base;
+  for (int i = 0; i < warp; ++i) off += s_cnt[i];
+  int32_t* out = idx_out + (size_t)row * k;
+  for (long long s = g0; s < g1; s += 32) {
+    const long long e = s + lane;
+    bool sel = false;
+    if (e < g1) sel = take_all || composite(order_key(sr[e]), (uint32_t)e) >= thr;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, sel);
+    const long long pos = off + __popc(m & ((1u << lane) - 1u));
+    if (sel && pos < k) out[pos] = (int32_t)e;
+    off += __popc(m);
+  }
+}
+
+}  // namespace
+
+size_t topk_workspace_bytes(long long rows, int N) {
+  const long long nchunks = ((long long)N + kTopkChunk - 1) / kTopkChunk;
+  size_t b = 0;
+  b += (size_t)rows * kHistBins * 4;
+  b += (size_t)rows * kRowStateWords * 4;
+  b += (size_t)rows * nchunks * 4 * 3;
+  b = (b + 255) & ~(size_t)255;
+  b += (size_t)rows * kCandCap * 8;
+  return (b + 255) & ~(size_t)255;
+}
+
+TopkWorkspace topk_workspace(void* base, long long rows, int N) {
+  const long long nchunks = ((long long)N + kTopkChunk - 1) / kTopkChunk;
+  TopkWorkspace w;
+  unsigned char* p = static_cast<unsigned char*>(base);
+  w.hist = reinterpret_cast<uint32_t*>(p);
+  p += (size_t)rows * kHistBins * 4;
+  w.row_state = reinterpret_cast<uint32_t*>(p);
+  p += (size_t)rows * kRowStateWords * 4;
+  w.chunk_sel = reinterpret_cast<uint32_t*>(p);
+  p += (size_t)rows * nchunks * 4;
+  w.zero_bytes = (size_t)(p - static_cast<unsigned char*>(base));
+  w.chunk_above = reinterpret_cast<uint32_t*>(p);
+  p += (size_t)rows * nchunks * 4;
+  w.chunk_off = reinterpret_cast<uint32_t*>(p);
+  p += (size_t)rows * nchunks * 4;
+  size_t off = (size_t)(p - static_cast<unsigned char*>(base));
+  off = (off + 255) & ~(size_t)255;
+  w.cand = reinterpret_cast<uint64_t*>(static_cast<unsigned char*>(base) + off);
+  return w;
+}
+
+cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
+                        const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream) {
+  const long long rows = (long long)B * T;
+  const long long vmax = visible_count(N, q_pos0, T - 1);
+  const long long nchunks_all = ((long long)N + kTopkChunk - 1) / kTopkChunk;
+  const long long nchunks_vis = (vmax + kTopkChunk - 1) / kTopkChunk;
+  (void)nchunks_vis;
+  cudaError_t e;
+  if (!hist_ready) {
+    e = cudaMemsetAsync(ws.hist, 0, ws.zero_bytes, stream);
+    if (e != cudaSuccess) return e;
+    topk_hist_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kHistThreads, 0, stream>>>(scores, T, N, q_pos0,
+                                                                                                ws.hist);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  // the select kernel needs every chunk of the row to take a ticket, so it runs over all
+  // chunks of N (chunks past the visible range count nothing)
+  const size_t smem = sizeof(SelectSmem);
+  e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  topk_select_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kSelThreads, smem, stream>>>(scores, T, N, q_pos0,
+                                                                                                  k, ws, idx);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  topk_compact_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kCmpThreads, 0, stream>>>(scores, T, N, q_pos0,
+                                                                                                k, ws, idx);
+  return cudaGetLastError();
+}
+
+}  // namespace dsa

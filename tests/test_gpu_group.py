@@ -1,0 +1,89 @@
+"""Parity of the IndexShare group driver (and the MTP reuse) against the CPU oracle."""
+import numpy as np
+import pytest
+
+import synth
+from gpu_util import assert_close, dev, dev_bf16, host
+from synth import configs as C
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dsa():
+    import sparse_long_context_score_b200 as m
+    from sparse_long_context_score_b200 import build
+    build.build()
+    m.lib()
+    return m
+
+
+def run_group(dsa, w, group=0, step=0):
+    iq, wt, ik, qs, kvs = C.host_group_inputs(w, group, step)
+    idx, outs = dsa.dsa_group_forward(dev_bf16(iq), dev(wt), dev_bf16(ik), [dev_bf16(x) for x in qs],
+                                      [dev_bf16(x) for x in kvs], w.q_pos0, w.k, C.SCALE)
+    return (iq, wt, ik, qs, kvs), host(idx), [host(o) for o in outs]
+
+
+@pytest.mark.parametrize("name,kw", [
+    ("tiny", {}),
+    ("decode128k", dict(B=2, N=20000, q_pos0=19999)),
+    ("prefill", dict(T=48, N=6000, q_pos0=6000 - 48)),
+    ("decode1m", dict(B=1, N=9000, q_pos0=8999, groups=1)),
+])
+def test_group_matches_oracle(dsa, orc, name, kw):
+    w = C.scaled(C.WORKLOADS[name], **kw)
+    (iq, wt, ik, qs, kvs), idx, outs = run_group(dsa, w)
+    ridx, routs = orc.group_forward(iq, wt, ik, qs, kvs, w.q_pos0, w.k, C.SCALE)
+    assert np.array_equal(idx, ridx)
+    for l in range(w.L):
+        assert_close(outs[l], routs[l], f"{name} layer {l}")
+    for t in range(w.T):
+        assert np.all(idx[:, t][idx[:, t] >= 0] <= w.q_pos0 + t)
+
+
+def test_index_list_is_shared_and_unchanged(dsa):
+    """compute_indices=0 reads idx_shared without writing it, and gives the same outputs
+    as the computing call for every layer."""
+    import torch
+    w = C.scaled(C.WORKLOADS["decode128k"], B=2, N=5000, q_pos0=4999)
+    iq, wt, ik, qs, kvs = C.host_group_inputs(w)
+    dq, dkv = [dev_bf16(x) for x in qs], [dev_bf16(x) for x in kvs]
+    idx, outs = dsa.dsa_group_forward(dev_bf16(iq), dev(wt), dev_bf16(ik), dq, dkv, w.q_pos0, w.k, C.SCALE)
+    before = idx.clone()
+    _, outs2 = dsa.dsa_group_forward(None, None, None, dq, dkv, w.q_pos0, w.k, C.SCALE, compute_indices=False,
+                                     idx_shared=idx)
+    torch.cuda.synchronize()
+    assert torch.equal(before, idx)
+    for a, b in zip(outs, outs2):
+        assert torch.equal(a, b)
+
+
+def test_mtp_draft_steps_reuse_step1_indices(dsa, orc):
+    """MTP drafting: step 1 runs the indexer over the target cache (the query sits at the
+    last target position, so the appended draft rows are invisible); steps 2.. reuse the
+    step-1 list unchanged, with a new query each step, on the same target cache."""
+    import torch
+    w = C.scaled(C.WORKLOADS["mtp"], B=3, N=4000 + 7, q_pos0=3999, k=256, steps=7)
+    iq, wt, ik, _, kvs = C.host_group_inputs(w)
+    kv = kvs[0]
+    dkv = dev_bf16(kv)
+    idx = None
+    for step in range(w.steps):
+        q = synth.normal_bf16(w.key(synth.KIND_Q, 0, 0, step), (w.B, 1, w.H, 576))
+        if step == 0:
+            didx, outs = dsa.dsa_group_forward(dev_bf16(iq), dev(wt), dev_bf16(ik), [dev_bf16(q)], [dkv], w.q_pos0,
+                                               w.k, C.SCALE)
+            idx = host(didx)
+            ridx, routs = orc.group_forward(iq, wt, ik, [q], [kv], w.q_pos0, w.k, C.SCALE)
+            assert np.array_equal(idx, ridx)
+            saved = didx.clone()
+        else:
+            _, outs = dsa.dsa_group_forward(None, None, None, [dev_bf16(q)], [dkv], w.q_pos0, w.k, C.SCALE,
+                                            compute_indices=False, idx_shared=didx)
+            _, routs = orc.group_forward(iq, wt, ik, [q], [kv], w.q_pos0, w.k, C.SCALE, compute_indices=False,
+                                         idx_shared=idx)
+            torch.cuda.synchronize()
+            assert torch.equal(didx, saved)
+        assert np.all(idx < 4000)
+        assert_close(host(outs[0]), routs[0], f"mtp step {step + 1}")
