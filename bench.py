@@ -1,0 +1,343 @@
+"""Benchmark of the DSA IndexShare group decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload decode128k]
+    python bench.py --impl reference ...        # the CPU oracle, timed on a bounded sample
+
+One step = one pass of the whole hot path over one batch: the indexer over the index-key
+cache, the top-k select, and sparse MLA attention for the 4 layers of the group (all
+IndexShare groups of the workload in sequence).  Inputs are seeded synthetic tensors
+generated in HBM before timing; the step is captured once in a CUDA graph and replayed.
+L2 is flushed (a 512 MiB write) before every timed step and the step alone is timed with
+CUDA events on the launching stream.  Under torchrun every rank runs its own batch
+(weak scaling, no data-path collective) and rank 0 reports the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+INDEXER_BYTES_PER_TOKEN = 128 * 2 + 4          # index key read + score write
+INDEXER_BYTES_PER_QUERY = 32 * 128 * 2 + 32 * 4  # indexer query + head weights
+ROW_BYTES = 576 * 2                             # one gathered compressed row
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--workload", default="decode128k")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--cpu-sample", type=int, default=2, help="sequences in the CPU-oracle sample")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def algorithmic(w):
+    """Algorithmic HBM bytes of one step, and of one indexer launch."""
+    idx_launch = w.B * w.T * INDEXER_BYTES_PER_QUERY + w.B * w.T * w.N * 4 + w.B * w.N * 128 * 2
+    attn = w.B * w.T * w.L * (w.k * ROW_BYTES + w.H * 576 * 2 + w.H * 512 * 4)
+    return w.groups * (idx_launch + attn + w.B * w.T * w.k * 4), idx_launch
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            m = json.load(fh)
+        return float(m["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def profiled_traffic(kernel_src: str, workload: str):
+    """Per-launch DRAM bytes of the indexer from the committed ncu summary, if it was taken
+    on the current kernel source; None otherwise."""
+    path = os.path.join(ROOT, "profiles", f"indexer_{workload}.md")
+    src = os.path.join(ROOT, "sparse_long_context_score_b200", "csrc", kernel_src)
+    try:
+        text = open(path).read()
+        digest = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        m = re.search(r"traffic_bytes_per_launch:\s*(\d+)\s*\(source sha256 ([0-9a-f]{16})\)", text)
+        if m and m.group(2) == digest:
+            return int(m.group(1))
+    except OSError:
+        pass
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.lines = []
+        if self.proc is not None:
+            time.sleep(0.15)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        rows = []
+        for l in self.lines:
+            parts = [x.strip() for x in l.split(",")]
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[2:]))
+            except (ValueError, IndexError):
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        sms = sorted(r[0] for r in rows)
+        return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": rows[0][1], "reasons": reasons, "samples": len(rows)}
+
+
+def make_inputs(w, device, rank):
+    import torch
+    import synth
+    import synth.device as sd
+    bf = torch.bfloat16
+    groups = []
+    for g in range(w.groups):
+        ik = torch.empty(w.B, w.N, 128, dtype=bf, device=device)
+        sd.int17_bf16(ik, w.key(synth.KIND_IK, g) ^ rank)
+        kvs = []
+        for l in range(w.L):
+            kv = torch.empty(w.B, w.N, 576, dtype=bf, device=device)
+            sd.normal_bf16(kv, w.key(synth.KIND_KV, g, l) ^ rank)
+            kvs.append(kv)
+        iq = torch.empty(w.B, w.T, 32, 128, dtype=bf, device=device)
+        sd.int17_bf16(iq, w.key(synth.KIND_IQ, g) ^ rank)
+        wt = torch.empty(w.B, w.T, 32, dtype=torch.float32, device=device)
+        sd.pow2_f32(wt, w.key(synth.KIND_W, g) ^ rank)
+        qs = []
+        for l in range(w.L):
+            q = torch.empty(w.B, w.T, w.H, 576, dtype=bf, device=device)
+            sd.normal_bf16(q, w.key(synth.KIND_Q, g, l) ^ rank)
+            qs.append(q)
+        idx = torch.empty(w.B, w.T, w.k, dtype=torch.int32, device=device)
+        outs = [torch.empty(w.B, w.T, w.H, 512, dtype=torch.float32, device=device) for _ in range(w.L)]
+        groups.append(dict(ik=ik, kvs=kvs, iq=iq, wt=wt, qs=qs, idx=idx, outs=outs))
+    return groups
+
+
+def run_ours(args, rank, world, device):
+    import torch
+    import sparse_long_context_score_b200 as dsa
+    from synth import configs as C
+
+    w = C.WORKLOADS[args.workload]
+    torch.cuda.set_device(device)
+    dsa.lib()
+    groups = make_inputs(w, device, rank)
+    ws = dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, device)
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+
+    def step():
+        for g in groups:
+            dsa.dsa_group_forward(g["iq"], g["wt"], g["ik"], g["qs"], g["kvs"], w.q_pos0, w.k, C.SCALE,
+                                  idx_shared=g["idx"], outs=g["outs"], ws=ws, stream=stream)
+
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        step()  # eager once (sets kernel attributes) before capture
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    torch.cuda.synchronize()
+
+    def timed(fn, K, W):
+        with torch.cuda.stream(stream):
+            for _ in range(W):
+                flush.zero_()
+                fn()
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+        with torch.cuda.stream(stream):
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        times = timed(graph.replay, args.steps, args.warmup)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    step_ms = sum(times) / len(times)
+
+    # the dominant kernel alone: the indexer over the first group's cache, same launch shape
+    g0 = groups[0]
+    scores = torch.empty(w.B, w.T, w.N, dtype=torch.float32, device=device)
+    idx_times = timed(lambda: dsa.dsa_index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores,
+                                                  stream=stream), args.steps, args.warmup)
+    idx_ms = sum(idx_times) / len(idx_times)
+
+    # end to end through the public API with host buffers: per step, the step's query-side
+    # inputs go host -> device from pinned memory and the outputs come back
+    pinned_in = [[t.cpu().pin_memory() for t in [g["iq"], g["wt"], *g["qs"]]] for g in groups]
+    pinned_out = [[torch.empty_like(t, device="cpu").pin_memory() for t in [g["idx"], *g["outs"]]] for g in groups]
+
+    def e2e_step():
+        for g, pin, pout in zip(groups, pinned_in, pinned_out):
+            for dst, src in zip([g["iq"], g["wt"], *g["qs"]], pin):
+                dst.copy_(src, non_blocking=True)
+        graph.replay()
+        for g, pout in zip(groups, pinned_out):
+            for dst, src in zip(pout, [g["idx"], *g["outs"]]):
+                dst.copy_(src, non_blocking=True)
+
+    h2d = sum(t.numel() * t.element_size() for pin in pinned_in for t in pin)
+    d2h = sum(t.numel() * t.element_size() for pout in pinned_out for t in pout)
+    e2e_times = timed(e2e_step, args.steps, args.warmup)
+    e2e_ms = sum(e2e_times) / len(e2e_times)
+
+    if world > 1:
+        t = torch.tensor([step_ms, e2e_ms, idx_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        step_ms, e2e_ms, idx_ms = t.tolist()
+    return w, step_ms, idx_ms, e2e_ms, h2d, d2h, clk.summary()
+
+
+def cpu_baseline(w, n_seq):
+    """The oracle as it stands, on n_seq sequences of the workload (one IndexShare group,
+    all its layers), timed on this host; returns tokens/s and a description."""
+    import numpy as np
+    import oracle
+    import synth
+    from synth import configs as C
+    o = oracle.default()
+    n_seq = max(1, min(n_seq, w.B))
+    elapsed = 0.0
+    for b in range(n_seq):
+        iq = synth.int17_bf16(w.key(synth.KIND_IQ), (w.B, w.T, 32, 128))[b:b + 1]
+        wt = synth.pow2_f32(w.key(synth.KIND_W), (w.B, w.T, 32))[b:b + 1]
+        ik = synth.int17_bf16(w.key(synth.KIND_IK), index=synth.rows_index(
+            np.arange(b * w.N, (b + 1) * w.N), 128)).reshape(1, w.N, 128)
+        t0 = time.perf_counter()
+        sc = o.index_score(iq, wt, ik, w.q_pos0).astype(np.float32)
+        idx = o.topk(sc, w.q_pos0, w.k)
+        elapsed += time.perf_counter() - t0
+        rows = idx[0, 0]
+        for l in range(w.L):
+            q = synth.normal_bf16(w.key(synth.KIND_Q, 0, l), (w.B, w.T, w.H, 576))[b:b + 1]
+            kv = synth.normal_bf16(w.key(synth.KIND_KV, 0, l), index=synth.rows_index(
+                b * w.N + rows.astype(np.uint64), 576)).reshape(1, w.k, 576)
+            local = np.arange(w.k, dtype=np.int32).reshape(1, 1, w.k)
+            t0 = time.perf_counter()
+            o.sparse_attn(q, kv, local, C.SCALE)
+            elapsed += time.perf_counter() - t0
+    tokens = n_seq * w.T * w.groups
+    per_group_s = elapsed / n_seq
+    value = 1.0 / (per_group_s * w.groups) * w.T
+    return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{n_seq} of {w.B} sequences, one IndexShare group (indexer over {w.N} keys, top-{w.k}, "
+                      f"{w.L} attention layers), scaled to {w.groups} group(s) per token; inputs generated "
+                      f"outside the timed region; {tokens} token-groups timed in {elapsed:.1f} s"}
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from synth import configs as C
+    w = C.WORKLOADS[args.workload]
+    metric = "DSA group decode tokens/s"
+    if args.impl == "reference":
+        if rank == 0:
+            K = args.steps
+            vals = []
+            cb = None
+            for _ in range(args.warmup + K):
+                cb = cpu_baseline(w, 1)
+                vals.append(cb["value"])
+            v = sum(vals[args.warmup:]) / max(1, K)
+            cb["value"] = v
+            print(json.dumps({"impl": "reference", "metric": metric, "value": v, "unit": "tokens/s",
+                              "n_gpus": args.gpus, "steps": K, "warmup": args.warmup,
+                              "ms_per_step": 1e3 / v * w.B, "higher_is_better": True, "scaling": "weak",
+                              "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                              "config": {"workload": w.name, "B": w.B, "N": w.N, "k": w.k, "H": w.H, "L": w.L,
+                                         "groups": w.groups},
+                              "cpu_baseline": cb,
+                              "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                      "d2h_bytes_per_step": 0}}))
+        return
+
+    import torch
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    w, step_ms, idx_ms, e2e_ms, h2d, d2h, clocks = run_ours(args, rank, world, device)
+    step_bytes, idx_bytes = algorithmic(w)
+    tokens = w.B * w.T * world
+    value = tokens / (step_ms * 1e-3)
+    peak, peak_kind = peaks()
+    achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+    line = {
+        "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "T": w.T, "N": w.N, "k": w.k, "H": w.H, "L": w.L,
+                   "groups": w.groups, "l2": "flushed (512 MiB write) before every timed step",
+                   "parallelism": f"dp{world}" if world > 1 else "single GPU",
+                   "step_hbm_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
+                   "step_roofline_frac": step_bytes / (step_ms * 1e-3) / 1e9 / peak},
+        "clocks": clocks,
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h},
+        "gpu_launches": 5 * w.groups * args.steps,
+        "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
+                     "traffic": profiled_traffic("indexer.cu", w.name), "launch_us": idx_ms * 1e3,
+                     "algorithmic_bytes_per_launch": idx_bytes},
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
+    if rank == 0:
+        print(json.dumps(line))
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

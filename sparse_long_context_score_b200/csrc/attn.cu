@@ -332,7 +332,9 @@ attn_combine_kernel(AttnLayers layers, int H, int nsplit, const float* __restric
 template <int MT>
 cudaError_t launch_mt(const AttnLayers& layers, int L, const int32_t* idx, long long rows, int T, int N, int k,
                       int nsplit, int chunk, float scale_log2, float* partial, cudaStream_t stream) {
-  cudaError_t e = cudaFuncSetAttribute(sparse_attn_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+  static DeviceOnce once;
+  cudaError_t e = once.run(
+      [] { return cudaFuncSetAttribute(sparse_attn_kernel<MT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes); });
   if (e != cudaSuccess) return e;
   sparse_attn_kernel<MT><<<dim3(nsplit, (unsigned)rows, L), kThreads, kSmemBytes, stream>>>(layers, idx, T, N, k, chunk,
                                                                                             scale_log2, partial);

@@ -5,7 +5,26 @@
 #include <cstdint>
 #include <cuda_runtime.h>
 
+#include <atomic>
+
 namespace dsa {
+
+// Runs a set-up call (a kernel attribute) once per device, outside any stream capture
+// that follows the first call on that device.
+struct DeviceOnce {
+  std::atomic<int> done[64] = {};
+  template <class F>
+  cudaError_t run(F f) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return f();
+    if (done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+    e = f();
+    if (e == cudaSuccess) done[dev].store(1, std::memory_order_release);
+    return e;
+  }
+};
 
 constexpr int kIndexHeads = 32;   // index_n_heads
 constexpr int kIndexDim = 128;    // index_head_dim

@@ -378,8 +378,11 @@ cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_po
   // the select kernel needs every chunk of the row to take a ticket, so it runs over all
   // chunks of N (chunks past the visible range count nothing)
   const size_t smem = sizeof(SelectSmem);
-  e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  if (e != cudaSuccess) return e;
+  static DeviceOnce once;
+  if ((e = once.run([&] {
+         return cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+       })) != cudaSuccess)
+    return e;
   topk_select_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kSelThreads, smem, stream>>>(scores, T, N, q_pos0,
                                                                                                   k, ws, idx);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
