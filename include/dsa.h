@@ -103,6 +103,28 @@ dsa_status dsa_topk(const float *scores, int B, int T, int N, long long q_pos0, 
                     cudaStream_t stream);
 
 /*
+ * Top-k select that allocates nothing -- for callers that cannot allocate device memory
+ * (an inference engine's plugin enqueue step, a serving loop held to a fixed memory
+ * plan, code being recorded into a CUDA graph where cudaMalloc is not allowed).  The
+ * pages have no counterpart of this entry point; it is the same select as dsa_topk with
+ * the same bit-exact output, taking dsa_topk's arguments minus the workspace: its
+ * scratch is a fixed DSA_NOALLOC_SCRATCH_BYTES array inside the library, held on every
+ * GPU that loads the library until the process exits.
+ *   - Sizes whose select needs more scratch than that return DSA_ERR_WORKSPACE: at most
+ *     25 query rows (B*T) for N up to 1,048,576 (fewer for longer rows); use dsa_topk
+ *     beyond that.
+ *   - The first call on a device looks up the array's device address (a runtime call,
+ *     not an allocation); make that first call before any stream capture.
+ *   - All calls share the array and it keeps the last call's contents; the parts that
+ *     must start at zero are cleared on `stream` by every call.  Calls that overlap on
+ *     the GPU (unordered streams) race on the array and must not be issued.
+ *   - It calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+#define DSA_NOALLOC_SCRATCH_BYTES (2u << 20)
+dsa_status dsa_topk_noalloc(const float *scores, int B, int T, int N, long long q_pos0, int k,
+                            int32_t *idx, cudaStream_t stream);
+
+/*
  * Step 3 -- sparse MLA attention over the selected rows.
  *   q    [B, T, H, 576] bf16   attention queries (absorbed form)
  *   kv   [B, N, 576]    bf16   compressed cache; value = first 512 entries of a row

@@ -29,7 +29,7 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
 
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_topk",
-           "dsa_sparse_attn", "dsa_group_forward")
+           "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc")
 
 
 class DsaError(RuntimeError):
@@ -59,7 +59,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk.argtypes = [P, I, I, I, LL, I, P, P, S, P]
         L.dsa_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, F, P, P, S, P]
         L.dsa_group_forward.argtypes = [P, P, P, P, P, I, I, I, I, LL, I, I, F, I, P, P, P, S, P]
-        for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward"):
+        L.dsa_topk_noalloc.argtypes = [P, I, I, I, LL, I, P, P]
+        for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -199,3 +200,17 @@ def dsa_group_forward(iq, w, ik, qs, kvs, q_pos0: int, k: int, scale: float, com
         _ptr(ws, (torch.uint8,), "workspace"), ws.numel(), _stream(stream))
     _check(rc, "dsa_group_forward")
     return idx_shared, outs
+
+
+def dsa_topk_noalloc(scores, q_pos0: int, k: int, idx=None, stream=None):
+    """dsa_topk for callers that cannot allocate device memory: the select's scratch is a
+    fixed array inside libdsa (see include/dsa.h), so no workspace is passed.  Calls that
+    overlap on the GPU share that array and must not be issued."""
+    torch = _torch()
+    B, T, N = scores.shape
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=scores.device)
+    rc = lib().dsa_topk_noalloc(_ptr(scores, (torch.float32,), "scores"), B, T, N, int(q_pos0), int(k),
+                                _ptr(idx, (torch.int32,), "idx", (B, T, k)), _stream(stream))
+    _check(rc, "dsa_topk_noalloc")
+    return idx

@@ -7,6 +7,8 @@
 
 #include <atomic>
 
+#include "dsa.h"
+
 namespace dsa {
 
 // Runs a set-up call (a kernel attribute) once per device, outside any stream capture
