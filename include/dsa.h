@@ -69,6 +69,14 @@ const char *dsa_status_string(int status);
 int dsa_version(void);
 
 /*
+ * Device-side error word of the tensor-core kernels.  Their pipeline waits are bounded:
+ * a wait that runs out records a nonzero code and the kernel returns early (its outputs
+ * are then incomplete).  Synchronises with the device, writes the code (0 = none) to
+ * *code and returns DSA_ERR_TIMEOUT if it is set, DSA_OK otherwise; clear != 0 resets it.
+ */
+dsa_status dsa_device_error(int *code, int clear);
+
+/*
  * Bytes of workspace needed by dsa_topk, dsa_sparse_attn and dsa_group_forward for these
  * sizes (the largest of the three; one workspace serves all calls of that size).
  * B sequences, T queries per sequence, N cached rows, k top-k, H attention heads,

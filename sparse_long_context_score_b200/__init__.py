@@ -29,7 +29,7 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
 
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_topk",
-           "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc")
+           "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error")
 
 
 class DsaError(RuntimeError):
@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, F, P, P, S, P]
         L.dsa_group_forward.argtypes = [P, P, P, P, P, I, I, I, I, LL, I, I, F, I, P, P, P, S, P]
         L.dsa_topk_noalloc.argtypes = [P, I, I, I, LL, I, P, P]
+        L.dsa_device_error.argtypes = [ctypes.POINTER(I), I]
+        L.dsa_device_error.restype = I
         for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc"):
             getattr(L, f).restype = I
         _lib = L
@@ -103,6 +105,15 @@ def _bf16_types():
 def _check(rc: int, where: str) -> None:
     if rc != DSA_OK:
         raise DsaError(rc, where)
+
+
+def dsa_device_error(clear: bool = False) -> int:
+    """Device error word of the tensor-core kernels' bounded waits (0 = none); syncs."""
+    code = ctypes.c_int(0)
+    rc = lib().dsa_device_error(ctypes.byref(code), int(bool(clear)))
+    if rc not in (DSA_OK, -5):
+        raise DsaError(rc, "dsa_device_error")
+    return code.value
 
 
 def dsa_workspace_size(B: int, T: int, N: int, k: int, H: int, L: int) -> int:

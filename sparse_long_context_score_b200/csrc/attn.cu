@@ -329,6 +329,16 @@ attn_combine_kernel(AttnLayers layers, int H, int nsplit, const float* __restric
   *reinterpret_cast<float4*>(out) = make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
 }
 
+}  // namespace
+
+cudaError_t launch_attn_combine(const AttnLayers& layers, int L, long long rows, int H, int nsplit, const float* partial,
+                                cudaStream_t stream) {
+  attn_combine_kernel<<<dim3(H, (unsigned)rows, L), 128, 0, stream>>>(layers, H, nsplit, partial);
+  return cudaGetLastError();
+}
+
+namespace {
+
 template <int MT>
 cudaError_t launch_mt(const AttnLayers& layers, int L, const int32_t* idx, long long rows, int T, int N, int k,
                       int nsplit, int chunk, float scale_log2, float* partial, cudaStream_t stream) {
@@ -339,27 +349,26 @@ cudaError_t launch_mt(const AttnLayers& layers, int L, const int32_t* idx, long 
   sparse_attn_kernel<MT><<<dim3(nsplit, (unsigned)rows, L), kThreads, kSmemBytes, stream>>>(layers, idx, T, N, k, chunk,
                                                                                             scale_log2, partial);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (nsplit > 1) {
-    attn_combine_kernel<<<dim3(MT * 16, (unsigned)rows, L), 128, 0, stream>>>(layers, MT * 16, nsplit, partial);
-    e = cudaGetLastError();
-  }
+  if (nsplit > 1) e = launch_attn_combine(layers, L, rows, MT * 16, nsplit, partial, stream);
   return e;
-}
-
-int split_chunk(int k, int nsplit) {
-  int chunk = (k + nsplit - 1) / nsplit;
-  return (chunk + kBc - 1) / kBc * kBc;
 }
 
 }  // namespace
 
+// Keys per split: a multiple of the 64-row tile of the tensor-core kernel.
+int attn_split_chunk(int k, int nsplit) {
+  const int chunk = (k + nsplit - 1) / nsplit;
+  return (chunk + kAttnTile - 1) / kAttnTile * kAttnTile;
+}
+
+// Splits per (query row, layer): about one CTA per SM in total.
 int attn_num_splits(long long rows, int L, int k) {
   const long long units = rows * L;
   long long ns = kNumSMs / (units > 0 ? units : 1);
   if (ns < 1) ns = 1;
-  const long long max_ns = (k + kBc - 1) / kBc;
+  const long long max_ns = (k + kAttnTile - 1) / kAttnTile;
   if (ns > max_ns) ns = max_ns;
-  const int chunk = split_chunk(k, (int)ns);
+  const int chunk = attn_split_chunk(k, (int)ns);
   return (k + chunk - 1) / chunk;
 }
 
@@ -369,11 +378,11 @@ size_t attn_workspace_bytes(long long rows, int L, int H, int k) {
   return (size_t)L * rows * ns * H * (kDv + 2) * sizeof(float);
 }
 
-cudaError_t launch_sparse_attn(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H, int k,
-                               float scale, void* ws, cudaStream_t stream) {
+cudaError_t launch_sparse_attn_mma(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
+                                   int k, float scale, void* ws, cudaStream_t stream) {
   const long long rows = (long long)B * T;
   const int nsplit = attn_num_splits(rows, L, k);
-  const int chunk = split_chunk(k, nsplit);
+  const int chunk = attn_split_chunk(k, nsplit);
   const float scale_log2 = scale * 1.4426950408889634f;
   float* partial = static_cast<float*>(ws);
   switch (H) {

@@ -1,0 +1,471 @@
+// attn_tc.cu -- sparse MLA attention on the 5th-generation tensor cores.
+//
+// "GLM-5.2 1M architecture teardown", Cut 1: DSA (full attention over only the 2048 keys
+// the indexer kept) and Cut 3: MLA (one compressed 576-wide row per token, shared by all
+// heads; in the absorbed form the logit of head h is scale * q[h] . c[j] and the value is
+// the row's first 512 entries).
+//
+// One CTA per (query row, layer, key split); tiles of 32 selected rows.
+//   S   = Q K^T   M = 64 heads, N = 32 keys, K = 576    (36 MMAs; TMEM lane = head)
+//   O^T = V^T P^T M = 4 x 128 value dims, N = 64 heads, K = 32 keys (8 MMAs)
+// Because S has one head per TMEM lane, each softmax thread owns one head: its running
+// max and sum stay in registers and need no cross-thread reduction.  The running max is
+// only moved (and O rescaled in TMEM) when a tile's max exceeds it by more than 2^8, so
+// rescaling is rare; exponentials may then exceed 1 by at most 2^8, which f32 and bf16
+// carry without loss of relative precision.
+//
+// Warp roles (288 threads):
+//   warps 0..3  gather: the selected rows as 16-byte cp.async chunks written straight into
+//               the 128-byte-swizzled tensor-core layout; warp w owns stage w and tiles
+//               w, w+4, ..., waits for its own copies, fences them to the async proxy and
+//               arrives on the stage barrier, so four tiles are in flight and each is
+//               published as soon as it lands (one TMA load brings the 64 query rows).  Random 1152-byte rows are too small for TMA: a
+//               4-row gather copy per 512 bytes ran latency-bound on B200.
+//   warp 4      TMEM allocation; one thread issues S(i) and then O += P(i-1) V(i-1), so
+//               the softmax of one tile overlaps the next tile's logits;
+//   warps 5..8  softmax (threads on lanes 0..15 of each warp own a head), P as bf16 in
+//               shared memory, and at the end the read-out of O^T (lane = value dim) into
+//               shared memory and one bulk (TMA) store of the [H][512] output block --
+//               per-thread 4-byte global stores of that block ran at a few GB/s from an SM
+//               whose shared memory leaves almost no L1.
+// All mbarrier waits are bounded (sm100.cuh).
+#include <cudaTypedefs.h>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+#include "sm100.cuh"
+
+namespace dsa {
+
+namespace {
+
+using namespace sm100;
+
+static __device__ int g_attn_tc_error;
+
+constexpr int kKeys = 32;                        // selected rows per tile
+constexpr int kStages = 4;
+constexpr int kBlocks = kDqk / 64;               // nine 64-wide column blocks of a row
+constexpr int kQBlockBytes = 64 * 128;           // 64 heads x 64 bf16
+constexpr int kBlockBytes = kKeys * 128;         // 32 rows x 64 bf16
+constexpr int kQBytes = kBlocks * kQBlockBytes;  // 73728
+constexpr int kStageBytes = kBlocks * kBlockBytes;  // 36864
+constexpr int kPBytes = 64 * 128;                // 64 heads x 128-byte rows (first 64 bytes used)
+constexpr int kThreadsA = 288;
+constexpr int kChunksPerTile = kKeys * (kDqk / 8);  // 16-byte chunks: 2304
+constexpr float kRescaleLog2 = 8.f;
+
+constexpr int kOffQ = 0;
+constexpr int kOffStage = kOffQ + kQBytes;
+constexpr int kOffP = kOffStage + kStages * kStageBytes;
+constexpr int kOffAlpha = kOffP + kPBytes;       // [2][64] f32 (tile parity)
+constexpr int kOffL = kOffAlpha + 2 * 64 * 4;    // [64] f32
+constexpr int kOffM = kOffL + 64 * 4;            // [64] f32
+constexpr int kOffMask = kOffM + 64 * 4;         // [kStages] u32
+constexpr int kOffRows = kOffMask + kStages * 4; // [kStages][kKeys] int
+constexpr int kNumBars = 2 * kStages + 9;
+constexpr int kOffBar = kOffRows + kStages * kKeys * 4;
+constexpr int kOffTmem = kOffBar + kNumBars * 8;
+constexpr int kSmemA = kOffTmem + 16 + 1024;
+static_assert(kSmemA <= 232448, "shared memory budget");
+
+constexpr int kTmemO = 0;      // O^T: 4 blocks x 64 columns, all 128 lanes
+constexpr int kTmemS = 256;    // S: 2 buffers x 32 columns, lanes 0..15 of each quarter
+constexpr int kTmemCols = 512;
+
+struct AttnMaps {
+  CUtensorMap q[kMaxLayers];
+};
+
+__global__ void __launch_bounds__(kThreadsA, 1)
+attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const int32_t* __restrict__ idx, int T, int N,
+               int H, int k, int chunk, float scale_log2, float* __restrict__ partial, int* __restrict__ err) {
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + kOffQ;
+  const uint32_t sStage = sbase + kOffStage;
+  const uint32_t sP = sbase + kOffP;
+  float* s_alpha = reinterpret_cast<float*>(smem + kOffAlpha);
+  float* s_l = reinterpret_cast<float*>(smem + kOffL);
+  float* s_m = reinterpret_cast<float*>(smem + kOffM);
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem + kOffMask);
+  int* s_rows = reinterpret_cast<int*>(smem + kOffRows);
+  const uint32_t bar0 = sbase + kOffBar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
+  auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
+  auto sfree_bar = [&](int s) { return bar0 + 8u * (2 * kStages + 2 + s); };
+  const uint32_t pfull_bar = bar0 + 8u * (2 * kStages + 4);
+  const uint32_t pfree_bar = bar0 + 8u * (2 * kStages + 5);
+  const uint32_t ofinal_bar = bar0 + 8u * (2 * kStages + 6);
+  const uint32_t qfull_bar = bar0 + 8u * (2 * kStages + 7);
+  const uint32_t grp_bar = bar0 + 8u * (2 * kStages + 8);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
+
+  const int split = blockIdx.x, row = blockIdx.y, layer = blockIdx.z;
+  const int nsplit = gridDim.x;
+  const int b = row / T;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int j0 = split * chunk;
+  const int nkeys = max(min(j0 + chunk, k) - j0, 0);
+  const int ntiles = (nkeys + kKeys - 1) / kKeys;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(full_bar(s), 32);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(sfull_bar(s), 1);
+      mbar_init(sfree_bar(s), 128);
+    }
+    mbar_init(pfull_bar, 128);
+    mbar_init(pfree_bar, 1);
+    mbar_init(ofinal_bar, 1);
+    mbar_init(qfull_bar, 1);
+    mbar_init(grp_bar, 128);
+    fence_mbar_init();
+    tma_prefetch(&maps.q[layer]);
+  }
+  if (warp == 4) {
+    tmem_alloc(smem_u32(s_tmem), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+
+  if (warp < 4) {
+    // ------------------------------------------------------------------ gather
+    // warp pw owns stage pw and fills tiles pw, pw + 4, ...: four tiles in flight, each
+    // published as soon as its own rows have landed
+    const int pw = warp;
+    if (pw == 0 && lane == 0) {
+      const CUtensorMap* qm = &maps.q[layer];
+      mbar_arrive_expect_tx(qfull_bar, kQBytes);
+      for (int kb = 0; kb < kBlocks; ++kb) tma_load_2d(sQ + kb * kQBlockBytes, qm, qfull_bar, 64 * kb, row * H);
+    }
+    const int32_t* sel = idx + (size_t)row * k + j0;
+    const uint16_t* kvb = layers.kv[layer] + (size_t)b * N * kDqk;
+    int* rows = s_rows + pw * kKeys;
+    const uint32_t st = sStage + pw * kStageBytes;
+    for (int i = pw; i < ntiles; i += kStages) {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(empty_bar(pw), ((i / kStages) & 1) ^ 1, err, 21);
+      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      if (!ok) break;
+      const int key = i * kKeys + lane;
+      const int v = key < nkeys ? __ldg(&sel[key]) : -1;
+      const bool valid = v >= 0 && v < N;
+      rows[lane] = valid ? v : 0;
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, valid);
+      if (lane == 0) s_mask[pw] = m;
+      __syncwarp();
+#pragma unroll 8
+      for (int c = lane; c < kChunksPerTile; c += 32) {
+        const int r = c / (kDqk / 8), cc = c - r * (kDqk / 8);
+        const uint32_t dst = st + (cc >> 3) * kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
+        cp_async_16(dst, kvb + (size_t)rows[r] * kDqk + cc * 8, 16);
+      }
+      cp_async_commit();
+      cp_async_wait<0>();
+      fence_proxy_async();  // the copies are visible to the tensor core (async proxy)
+      mbar_arrive(full_bar(pw));
+    }
+    if (pw == 0 && lane == 0) mbar_wait_drain(qfull_bar, 0);
+  } else if (warp == 4) {
+    // ------------------------------------------------------------------ MMA issuer
+    // the whole warp runs the loop (descriptor arithmetic stays warp-uniform); one
+    // elected lane issues the tensor-core instructions
+    const bool leader = elect_one();
+    constexpr uint32_t idS = idesc_bf16_f32(64, kKeys);              // Q (K-major) x K (K-major)
+    constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true, false);  // V^T (M-major) x P (K-major)
+    bool ok = mbar_wait(qfull_bar, 0, err, 22);
+    const uint64_t dq = sdesc_kmajor_sw128(sQ);
+    const uint64_t dp = sdesc_kmajor_sw128(sP);
+    for (int i = 0; i <= ntiles && ok; ++i) {
+      if (i < ntiles) {
+        const int s = i % kStages, sb = i & 1;
+        ok = mbar_wait(full_bar(s), (i / kStages) & 1, err, 23);
+        if (ok) ok = mbar_wait(sfree_bar(sb), ((i >> 1) & 1) ^ 1, err, 24);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t dS = tmem + kTmemS + kKeys * sb;
+        // descriptors differ only in their start address: compile-time offsets from a base
+        const uint64_t dk = sdesc_kmajor_sw128(sStage + s * kStageBytes);
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < 4 * kBlocks; ++kk)
+            mma_bf16(dS, dq + (uint64_t)((((kk >> 2) * kQBlockBytes) + (kk & 3) * 32) >> 4),
+                     dk + (uint64_t)((((kk >> 2) * kBlockBytes) + (kk & 3) * 32) >> 4), idS, kk > 0);
+          mma_commit(sfull_bar(sb));
+        }
+        __syncwarp();
+      }
+      if (i >= 1) {
+        const int jt = i - 1, sj = jt % kStages;
+        ok = mbar_wait(pfull_bar, jt & 1, err, 25);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t da = sdesc_mnmajor_sw128(sStage + sj * kStageBytes, kBlockBytes, 1024);
+        const uint32_t first = jt > 0 ? 1u : 0u;
+        if (leader) {
+#pragma unroll
+          for (int mb = 0; mb < 4; ++mb)
+#pragma unroll
+            for (int ks = 0; ks < kKeys / 16; ++ks)
+              mma_bf16(tmem + kTmemO + 64 * mb, da + (uint64_t)(((2 * mb) * kBlockBytes + ks * 16 * 128) >> 4),
+                       dp + (uint64_t)((ks * 32) >> 4), idPV, first | (ks > 0 ? 1u : 0u));
+          mma_commit(pfree_bar);
+          mma_commit(empty_bar(sj));
+        }
+        __syncwarp();
+      }
+    }
+    if (leader) {
+      mma_commit(ofinal_bar);
+      if (!mbar_wait_drain(ofinal_bar, 0)) atomicCAS(err, 0, 26);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------------ softmax + read-out
+    const int quarter = warp & 3;
+    const int st_tid = threadIdx.x - 160;         // 0..127
+    const bool owner = lane < 16;                 // this thread's TMEM lane holds a head of S
+    const int head = 16 * quarter + (lane & 15);
+    const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
+    float m_used = -INFINITY, l_run = 0.f;
+    uint32_t grp_phase = 0;
+    bool ok = true;
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int sb = i & 1, s = i % kStages;
+      ok = mbar_wait(sfull_bar(sb), (i >> 1) & 1, err, 27);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t r[kKeys];
+      tmem_ld32(tmem + lane_addr + kTmemS + kKeys * sb, r);
+      tmem_ld_wait();
+      tc_fence_before();
+      mbar_arrive(sfree_bar(sb));
+      ok = mbar_wait(full_bar(s), (i / kStages) & 1, err, 28);  // orders the gather's mask write
+      if (!ok) break;
+      const uint32_t mask = s_mask[s];
+      float* alpha = s_alpha + 64 * (i & 1);
+      float mt = -INFINITY;
+#pragma unroll
+      for (int j = 0; j < kKeys; ++j) {
+        const float z = ((mask >> j) & 1u) ? __uint_as_float(r[j]) * scale_log2 : -INFINITY;
+        r[j] = __float_as_uint(z);
+        mt = fmaxf(mt, z);
+      }
+      float a = 1.f;
+      if (mt > m_used + kRescaleLog2 || (m_used == -INFINITY && mt > -INFINITY)) {
+        a = m_used == -INFINITY ? 0.f : exp2f(m_used - mt);
+        m_used = mt;
+        l_run *= a;
+      }
+      if (owner) alpha[head] = a;
+      // every head's factor is known before O is touched
+      mbar_arrive(grp_bar);
+      ok = mbar_wait(grp_bar, grp_phase, err, 29);
+      grp_phase ^= 1;
+      if (!ok) break;
+      if (i > 0) {
+        ok = mbar_wait(pfree_bar, (i - 1) & 1, err, 30);  // O^T and P are no longer in use
+        if (!ok) break;
+        tc_fence_after();
+        bool any = false;
+#pragma unroll 8
+        for (int h = 0; h < 64; ++h) any |= h < H && alpha[h] != 1.f;
+        if (any) {
+          // rescale O^T: this thread's lane is one value dim, its columns the heads
+#pragma unroll 1
+          for (int mb = 0; mb < 4; ++mb)
+#pragma unroll 1
+            for (int half = 0; half < 2; ++half) {
+              uint32_t o[32];
+              const uint32_t ta = tmem + lane_addr + kTmemO + 64 * mb + 32 * half;
+              tmem_ld32(ta, o);
+              tmem_ld_wait();
+#pragma unroll
+              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha[32 * half + c]);
+              tmem_st32(ta, o);
+            }
+          tmem_st_wait();
+        }
+      }
+      if (owner) {
+        const float mu = m_used == -INFINITY ? 0.f : m_used;
+        float ls = 0.f;
+        uint32_t packed[kKeys / 2];
+#pragma unroll
+        for (int j = 0; j < kKeys; j += 2) {
+          const float p0 = exp2f(__uint_as_float(r[j]) - mu);
+          const float p1 = exp2f(__uint_as_float(r[j + 1]) - mu);
+          ls += p0 + p1;
+          packed[j / 2] = pack_bf16x2(p0, p1);
+        }
+        l_run += ls;
+        // P row `head`: 32 keys in the first 64 bytes of a 128-byte swizzled row (K-major)
+        unsigned char* prow = smem + kOffP + head * 128;
+#pragma unroll
+        for (int c = 0; c < kKeys / 8; ++c)
+          *reinterpret_cast<uint4*>(prow + ((c ^ (head & 7)) << 4)) =
+              make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
+        fence_proxy_async();
+      }
+      tc_fence_before();
+      mbar_arrive(pfull_bar);
+    }
+    // ------------------------------------------------------------------ read-out
+    if (ok && ntiles > 0) ok = mbar_wait(ofinal_bar, 0, err, 31);
+    tc_fence_after();
+    if (owner) {
+      s_l[head] = l_run;
+      s_m[head] = m_used;
+    }
+    mbar_arrive(grp_bar);
+    if (ok) ok = mbar_wait(grp_bar, grp_phase, err, 32);
+    if (ok) {
+      // O^T (lane = value dim, column = head) -> shared [head][512] (the stage ring is idle
+      // now) -> one bulk store of the whole [H][512] block
+      float* s_out = reinterpret_cast<float*>(smem + kOffStage);
+      const int dim_lane = 32 * quarter + lane;
+      // the 64 normalisers in registers once: a dependent shared load per element,
+      // serialised against the shared stores below, made this loop ~20x slower
+      float inv[64];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float4 l4 = reinterpret_cast<const float4*>(s_l)[j];
+        inv[4 * j + 0] = nsplit > 1 ? 1.f : (l4.x > 0.f ? 1.f / l4.x : 0.f);
+        inv[4 * j + 1] = nsplit > 1 ? 1.f : (l4.y > 0.f ? 1.f / l4.y : 0.f);
+        inv[4 * j + 2] = nsplit > 1 ? 1.f : (l4.z > 0.f ? 1.f / l4.z : 0.f);
+        inv[4 * j + 3] = nsplit > 1 ? 1.f : (l4.w > 0.f ? 1.f / l4.w : 0.f);
+      }
+#pragma unroll 1
+      for (int mb = 0; mb < 4; ++mb) {
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o[32];
+          if (ntiles > 0) {
+            tmem_ld32(tmem + lane_addr + kTmemO + 64 * mb + 32 * half, o);
+            tmem_ld_wait();
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; ++c) o[c] = 0u;
+          }
+          const int dim = 128 * mb + dim_lane;
+          // rows h >= H are written too (the store below copies only the first H)
+#pragma unroll
+          for (int c = 0; c < 32; ++c) s_out[(32 * half + c) * kDv + dim] = __uint_as_float(o[c]) * inv[32 * half + c];
+        }
+      }
+      fence_proxy_async();
+      mbar_arrive(grp_bar);
+      grp_phase ^= 1;
+      ok = mbar_wait(grp_bar, grp_phase, err, 33);
+      const size_t unit = ((size_t)layer * gridDim.y + row) * nsplit + split;
+      if (ok && st_tid == 0) {
+        float* dst = nsplit == 1 ? layers.out[layer] + (size_t)row * H * kDv : partial + unit * (size_t)H * (kDv + 2);
+        bulk_store(dst, smem_u32(s_out), (uint32_t)(H * kDv * 4));
+        bulk_commit();
+        bulk_wait_all();
+      }
+      if (ok && nsplit > 1 && st_tid < H) {
+        float* pm = partial + unit * (size_t)H * (kDv + 2) + (size_t)H * kDv;
+        pm[2 * st_tid] = ntiles > 0 ? s_m[st_tid] : -INFINITY;
+        pm[2 * st_tid + 1] = ntiles > 0 ? s_l[st_tid] : 0.f;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 map over [rows][576] with a 64-column x box_rows box and 128-byte swizzle
+bool make_map_576(CUtensorMap* map, const void* base, long long rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kDqk, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)kDqk * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct ErrAddr {
+  std::atomic<int*> ptr[64] = {};
+  cudaError_t get(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int* p = ptr[dev].load();
+    if (!p) {
+      void* v = nullptr;
+      if ((e = cudaGetSymbolAddress(&v, g_attn_tc_error)) != cudaSuccess) return e;
+      p = static_cast<int*>(v);
+      ptr[dev].store(p);
+    }
+    *out = p;
+    return cudaSuccess;
+  }
+};
+ErrAddr g_err_addr;
+
+}  // namespace
+
+cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
+                                  int k, float scale, void* ws, cudaStream_t stream) {
+  const long long rows = (long long)B * T;
+  AttnMaps maps;
+  for (int l = 0; l < L; ++l)
+    if (!make_map_576(&maps.q[l], layers.q[l], rows * H, 64)) return cudaErrorInvalidValue;
+  int* err = nullptr;
+  cudaError_t e = g_err_addr.get(&err);
+  if (e != cudaSuccess) return e;
+  static DeviceOnce once;
+  if ((e = once.run([] { return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA); })) !=
+      cudaSuccess)
+    return e;
+  const int nsplit = attn_num_splits(rows, L, k);
+  const int chunk = attn_split_chunk(k, nsplit);
+  float* partial = static_cast<float*>(ws);
+  attn_tc_kernel<<<dim3(nsplit, (unsigned)rows, L), kThreadsA, kSmemA, stream>>>(maps, layers, idx, T, N, H, k, chunk,
+                                                                                 scale * 1.4426950408889634f, partial, err);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (nsplit > 1) e = launch_attn_combine(layers, L, rows, H, nsplit, partial, stream);
+  return e;
+}
+
+cudaError_t attn_tc_device_error(int* code, bool clear) {
+  int* p = nullptr;
+  cudaError_t e = g_err_addr.get(&p);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemcpy(code, p, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess) return e;
+  if (clear && *code) e = cudaMemset(p, 0, sizeof(int));
+  return e;
+}
+
+}  // namespace dsa

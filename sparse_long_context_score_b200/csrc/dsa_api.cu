@@ -67,6 +67,16 @@ const char* dsa_status_string(int status) {
 
 int dsa_version(void) { return 10000; }
 
+dsa_status dsa_device_error(int* code, int clear) {
+  if (!code) return DSA_ERR_INVALID_ARG;
+  *code = 0;
+  int a = 0;
+  if (indexer_tc_device_error(code, clear != 0) != cudaSuccess) return DSA_ERR_CUDA;
+  if (attn_tc_device_error(&a, clear != 0) != cudaSuccess) return DSA_ERR_CUDA;
+  if (!*code) *code = a;
+  return *code ? DSA_ERR_TIMEOUT : DSA_OK;
+}
+
 size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L) {
   if (!sizes_ok(B, T, N) || k <= 0 || k > DSA_MAX_TOPK || H <= 0 || L <= 0 || L > DSA_MAX_LAYERS) return 0;
   return group_layout(B, T, N, k, H, L).total;
@@ -76,7 +86,7 @@ dsa_status dsa_index_score(const uint16_t* q, const float* w, const uint16_t* k,
                            long long q_pos0, float* scores, cudaStream_t stream) {
   if (!q || !w || !k || !scores || !sizes_ok(B, T, N)) return DSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 4) || !aligned(scores, 4)) return DSA_ERR_INVALID_ARG;
-  return cuda_status(launch_index_score(q, w, k, B, T, N, q_pos0, scores, nullptr, stream));
+  return cuda_status(launch_index_score_tc(q, w, k, B, T, N, q_pos0, scores, nullptr, stream));
 }
 
 dsa_status dsa_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx, void* workspace,
@@ -103,7 +113,7 @@ dsa_status dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const int32_t*
   layers.q[0] = q;
   layers.kv[0] = kv;
   layers.out[0] = out;
-  return cuda_status(launch_sparse_attn(layers, 1, idx, B, T, N, H, k, scale, workspace, stream));
+  return cuda_status(launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, workspace, stream));
 }
 
 dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t* ik, const uint16_t* const* q,
@@ -132,14 +142,16 @@ dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t*
   if (compute_indices) {
     TopkWorkspace tws = topk_workspace(base + g.topk_off, rows, N);
     float* scores = reinterpret_cast<float*>(base + g.scores_off);
-    // the indexer folds the first radix digit of the select into its epilogue
-    if ((e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess) return DSA_ERR_CUDA;
-    if ((e = launch_index_score(iq, w, ik, B, T, N, q_pos0, scores, tws.hist, stream)) != cudaSuccess)
+    // in decode the indexer folds the first radix digit of the select into its epilogue
+    const bool fused_hist = T == 1 && B <= kNumSMs;
+    if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess) return DSA_ERR_CUDA;
+    if ((e = launch_index_score_tc(iq, w, ik, B, T, N, q_pos0, scores, fused_hist ? tws.hist : nullptr, stream)) !=
+        cudaSuccess)
       return DSA_ERR_CUDA;
-    if ((e = launch_topk(scores, B, T, N, q_pos0, k, idx_shared, tws, true, stream)) != cudaSuccess)
+    if ((e = launch_topk(scores, B, T, N, q_pos0, k, idx_shared, tws, fused_hist, stream)) != cudaSuccess)
       return DSA_ERR_CUDA;
   }
-  e = launch_sparse_attn(layers, L, idx_shared, B, T, N, H, k, scale, base + g.attn_off, stream);
+  e = launch_sparse_attn_tc(layers, L, idx_shared, B, T, N, H, k, scale, base + g.attn_off, stream);
   return cuda_status(e);
 }
 

@@ -62,16 +62,32 @@ struct AttnLayers {
   float* out[kMaxLayers];
 };
 
+constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core attention
+
 int attn_num_splits(long long rows, int L, int k);
+int attn_split_chunk(int k, int nsplit);
+cudaError_t launch_attn_combine(const AttnLayers& layers, int L, long long rows, int H, int nsplit, const float* partial,
+                                cudaStream_t stream);
 size_t attn_workspace_bytes(long long rows, int L, int H, int k);
 
 cudaError_t launch_index_score(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
                                long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream);
 
+// tcgen05 indexer (T == 1: decode, one query per MMA; T > 1: 8 queries per MMA).  With a
+// histogram pointer (decode only, B <= 148) the first radix digit of the select is counted.
+cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
+                                  long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream);
+// error word of the tensor-core kernels' bounded waits (0 = none)
+cudaError_t indexer_tc_device_error(int* code, bool clear);
+
 cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
                         const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream);
 
-cudaError_t launch_sparse_attn(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                               int k, float scale, void* ws, cudaStream_t stream);
+// tcgen05 attention (the product path) and the warp-level mma.sync one (kept for comparison)
+cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
+                                  int k, float scale, void* ws, cudaStream_t stream);
+cudaError_t launch_sparse_attn_mma(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
+                                   int k, float scale, void* ws, cudaStream_t stream);
+cudaError_t attn_tc_device_error(int* code, bool clear);
 
 }  // namespace dsa

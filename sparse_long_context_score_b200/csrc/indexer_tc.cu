@@ -1,0 +1,434 @@
+// indexer_tc.cu -- lightweight indexer score on the 5th-generation tensor cores.
+//
+// I(t,s) = sum_h w[t,h] * ReLU(q[t,h] . k[s])   ("GLM-5.2 1M architecture teardown",
+// Cut 1: DSA -- index_n_heads 32, index_head_dim 128).
+//
+// For a tile of 128 cached keys and a group of QG queries the head dot products are one
+// matrix product: D[key][(query, head)] = K[128 x 128] * Q[(QG*32) x 128]^T, M = 128,
+// N = 32*QG, K = 128 (8 MMAs of K = 16).  QG = 1 for decode (the key stream is the whole
+// cost; the tensor core is ~10% busy), QG = 8 for chunked prefill (a dense contraction).
+//
+// Warp roles (192 threads, one CTA per SM, persistent over a contiguous range of
+// (query group, key tile) items):
+//   warp 0      TMA producer: 128x128 bf16 key tiles (two 64-column boxes, 128-byte
+//               swizzle) into a ring of shared-memory stages; the query group once per
+//               group change;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma into one of two TMEM
+//               accumulators (2 x 32*QG columns) and commits to the stage / accumulator
+//               barriers;
+//   warps 2..5  epilogue: each thread owns one key row of the accumulator (its warp's
+//               TMEM lane quarter), loads the 32 head columns of each query, applies
+//               ReLU and the head weights, sums, and stores the score (coalesced: a warp
+//               writes 32 consecutive keys).  In decode it can also count the first radix
+//               digit of each score into a per-row histogram for the top-k select.
+// Every mbarrier wait is bounded (see sm100.cuh); a timeout sets the device error word.
+#include <cudaTypedefs.h>
+
+#include "dsa_common.cuh"
+#include "dsa_internal.h"
+#include "sm100.cuh"
+
+namespace dsa {
+
+namespace {
+
+using namespace sm100;
+
+static __device__ int g_indexer_tc_error;
+
+constexpr int kTileKeys = 128;
+constexpr int kThreadsTC = 192;
+constexpr int kHalfBytesA = kTileKeys * 128;  // 128 rows x 64 bf16 = 16 KB
+constexpr int kStageBytesA = 2 * kHalfBytesA;
+
+template <int QG, bool kHist>
+struct TcCfg {
+  static constexpr int kN = 32 * QG;                  // MMA N
+  static constexpr int kStages = QG == 1 ? 5 : 4;
+  static constexpr int kHalfBytesB = kN * 128;
+  static constexpr int kBytesB = 2 * kHalfBytesB;
+  static constexpr int kTmemCols = (2 * kN) < 32 ? 32 : 2 * kN;  // power of two for QG in {1, 8}
+  static constexpr int kOffA = 0;
+  static constexpr int kOffB = kOffA + kStages * kStageBytesA;
+  static constexpr int kOffHist = kOffB + kBytesB;     // two row histograms (a CTA spans <= 2 rows)
+  static constexpr int kOffBar = kOffHist + (kHist ? 2 * kHistBins * 4 : 0);
+  static constexpr int kNumBars = 2 * kStages + 4 + 3;
+  static constexpr int kOffTmem = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffTmem + 16 + 1024;  // + alignment slack
+};
+
+struct Items {
+  int B, T, N, G;  // G = query groups per sequence
+  long long q_pos0;
+  int QG;
+  __device__ int tiles(int qg) const {
+    const int t0 = (qg % G) * QG;
+    const int tl = min(t0 + QG, T) - 1;
+    const long long v = visible_count(N, q_pos0, tl);
+    return (int)((v + kTileKeys - 1) / kTileKeys);
+  }
+};
+
+// Walks the flattened (query group, key tile) items [begin, end).
+struct Cursor {
+  int qg, tile, left_in_qg;
+  long long remaining;
+  __device__ void start(const Items& it, long long begin, long long end) {
+    remaining = end - begin;
+    qg = 0;
+    long long acc = 0;
+    const int nqg = it.B * it.G;
+    while (qg < nqg) {
+      const int n = it.tiles(qg);
+      if (acc + n > begin) break;
+      acc += n;
+      ++qg;
+    }
+    tile = (int)(begin - acc);
+    left_in_qg = qg < nqg ? it.tiles(qg) - tile : 0;
+  }
+  __device__ bool valid() const { return remaining > 0; }
+  __device__ void next(const Items& it) {
+    --remaining;
+    ++tile;
+    if (--left_in_qg == 0 && remaining > 0) {
+      do {
+        ++qg;
+        tile = 0;
+        left_in_qg = it.tiles(qg);
+      } while (left_in_qg == 0);
+    }
+  }
+};
+
+template <int QG, bool kHist>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                  const float* __restrict__ w, int B, int T, int N, long long q_pos0, long long total_items,
+                  float* __restrict__ scores, uint32_t* __restrict__ hist, int* __restrict__ err) {
+  using C = TcCfg<QG, kHist>;
+  extern __shared__ unsigned char smem_raw[];
+  unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sA = sbase + C::kOffA;
+  const uint32_t sB = sbase + C::kOffB;
+  uint32_t* s_hist = reinterpret_cast<uint32_t*>(smem + C::kOffHist);
+  const uint32_t bar0 = sbase + C::kOffBar;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
+  auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
+  const uint32_t qfull_bar = bar0 + 8u * (2 * C::kStages + 4);
+  const uint32_t qfree_bar = bar0 + 8u * (2 * C::kStages + 5);
+  const uint32_t done_bar = bar0 + 8u * (2 * C::kStages + 6);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  Items it{B, T, N, (T + QG - 1) / QG, q_pos0, QG};
+  const long long per = total_items / gridDim.x, extra = total_items % gridDim.x;
+  const long long begin = blockIdx.x * per + min((long long)blockIdx.x, extra);
+  const long long end = begin + per + (blockIdx.x < extra ? 1 : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(tfull_bar(b), 1);
+      mbar_init(tempty_bar(b), 128);
+    }
+    mbar_init(qfull_bar, 1);
+    mbar_init(qfree_bar, 1);
+    mbar_init(done_bar, 1);
+    fence_mbar_init();
+    tma_prefetch(&kmap);
+    tma_prefetch(&qmap);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(s_tmem), C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (kHist)
+    for (int i = threadIdx.x; i < 2 * kHistBins; i += kThreadsTC) s_hist[i] = 0;
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *s_tmem;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      Cursor cur;
+      cur.start(it, begin, end);
+      int stage = 0;
+      uint32_t phase = 0, qfree_phase = 0;
+      int cur_qg = -1;
+      long long issued = 0;
+      bool ok = true, q_pending = false;
+      uint32_t q_parity = 0;
+      while (cur.valid() && ok) {
+        if (cur.qg != cur_qg) {
+          if (cur_qg >= 0) {
+            ok = mbar_wait(qfree_bar, qfree_phase, err, 1);
+            qfree_phase ^= 1;
+            if (!ok) break;
+          }
+          const int b = cur.qg / it.G, t0 = (cur.qg % it.G) * QG;
+          mbar_arrive_expect_tx(qfull_bar, C::kBytesB);
+          tma_load_3d(sB, &qmap, qfull_bar, 0, t0 * 32, b);
+          tma_load_3d(sB + C::kHalfBytesB, &qmap, qfull_bar, 64, t0 * 32, b);
+          q_pending = true;
+          q_parity = (cur_qg >= 0) ? (q_parity ^ 1) : 0;
+          cur_qg = cur.qg;
+        }
+        ok = mbar_wait(empty_bar(stage), phase ^ 1, err, 2);
+        if (!ok) break;
+        const int b = cur.qg / it.G;
+        const uint32_t dst = sA + stage * kStageBytesA;
+        mbar_arrive_expect_tx(full_bar(stage), kStageBytesA);
+        tma_load_3d(dst, &kmap, full_bar(stage), 0, cur.tile * kTileKeys, b);
+        tma_load_3d(dst + kHalfBytesA, &kmap, full_bar(stage), 64, cur.tile * kTileKeys, b);
+        ++issued;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        cur.next(it);
+      }
+      if (!ok) {
+        // let the loads already in flight land before the CTA exits
+        for (long long j = issued > C::kStages ? issued - C::kStages : 0; j < issued; ++j)
+          mbar_wait_drain(full_bar((int)(j % C::kStages)), (uint32_t)((j / C::kStages) & 1));
+        if (q_pending) mbar_wait_drain(qfull_bar, q_parity);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16_f32(kTileKeys, C::kN);
+      Cursor cur;
+      cur.start(it, begin, end);
+      int stage = 0;
+      uint32_t phase = 0, qfull_phase = 0;
+      long long acc = 0;
+      int cur_qg = -1;
+      bool ok = true;
+      while (cur.valid() && ok) {
+        if (cur.qg != cur_qg) {
+          if (cur_qg >= 0) mma_commit(qfree_bar);
+          ok = mbar_wait(qfull_bar, qfull_phase, err, 4);
+          qfull_phase ^= 1;
+          if (!ok) break;
+          cur_qg = cur.qg;
+        }
+        const int buf = (int)(acc & 1);
+        const uint32_t use = (uint32_t)(acc >> 1);
+        ok = mbar_wait(tempty_bar(buf), (use & 1) ^ 1, err, 5);
+        if (!ok) break;
+        tc_fence_after();
+        ok = mbar_wait(full_bar(stage), phase, err, 6);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + buf * C::kN;
+        const uint64_t ad0 = sdesc_kmajor_sw128(sA + stage * kStageBytesA);
+        const uint64_t bd0 = sdesc_kmajor_sw128(sB);
+#pragma unroll
+        for (int kh = 0; kh < 2; ++kh)
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(d, ad0 + (uint64_t)((kh * kHalfBytesA + ks * 32) >> 4),
+                     bd0 + (uint64_t)((kh * C::kHalfBytesB + ks * 32) >> 4), idesc, (kh | ks) != 0);
+        mma_commit(empty_bar(stage));
+        mma_commit(tfull_bar(buf));
+        ++acc;
+        if (++stage == C::kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+        cur.next(it);
+      }
+      // every MMA issued so far has finished before TMEM is released
+      mma_commit(done_bar);
+      if (!mbar_wait_drain(done_bar, 0)) atomicCAS(err, 0, 7);
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int row_in_tile = 32 * quarter + lane;
+    Cursor cur;
+    cur.start(it, begin, end);
+    const int b_first = cur.valid() ? cur.qg / it.G : 0;
+    long long acc = 0;
+    int cur_qg = -1;
+    float wr[32];  // head weights of the current query (decode)
+    bool ok = true;
+    while (cur.valid() && ok) {
+      const int b = cur.qg / it.G, t0 = (cur.qg % it.G) * QG;
+      if (QG == 1 && cur.qg != cur_qg) {
+        const float* wq = w + ((size_t)b * T + t0) * 32;
+#pragma unroll
+        for (int h = 0; h < 32; ++h) wr[h] = __ldg(&wq[h]);
+        cur_qg = cur.qg;
+      }
+      const int buf = (int)(acc & 1);
+      const uint32_t use = (uint32_t)(acc >> 1);
+      ok = mbar_wait(tfull_bar(buf), use & 1, err, 8);
+      if (!ok) break;
+      tc_fence_after();
+      const long long key = (long long)cur.tile * kTileKeys + row_in_tile;
+      int slot = kHist ? b - b_first : 0;
+      if (slot > 1) {  // cannot happen for B <= 148 (checked by the host); never write past the slots
+        atomicCAS(err, 0, 9);
+        slot = 1;
+      }
+      uint32_t* hslot = s_hist + slot * kHistBins;
+#pragma unroll 1
+      for (int g = 0; g < QG; ++g) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * C::kN + 32 * g, r);
+        tmem_ld_wait();
+        const int t = t0 + g;
+        float sc = 0.f;
+        if (QG == 1) {
+#pragma unroll
+          for (int h = 0; h < 32; ++h) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
+        } else {
+          const float* wq = w + ((size_t)b * T + (t < T ? t : T - 1)) * 32;
+#pragma unroll
+          for (int h = 0; h < 32; ++h) sc = fmaf(__ldg(&wq[h]), fmaxf(__uint_as_float(r[h]), 0.f), sc);
+        }
+        if (t < T && key < visible_count(N, q_pos0, t)) {
+          scores[((size_t)b * T + t) * N + key] = sc;
+          if (kHist) atomicAdd(&hslot[order_key(sc) >> kHistShift], 1u);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(buf));
+      ++acc;
+      cur.next(it);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+  if (kHist && begin < end) {
+    // fold this CTA's counts into the per-row histograms (decode: row = sequence)
+    Cursor cur;
+    cur.start(it, begin, end);
+    const int b_first = cur.qg / it.G;
+    for (int i = threadIdx.x; i < 2 * kHistBins; i += kThreadsTC) {
+      const uint32_t c = s_hist[i];
+      const int row = b_first + i / kHistBins;
+      if (c && row < B) atomicAdd(&hist[(size_t)row * kHistBins + (i % kHistBins)], c);
+    }
+  }
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D bf16 map over [d2][d1][128] with a box of 64 x rows x 1 and 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, long long d1, long long d2, int rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {128, (cuuint64_t)d1, (cuuint64_t)d2};
+  cuuint64_t strides[2] = {256, (cuuint64_t)d1 * 256};
+  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+struct ErrAddr {
+  std::atomic<int*> ptr[64] = {};
+  cudaError_t get(int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int* p = ptr[dev].load();
+    if (!p) {
+      void* v = nullptr;
+      if ((e = cudaGetSymbolAddress(&v, g_indexer_tc_error)) != cudaSuccess) return e;
+      p = static_cast<int*>(v);
+      ptr[dev].store(p);
+    }
+    *out = p;
+    return cudaSuccess;
+  }
+};
+ErrAddr g_err_addr;
+
+template <int QG, bool kHist>
+cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N, long long q_pos0,
+                      float* scores, uint32_t* hist, cudaStream_t stream) {
+  using C = TcCfg<QG, kHist>;
+  CUtensorMap kmap, qmap;
+  if (!make_map(&kmap, k, N, B, kTileKeys) || !make_map(&qmap, q, (long long)T * 32, B, C::kN))
+    return cudaErrorInvalidValue;
+  int* err = nullptr;
+  cudaError_t e = g_err_addr.get(&err);
+  if (e != cudaSuccess) return e;
+  static DeviceOnce once;
+  if ((e = once.run([] {
+         return cudaFuncSetAttribute(indexer_tc_kernel<QG, kHist>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+       })) != cudaSuccess)
+    return e;
+  // items = sum over query groups of the key tiles they see
+  const int G = (T + QG - 1) / QG;
+  long long total = 0;
+  for (int j = 0; j < B * G; ++j) {
+    const int t0 = (j % G) * QG;
+    const int tl = (t0 + QG < T ? t0 + QG : T) - 1;
+    const long long v = visible_count(N, q_pos0, tl);
+    total += (v + kTileKeys - 1) / kTileKeys;
+  }
+  if (total == 0) return cudaSuccess;
+  const int grid = (int)(total < kNumSMs ? total : kNumSMs);
+  indexer_tc_kernel<QG, kHist><<<grid, kThreadsTC, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
+                                                                       hist, err);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
+                                  long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream) {
+  // the fused histogram keeps two row slots per CTA: with contiguous item ranges over
+  // at most 148 CTAs a range spans at most two sequences when B <= 148
+  if (hist && (T != 1 || B > kNumSMs)) return cudaErrorNotSupported;
+  if (T == 1) {
+    return hist ? launch_tc<1, true>(q, w, k, B, T, N, q_pos0, scores, hist, stream)
+                : launch_tc<1, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, stream);
+  }
+  return launch_tc<8, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, stream);
+}
+
+cudaError_t indexer_tc_device_error(int* code, bool clear) {
+  int* p = nullptr;
+  cudaError_t e = g_err_addr.get(&p);
+  if (e != cudaSuccess) return e;
+  if ((e = cudaMemcpy(code, p, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess) return e;
+  if (clear && *code) e = cudaMemset(p, 0, sizeof(int));
+  return e;
+}
+
+}  // namespace dsa

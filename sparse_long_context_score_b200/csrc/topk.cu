@@ -97,28 +97,68 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
   return r;
 }
 
+constexpr int kRadixBins = 2048;  // digits of the resolve: 10, 10, 11, 11, 10 bits
+
 struct SelectSmem {
-  uint32_t radix[256];
+  uint32_t radix[kRadixBins];
   uint32_t warp_tmp[32];
   uint32_t total;
-  uint32_t bstar, above, remaining, digit, digit_count, is_last;
-  unsigned long long prefix;
+  uint32_t digit, digit_above, digit_count, is_last;
   uint64_t cand[kCandCap];
 };
 
-// Radix passes over the low 52 bits of the threshold-bin composites.  `get(i, c)` yields
-// element i's composite (returns false if element i is not in the threshold bin).
+// Digit search: with `bins` counts (bins <= 8 * kSelThreads), find the
+// digit d where the count from the top reaches r:  above(d) < r <= above(d) + count(d).
+// Every thread of the block must call it; results land in sm.digit / digit_above /
+// digit_count.
+template <class Load>
+__device__ __forceinline__ void find_digit(SelectSmem& sm, int bins, uint32_t r, Load load) {
+  const int per = bins > kSelThreads ? bins / kSelThreads : 1;
+  const int hi = bins - (int)threadIdx.x * per;  // this thread owns bins [hi - per, hi)
+  uint32_t local[8];
+  uint32_t lsum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = hi - 1 - i;
+    local[i] = (i < per && b >= 0) ? load(b) : 0u;
+    lsum += local[i];
+  }
+  if (threadIdx.x == 0) {
+    sm.digit = 0;
+    sm.digit_above = 0;
+    sm.digit_count = 0;
+  }
+  const uint32_t above = block_excl_scan(lsum, sm.warp_tmp, &sm.total);
+  uint32_t run = above;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i < per && hi - 1 - i >= 0 && run < r && run + local[i] >= r) {
+      sm.digit = (uint32_t)(hi - 1 - i);
+      sm.digit_above = run;
+      sm.digit_count = local[i];
+    }
+    run += local[i];
+  }
+  __syncthreads();
+}
+
+// Radix passes over the low 52 bits of the threshold-bin composites (key bits 19..0,
+// then the inverted index).  `get(i, c)` yields element i's composite, or false when
+// element i is not in the threshold bin.  Returns the threshold: the selected elements
+// are exactly those whose composite is >= it.
 template <class Get>
 __device__ uint64_t resolve_threshold(SelectSmem& sm, long long count, uint32_t remaining, Get get) {
+  constexpr int kWidths[5] = {10, 10, 11, 11, 10};
   unsigned long long prefix = 0;
   int shift = 52;
-  while (true) {
-    const int width = shift >= 8 ? 8 : shift;
+#pragma unroll 1
+  for (int pass = 0; pass < 5; ++pass) {
+    const int width = kWidths[pass];
+    const int hi_shift = shift;
     shift -= width;
     const uint32_t mask = (1u << width) - 1u;
-    for (int i = threadIdx.x; i < 256; i += kSelThreads) sm.radix[i] = 0;
+    for (int i = threadIdx.x; i < (1 << width); i += kSelThreads) sm.radix[i] = 0;
     __syncthreads();
-    const int hi_shift = shift + width;
     for (long long i = threadIdx.x; i < count; i += kSelThreads) {
       uint64_t c;
       if (!get(i, c)) continue;
@@ -127,21 +167,10 @@ __device__ uint64_t resolve_threshold(SelectSmem& sm, long long count, uint32_t 
         atomicAdd(&sm.radix[(uint32_t)(c >> shift) & mask], 1u);
     }
     __syncthreads();
-    if (threadIdx.x == 0) {
-      uint32_t cum = 0;
-      int d = (int)mask;
-      for (; d > 0; --d) {
-        if (cum + sm.radix[d] >= remaining) break;
-        cum += sm.radix[d];
-      }
-      sm.digit = (uint32_t)d;
-      sm.digit_count = sm.radix[d];
-      sm.remaining = remaining - cum;
-    }
-    __syncthreads();
-    remaining = sm.remaining;
+    find_digit(sm, 1 << width, remaining, [&](int b) { return sm.radix[b]; });
+    remaining -= sm.digit_above;
     prefix |= (unsigned long long)sm.digit << shift;
-    const bool done = (sm.digit_count == remaining) || shift == 0;
+    const bool done = sm.digit_count == remaining;  // every element of this digit is selected
     __syncthreads();
     if (done) break;
   }
@@ -158,6 +187,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   const int nchunks = gridDim.y;
   const long long V = visible_count(N, q_pos0, row_t(row, T));
   uint32_t* state = ws.row_state + (size_t)row * kRowStateWords;
+  const int lane = threadIdx.x & 31;
 
   if (V <= k) {
     // every visible position is kept; pad the rest of the row
@@ -168,51 +198,53 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
 
   // 1. threshold bin b*: the bin where the count from the top reaches k
   const uint32_t* gh = ws.hist + (size_t)row * kHistBins;
-  constexpr int kPer = kHistBins / kSelThreads;  // 8 bins per thread
-  const int rt = kSelThreads - 1 - threadIdx.x;   // thread 0 owns the highest bins
-  uint32_t local[kPer];
-  uint32_t lsum = 0;
-#pragma unroll
-  for (int i = 0; i < kPer; ++i) {
-    local[i] = __ldcg(&gh[rt * kPer + i]);
-    lsum += local[i];
-  }
-  if (threadIdx.x == 0) {
-    sm.bstar = 0;
-    sm.above = 0;
-  }
-  // suffix sums over threads ordered from the top bin down
-  const uint32_t above_mine = block_excl_scan(lsum, sm.warp_tmp, &sm.total);
-  {
-    uint32_t run = above_mine;
-    for (int i = kPer - 1; i >= 0; --i) {
-      if (run < (uint32_t)k && run + local[i] >= (uint32_t)k) {
-        sm.bstar = (uint32_t)(rt * kPer + i);
-        sm.above = run;
-      }
-      run += local[i];
-    }
-  }
-  __syncthreads();
-  const uint32_t bstar = sm.bstar;
-  const uint32_t above = sm.above;
-  const uint32_t bcount = __ldcg(&gh[bstar]);
+  find_digit(sm, kHistBins, (uint32_t)k, [&](int b) { return __ldcg(&gh[b]); });
+  const uint32_t bstar = sm.digit;
+  const uint32_t above = sm.digit_above;
+  const uint32_t bcount = sm.digit_count;
   const bool use_cand = bcount <= (uint32_t)kCandCap;
 
-  // 2. scan this chunk
+  // 2. scan this chunk: count the elements above b*, append the elements of b*
   const float* sr = scores + (size_t)row * N;
   const long long s0 = (long long)chunk * kTopkChunk;
   const long long s1 = min(s0 + (long long)kTopkChunk, V);
   uint64_t* cand = ws.cand + (size_t)row * kCandCap;
   uint32_t n_above = 0;
-  for (long long s = s0 + threadIdx.x; s < s1; s += kSelThreads) {
-    const uint32_t key = order_key(sr[s]);
+  auto visit = [&](long long s, float v) {
+    const bool in = s < s1;
+    const uint32_t key = order_key(v);
     const uint32_t bin = key >> kHistShift;
-    if (bin > bstar) ++n_above;
-    else if (bin == bstar && use_cand) {
-      const uint32_t pos = atomicAdd(&state[RS_CAND], 1u);
-      if (pos < (uint32_t)kCandCap) cand[pos] = composite(key, (uint32_t)s);
+    n_above += (in && bin > bstar) ? 1u : 0u;
+    const bool app = in && use_cand && bin == bstar;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, app);
+    if (m) {
+      uint32_t base = 0;
+      if (lane == __ffs(m) - 1) base = atomicAdd(&state[RS_CAND], (uint32_t)__popc(m));
+      base = __shfl_sync(0xFFFFFFFFu, base, __ffs(m) - 1);
+      const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
+      if (app && pos < (uint32_t)kCandCap) cand[pos] = composite(key, (uint32_t)s);
     }
+  };
+  if ((N & 3) == 0) {
+    // 16 scores per thread as four 16-byte loads, all issued before use
+    float4 v[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const long long e = s0 + 4LL * (threadIdx.x + kSelThreads * i);
+      v[i] = e + 3 < s1 ? __ldcg(reinterpret_cast<const float4*>(sr + e))
+                        : make_float4(e < s1 ? sr[e] : 0.f, e + 1 < s1 ? sr[e + 1] : 0.f,
+                                      e + 2 < s1 ? sr[e + 2] : 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const long long e = s0 + 4LL * (threadIdx.x + kSelThreads * i);
+      visit(e, v[i].x);
+      visit(e + 1, v[i].y);
+      visit(e + 2, v[i].z);
+      visit(e + 3, v[i].w);
+    }
+  } else {
+    for (long long s = s0 + threadIdx.x; s < s0 + kTopkChunk; s += kSelThreads) visit(s, s < s1 ? sr[s] : 0.f);
   }
   (void)block_excl_scan(n_above, sm.warp_tmp, &sm.total);
   if (threadIdx.x == 0) ws.chunk_above[(size_t)row * nchunks + chunk] = sm.total;
@@ -236,7 +268,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
     });
   } else {
     thr52 = resolve_threshold(sm, V, remaining, [&](long long s, uint64_t& c) {
-      const uint32_t key = order_key(sr[s]);
+      const uint32_t key = order_key(__ldcg(&sr[s]));
       if ((key >> kHistShift) != bstar) return false;
       c = composite(key, (uint32_t)s);
       return true;
@@ -253,7 +285,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
     }
   } else {
     for (long long s = threadIdx.x; s < V; s += kSelThreads) {
-      const uint32_t key = order_key(sr[s]);
+      const uint32_t key = order_key(__ldcg(&sr[s]));
       if ((key >> kHistShift) == bstar && composite(key, (uint32_t)s) >= thr) atomicAdd(&csel[s / kTopkChunk], 1u);
     }
   }
@@ -297,32 +329,84 @@ topk_compact_kernel(const float* __restrict__ scores, int T, int N, long long q_
     base = __ldcg(&ws.chunk_off[(size_t)row * nchunks + chunk]);
   }
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  constexpr int kSeg = kTopkChunk / (kCmpThreads / 32);
+  constexpr int kWarpsC = kCmpThreads / 32;
+  constexpr int kSeg = kTopkChunk / kWarpsC;  // 1024 scores per warp
+  constexpr int kGroups = kSeg / 128;          // 8 groups of 32 lanes x 4 scores
   const long long g0 = s0 + (long long)warp * kSeg;
-  const long long g1 = min(g0 + kSeg, s1);
   const float* sr = scores + (size_t)row * N;
-  __shared__ uint32_t s_cnt[kCmpThreads / 32];
-
-  uint32_t cnt = 0;
-  for (long long s = g0; s < g1; s += 32) {
-    const long long e = s + lane;
-    bool sel = false;
-    if (e < g1) sel = take_all || composite(order_key(sr[e]), (uint32_t)e) >= thr;
-    cnt += __popc(__ballot_sync(0xFFFFFFFFu, sel));
-  }
-  if (lane == 0) s_cnt[warp] = cnt;
-  __syncthreads();
-  long long off = base;
-  for (int i = 0; i < warp; ++i) off += s_cnt[i];
+  __shared__ uint32_t s_cnt[kWarpsC];
   int32_t* out = idx_out + (size_t)row * k;
-  for (long long s = g0; s < g1; s += 32) {
-    const long long e = s + lane;
-    bool sel = false;
-    if (e < g1) sel = take_all || composite(order_key(sr[e]), (uint32_t)e) >= thr;
-    const uint32_t m = __ballot_sync(0xFFFFFFFFu, sel);
-    const long long pos = off + __popc(m & ((1u << lane) - 1u));
-    if (sel && pos < k) out[pos] = (int32_t)e;
-    off += __popc(m);
+
+  auto sel = [&](long long e, float v) {
+    return e < s1 && (take_all || composite(order_key(v), (uint32_t)e) >= thr);
+  };
+
+  if ((N & 3) == 0) {
+    float4 v[kGroups];
+#pragma unroll
+    for (int i = 0; i < kGroups; ++i) {
+      const long long e = g0 + 128LL * i + 4 * lane;
+      v[i] = e + 3 < s1 ? __ldcg(reinterpret_cast<const float4*>(sr + e))
+                        : make_float4(e < s1 ? sr[e] : 0.f, e + 1 < s1 ? sr[e + 1] : 0.f,
+                                      e + 2 < s1 ? sr[e + 2] : 0.f, 0.f);
+    }
+    uint32_t bits[kGroups];
+    uint32_t total = 0;
+#pragma unroll
+    for (int i = 0; i < kGroups; ++i) {
+      const long long e = g0 + 128LL * i + 4 * lane;
+      bits[i] = (sel(e, v[i].x) ? 1u : 0u) | (sel(e + 1, v[i].y) ? 2u : 0u) | (sel(e + 2, v[i].z) ? 4u : 0u) |
+                (sel(e + 3, v[i].w) ? 8u : 0u);
+      uint32_t c = __popc(bits[i]);
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, c, o);
+        if (lane >= o) c += y;
+      }
+      total += __shfl_sync(0xFFFFFFFFu, c, 31);
+    }
+    if (lane == 0) s_cnt[warp] = total;
+    __syncthreads();
+    long long off = base;
+    for (int w = 0; w < warp; ++w) off += s_cnt[w];
+#pragma unroll
+    for (int i = 0; i < kGroups; ++i) {
+      const uint32_t c = __popc(bits[i]);
+      uint32_t incl = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      const long long e = g0 + 128LL * i + 4 * lane;
+      long long pos = off + incl - c;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (bits[i] & (1u << j)) {
+          if (pos < k) out[pos] = (int32_t)(e + j);
+          ++pos;
+        }
+      off += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+  } else {
+    const long long g1 = min(g0 + kSeg, s1);
+    uint32_t cnt = 0;
+    for (long long s = g0; s < g1; s += 32) {
+      const long long e = s + lane;
+      cnt += __popc(__ballot_sync(0xFFFFFFFFu, e < g1 && sel(e, sr[e])));
+    }
+    if (lane == 0) s_cnt[warp] = cnt;
+    __syncthreads();
+    long long off = base;
+    for (int w = 0; w < warp; ++w) off += s_cnt[w];
+    for (long long s = g0; s < g1; s += 32) {
+      const long long e = s + lane;
+      const bool p = e < g1 && sel(e, sr[e]);
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, p);
+      const long long pos = off + __popc(m & ((1u << lane) - 1u));
+      if (p && pos < k) out[pos] = (int32_t)e;
+      off += __popc(m);
+    }
   }
 }
 
