@@ -7,7 +7,8 @@ One step = one pass of the whole hot path over one batch: the indexer over the i
 cache, the top-k select, and sparse MLA attention for the 4 layers of the group (all
 IndexShare groups of the workload in sequence).  Inputs are seeded synthetic tensors
 generated in HBM before timing; the step is captured once in a CUDA graph and replayed.
-L2 is flushed (a 512 MiB write) before every timed step and the step alone is timed with
+L2 is flushed (a 512 MiB write, then a 512 MiB read that evicts the dirty lines) before
+every timed step and the step alone is timed with
 CUDA events on the launching stream.  Under torchrun every rank runs its own batch
 (weak scaling, no data-path collective) and rank 0 reports the max over ranks.
 """
@@ -39,14 +40,24 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--cpu-sample", type=int, default=2, help="sequences in the CPU-oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-extra", action="store_true", help="skip the 1M / MTP / prefill workloads")
     return p.parse_args()
 
 
 def algorithmic(w):
-    """Algorithmic HBM bytes of one step, and of one indexer launch."""
-    idx_launch = w.B * w.T * INDEXER_BYTES_PER_QUERY + w.B * w.T * w.N * 4 + w.B * w.N * 128 * 2
-    attn = w.B * w.T * w.L * (w.k * ROW_BYTES + w.H * 576 * 2 + w.H * 512 * 4)
+    """Algorithmic HBM bytes of one step, and of one indexer launch.  The indexer reads the
+    visible index keys once per query group and writes one score per visible key; the
+    attention gathers k rows per (query, layer, draft step) and writes the outputs."""
+    vis = min(w.N, w.q_pos0 + w.T)
+    idx_launch = w.B * w.T * INDEXER_BYTES_PER_QUERY + w.B * w.T * vis * 4 + w.B * vis * 128 * 2
+    attn = w.B * w.T * w.L * w.steps * (w.k * ROW_BYTES + w.H * 576 * 2 + w.H * 512 * 4)
     return w.groups * (idx_launch + attn + w.B * w.T * w.k * 4), idx_launch
+
+
+def prefill_indexer_flops(w):
+    """Tensor FLOPs of the prefill indexer: 2 * 32 heads * 128 dims per (query, visible key)."""
+    pairs = sum(min(w.N, w.q_pos0 + t + 1) for t in range(w.T))
+    return w.B * pairs * 2 * 32 * 128
 
 
 def peaks():
@@ -56,6 +67,14 @@ def peaks():
         return float(m["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def _bf16_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            return float(json.load(fh)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def profiled_traffic(kernel_src: str, workload: str):
@@ -144,27 +163,44 @@ def make_inputs(w, device, rank):
             qs.append(q)
         idx = torch.empty(w.B, w.T, w.k, dtype=torch.int32, device=device)
         outs = [torch.empty(w.B, w.T, w.H, 512, dtype=torch.float32, device=device) for _ in range(w.L)]
-        groups.append(dict(ik=ik, kvs=kvs, iq=iq, wt=wt, qs=qs, idx=idx, outs=outs))
+        draft_qs = []
+        for st in range(1, w.steps):
+            qd = torch.empty(w.B, w.T, w.H, 576, dtype=bf, device=device)
+            sd.normal_bf16(qd, w.key(synth.KIND_Q, g, 0, st) ^ rank)
+            draft_qs.append(qd)
+        groups.append(dict(ik=ik, kvs=kvs, iq=iq, wt=wt, qs=qs, idx=idx, outs=outs, draft_qs=draft_qs))
     return groups
 
 
-def run_ours(args, rank, world, device):
+def run_ours(args, rank, world, device, w=None, e2e=True):
     import torch
     import sparse_long_context_score_b200 as dsa
     from synth import configs as C
 
-    w = C.WORKLOADS[args.workload]
+    w = w or C.WORKLOADS[args.workload]
     torch.cuda.set_device(device)
     dsa.lib()
     groups = make_inputs(w, device, rank)
     ws = dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, device)
     stream = torch.cuda.Stream(device)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(512 << 20, dtype=torch.uint8, device=device)
+
+    def flush_l2():
+        # write a buffer larger than L2, then read another: the dirty lines of the write are
+        # evicted (written back) by the read, before the timed region, not during it
+        flush.zero_()
+        flush_rd.view(torch.int64).sum()
 
     def step():
         for g in groups:
             dsa.dsa_group_forward(g["iq"], g["wt"], g["ik"], g["qs"], g["kvs"], w.q_pos0, w.k, C.SCALE,
                                   idx_shared=g["idx"], outs=g["outs"], ws=ws, stream=stream)
+            # MTP draft steps 2..: the step-1 index list and the target cache are reused
+            for qd in g.get("draft_qs", []):
+                dsa.dsa_group_forward(None, None, None, [qd], g["kvs"], w.q_pos0, w.k, C.SCALE,
+                                      compute_indices=False, idx_shared=g["idx"], outs=g["outs"], ws=ws,
+                                      stream=stream)
 
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
@@ -178,13 +214,13 @@ def run_ours(args, rank, world, device):
     def timed(fn, K, W):
         with torch.cuda.stream(stream):
             for _ in range(W):
-                flush.zero_()
+                flush_l2()
                 fn()
         torch.cuda.synchronize()
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
         with torch.cuda.stream(stream):
             for a, b in ev:
-                flush.zero_()
+                flush_l2()
                 a.record(stream)
                 fn()
                 b.record(stream)
@@ -204,18 +240,31 @@ def run_ours(args, rank, world, device):
     # the dominant kernel alone: the indexer over the first group's cache, same launch shape
     g0 = groups[0]
     scores = torch.empty(w.B, w.T, w.N, dtype=torch.float32, device=device)
-    idx_times = timed(lambda: dsa.dsa_index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores,
-                                                  stream=stream), args.steps, args.warmup)
+    # captured in a graph like the step, so the host-side set-up of a launch (tensor-map
+    # encoding) is not inside the timed region
+    with torch.cuda.stream(stream):
+        dsa.dsa_index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores, stream=stream)
+    torch.cuda.synchronize()
+    igraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(igraph, stream=stream):
+        dsa.dsa_index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores, stream=stream)
+    torch.cuda.synchronize()
+    idx_times = timed(igraph.replay, args.steps, args.warmup)
     idx_ms = sum(idx_times) / len(idx_times)
+
+    if not e2e:
+        del groups, ws, flush, flush_rd, scores, graph, igraph
+        torch.cuda.empty_cache()
+        return w, step_ms, idx_ms, None, 0, 0, clk.summary()
 
     # end to end through the public API with host buffers: per step, the step's query-side
     # inputs go host -> device from pinned memory and the outputs come back
-    pinned_in = [[t.cpu().pin_memory() for t in [g["iq"], g["wt"], *g["qs"]]] for g in groups]
+    pinned_in = [[t.cpu().pin_memory() for t in [g["iq"], g["wt"], *g["qs"], *g["draft_qs"]]] for g in groups]
     pinned_out = [[torch.empty_like(t, device="cpu").pin_memory() for t in [g["idx"], *g["outs"]]] for g in groups]
 
     def e2e_step():
         for g, pin, pout in zip(groups, pinned_in, pinned_out):
-            for dst, src in zip([g["iq"], g["wt"], *g["qs"]], pin):
+            for dst, src in zip([g["iq"], g["wt"], *g["qs"], *g["draft_qs"]], pin):
                 dst.copy_(src, non_blocking=True)
         graph.replay()
         for g, pout in zip(groups, pinned_out):
@@ -317,7 +366,7 @@ def main():
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "T": w.T, "N": w.N, "k": w.k, "H": w.H, "L": w.L,
-                   "groups": w.groups, "l2": "flushed (512 MiB write) before every timed step",
+                   "groups": w.groups, "l2": "flushed before every timed step (512 MiB write, then a 512 MiB read so the write-back is not timed)",
                    "parallelism": f"dp{world}" if world > 1 else "single GPU",
                    "step_hbm_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
                    "step_roofline_frac": step_bytes / (step_ms * 1e-3) / 1e9 / peak},
@@ -330,6 +379,24 @@ def main():
                      "traffic": profiled_traffic("indexer.cu", w.name), "launch_us": idx_ms * 1e3,
                      "algorithmic_bytes_per_launch": idx_bytes},
     }
+    if not args.no_extra and args.workload == "decode128k":
+        extra = {}
+        for name in ("decode1m", "mtp", "prefill"):
+            we = C.WORKLOADS[name]
+            _, ms, ims, _, _, _, clk2 = run_ours(args, rank, world, device, w=we, e2e=False)
+            b2, ib2 = algorithmic(we)
+            toks = we.B * we.T * (we.steps if we.steps > 1 else 1) * world
+            ent = {"tokens_per_s": toks / (ms * 1e-3), "ms_per_step": ms, "step_hbm_gbs": b2 / (ms * 1e-3) / 1e9,
+                   "step_roofline_frac": b2 / (ms * 1e-3) / 1e9 / peak, "indexer_launch_us": ims * 1e3,
+                   "indexer_hbm_gbs": ib2 / (ims * 1e-3) / 1e9, "clocks_sm_mhz": clk2.get("sm_mhz"),
+                   "clock_reasons": clk2.get("reasons")}
+            if name == "prefill":
+                fl = prefill_indexer_flops(we)
+                ent["indexer_tflops"] = fl / (ims * 1e-3) / 1e12
+                ent["indexer_tensor_frac_of_measured_bf16"] = ent["indexer_tflops"] / _bf16_peak()
+                ent["tokens_per_s"] = we.B * we.T * world / (ms * 1e-3)
+            extra[name] = ent
+        line["config"]["other_workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
     if rank == 0:

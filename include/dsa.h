@@ -22,8 +22,9 @@
  *
  * Conventions for every entry point
  *   - Tensors are caller-owned DEVICE pointers, dense row-major, in the layouts given.
- *     bf16 tensors are passed as uint16_t bit patterns.  bf16 tensors and the score,
- *     output and workspace buffers must be 16-byte aligned; float/int tensors 4-byte.
+ *     bf16 tensors are passed as uint16_t bit patterns.  bf16 tensors, the head weights,
+ *     the output buffers and the workspace must be 16-byte aligned (the workspace
+ *     256-byte); scores and index lists 4-byte.
  *   - Calls are asynchronous: work is enqueued on `stream` and the call returns.  The
  *     library allocates no memory and keeps no per-call state; scratch memory is the
  *     caller's `workspace` (size from dsa_workspace_size).
@@ -119,7 +120,7 @@ dsa_status dsa_topk(const float *scores, int B, int T, int N, long long q_pos0, 
  * scratch is a fixed DSA_NOALLOC_SCRATCH_BYTES array inside the library, held on every
  * GPU that loads the library until the process exits.
  *   - Sizes whose select needs more scratch than that return DSA_ERR_WORKSPACE: at most
- *     25 query rows (B*T) for N up to 1,048,576 (fewer for longer rows); use dsa_topk
+ *     23 query rows (B*T) for N up to 1,048,576 (fewer for longer rows); use dsa_topk
  *     beyond that.
  *   - The first call on a device looks up the array's device address (a runtime call,
  *     not an allocation); make that first call before any stream capture.

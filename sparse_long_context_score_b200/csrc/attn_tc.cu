@@ -14,16 +14,18 @@
 // rescaling is rare; exponentials may then exceed 1 by at most 2^8, which f32 and bf16
 // carry without loss of relative precision.
 //
-// Warp roles (288 threads):
-//   warps 0..3  gather: the selected rows as 16-byte cp.async chunks written straight into
-//               the 128-byte-swizzled tensor-core layout; warp w owns stage w and tiles
-//               w, w+4, ..., waits for its own copies, fences them to the async proxy and
-//               arrives on the stage barrier, so four tiles are in flight and each is
-//               published as soon as it lands (one TMA load brings the 64 query rows).  Random 1152-byte rows are too small for TMA: a
+// Warp roles (416 threads):
+//   warps 0..7  gather: the selected rows as 16-byte cp.async chunks written straight into
+//               the 128-byte-swizzled tensor-core layout; warps 2s, 2s+1 own stage s
+//               (16 rows each) and tiles s, s+4, ..., wait for their own copies, fence
+//               them to the async proxy and arrive on the stage barrier, so four tiles are
+//               in flight and each is published as soon as it lands (one TMA load brings
+//               the 64 query rows).  Issue parallelism matters: a random-row gather probe
+//               reached ~3.1 TB/s with 4 warps and ~3.9 TB/s with 6 on 128 SMs.  Random 1152-byte rows are too small for TMA: a
 //               4-row gather copy per 512 bytes ran latency-bound on B200.
-//   warp 4      TMEM allocation; one thread issues S(i) and then O += P(i-1) V(i-1), so
-//               the softmax of one tile overlaps the next tile's logits;
-//   warps 5..8  softmax (threads on lanes 0..15 of each warp own a head), P as bf16 in
+//   warp 8      TMEM allocation; one elected lane issues S(i) and then O += P(i-1) V(i-1),
+//               so the softmax of one tile overlaps the next tile's logits;
+//   warps 9..12 softmax (threads on lanes 0..15 of each warp own a head), P as bf16 in
 //               shared memory, and at the end the read-out of O^T (lane = value dim) into
 //               shared memory and one bulk (TMA) store of the [H][512] output block --
 //               per-thread 4-byte global stores of that block ran at a few GB/s from an SM
@@ -50,21 +52,23 @@ constexpr int kQBlockBytes = 64 * 128;           // 64 heads x 64 bf16
 constexpr int kBlockBytes = kKeys * 128;         // 32 rows x 64 bf16
 constexpr int kQBytes = kBlocks * kQBlockBytes;  // 73728
 constexpr int kStageBytes = kBlocks * kBlockBytes;  // 36864
-constexpr int kPBytes = 64 * 128;                // 64 heads x 128-byte rows (first 64 bytes used)
-constexpr int kThreadsA = 288;
-constexpr int kChunksPerTile = kKeys * (kDqk / 8);  // 16-byte chunks: 2304
+constexpr int kPBytes = 64 * kKeys * 2;          // one P buffer: 64 heads x 64-byte rows (4 KB)
+constexpr int kProducerWarps = 8;                // two warps per stage, 16 rows each
+constexpr int kMmaWarp = kProducerWarps;
+constexpr int kSoftmaxWarp0 = kProducerWarps + 1;
+constexpr int kThreadsA = (kProducerWarps + 5) * 32;  // 416
 constexpr float kRescaleLog2 = 8.f;
 
 constexpr int kOffQ = 0;
 constexpr int kOffStage = kOffQ + kQBytes;
 constexpr int kOffP = kOffStage + kStages * kStageBytes;
-constexpr int kOffAlpha = kOffP + kPBytes;       // [2][64] f32 (tile parity)
+constexpr int kOffAlpha = kOffP + 2 * kPBytes;   // [2][64] f32 (tile parity)
 constexpr int kOffL = kOffAlpha + 2 * 64 * 4;    // [64] f32
 constexpr int kOffM = kOffL + 64 * 4;            // [64] f32
-constexpr int kOffMask = kOffM + 64 * 4;         // [kStages] u32
-constexpr int kOffRows = kOffMask + kStages * 4; // [kStages][kKeys] int
-constexpr int kNumBars = 2 * kStages + 9;
-constexpr int kOffBar = kOffRows + kStages * kKeys * 4;
+constexpr int kOffMask = kOffM + 64 * 4;         // [kStages][2] u16 (one half per producer warp)
+constexpr int kOffFlag = kOffMask + kStages * 4;   // u32: this CTA merges the splits
+constexpr int kNumBars = 2 * kStages + 11;
+constexpr int kOffBar = kOffFlag + 16;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmemA = kOffTmem + 16 + 1024;
 static_assert(kSmemA <= 232448, "shared memory budget");
@@ -79,7 +83,8 @@ struct AttnMaps {
 
 __global__ void __launch_bounds__(kThreadsA, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const int32_t* __restrict__ idx, int T, int N,
-               int H, int k, int chunk, float scale_log2, float* __restrict__ partial, int* __restrict__ err) {
+               int H, int k, int chunk, float scale_log2, float* __restrict__ partial, uint32_t* __restrict__ tickets,
+               int* __restrict__ err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -89,18 +94,18 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   float* s_alpha = reinterpret_cast<float*>(smem + kOffAlpha);
   float* s_l = reinterpret_cast<float*>(smem + kOffL);
   float* s_m = reinterpret_cast<float*>(smem + kOffM);
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(smem + kOffMask);
-  int* s_rows = reinterpret_cast<int*>(smem + kOffRows);
+  uint16_t* s_mask = reinterpret_cast<uint16_t*>(smem + kOffMask);
+  uint32_t* s_last = reinterpret_cast<uint32_t*>(smem + kOffFlag);
   const uint32_t bar0 = sbase + kOffBar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
   auto sfull_bar = [&](int s) { return bar0 + 8u * (2 * kStages + s); };
   auto sfree_bar = [&](int s) { return bar0 + 8u * (2 * kStages + 2 + s); };
-  const uint32_t pfull_bar = bar0 + 8u * (2 * kStages + 4);
-  const uint32_t pfree_bar = bar0 + 8u * (2 * kStages + 5);
-  const uint32_t ofinal_bar = bar0 + 8u * (2 * kStages + 6);
-  const uint32_t qfull_bar = bar0 + 8u * (2 * kStages + 7);
-  const uint32_t grp_bar = bar0 + 8u * (2 * kStages + 8);
+  auto pfull_bar = [&](int pb) { return bar0 + 8u * (2 * kStages + 4 + pb); };
+  auto pfree_bar = [&](int pb) { return bar0 + 8u * (2 * kStages + 6 + pb); };
+  const uint32_t ofinal_bar = bar0 + 8u * (2 * kStages + 8);
+  const uint32_t qfull_bar = bar0 + 8u * (2 * kStages + 9);
+  const uint32_t grp_bar = bar0 + 8u * (2 * kStages + 10);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
 
   const int split = blockIdx.x, row = blockIdx.y, layer = blockIdx.z;
@@ -113,22 +118,25 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(full_bar(s), 32);
+      mbar_init(full_bar(s), 64);
       mbar_init(empty_bar(s), 1);
     }
     for (int s = 0; s < 2; ++s) {
       mbar_init(sfull_bar(s), 1);
       mbar_init(sfree_bar(s), 128);
     }
-    mbar_init(pfull_bar, 128);
-    mbar_init(pfree_bar, 1);
+    for (int pb = 0; pb < 2; ++pb) {
+      mbar_init(pfull_bar(pb), 128);
+      mbar_init(pfree_bar(pb), 1);
+    }
     mbar_init(ofinal_bar, 1);
     mbar_init(qfull_bar, 1);
     mbar_init(grp_bar, 128);
+    *s_last = 0;
     fence_mbar_init();
     tma_prefetch(&maps.q[layer]);
   }
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tmem_alloc(smem_u32(s_tmem), kTmemCols);
     tmem_relinquish();
   }
@@ -137,45 +145,52 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   tc_fence_after();
   const uint32_t tmem = *s_tmem;
 
-  if (warp < 4) {
+  if (warp < kProducerWarps) {
     // ------------------------------------------------------------------ gather
-    // warp pw owns stage pw and fills tiles pw, pw + 4, ...: four tiles in flight, each
-    // published as soon as its own rows have landed
-    const int pw = warp;
-    if (pw == 0 && lane == 0) {
+    // warps 2s and 2s+1 own stage s and fill rows [0,16) and [16,32) of tiles s, s+4, ...;
+    // each waits for its own copies, fences them to the async proxy and arrives, so
+    // four tiles are in flight and each is published as soon as it lands
+    const int ps = warp >> 1, half = warp & 1;
+    if (warp == 0 && lane == 0) {
       const CUtensorMap* qm = &maps.q[layer];
       mbar_arrive_expect_tx(qfull_bar, kQBytes);
       for (int kb = 0; kb < kBlocks; ++kb) tma_load_2d(sQ + kb * kQBlockBytes, qm, qfull_bar, 64 * kb, row * H);
     }
     const int32_t* sel = idx + (size_t)row * k + j0;
     const uint16_t* kvb = layers.kv[layer] + (size_t)b * N * kDqk;
-    int* rows = s_rows + pw * kKeys;
-    const uint32_t st = sStage + pw * kStageBytes;
-    for (int i = pw; i < ntiles; i += kStages) {
+    const uint32_t st = sStage + ps * kStageBytes;
+    // this lane copies 16-byte chunks lane, lane+32, lane+64 (< 72) of every row: the
+    // column block and in-row offset of each are constants
+    const int c0 = lane, c1 = lane + 32, c2 = lane + 64;
+    const uint32_t kb0 = (c0 >> 3) * kBlockBytes, kb1 = (c1 >> 3) * kBlockBytes, kb2 = (c2 >> 3) * kBlockBytes;
+    for (int i = ps; i < ntiles; i += kStages) {
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(empty_bar(pw), ((i / kStages) & 1) ^ 1, err, 21);
+      if (lane == 0) ok = mbar_wait(empty_bar(ps), ((i / kStages) & 1) ^ 1, err, 21);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
-      const int key = i * kKeys + lane;
+      const int key = i * kKeys + 16 * half + (lane & 15);
       const int v = key < nkeys ? __ldg(&sel[key]) : -1;
       const bool valid = v >= 0 && v < N;
-      rows[lane] = valid ? v : 0;
-      const uint32_t m = __ballot_sync(0xFFFFFFFFu, valid);
-      if (lane == 0) s_mask[pw] = m;
-      __syncwarp();
-#pragma unroll 8
-      for (int c = lane; c < kChunksPerTile; c += 32) {
-        const int r = c / (kDqk / 8), cc = c - r * (kDqk / 8);
-        const uint32_t dst = st + (cc >> 3) * kBlockBytes + r * 128 + (((cc & 7) ^ (r & 7)) << 4);
-        cp_async_16(dst, kvb + (size_t)rows[r] * kDqk + cc * 8, 16);
+      const int my_row = valid ? v : 0;
+      const uint32_t m = __ballot_sync(0xFFFFFFFFu, valid) & 0xFFFFu;
+      if (lane == 0) s_mask[2 * ps + half] = (uint16_t)m;
+#pragma unroll 4
+      for (int rr = 0; rr < 16; ++rr) {
+        const int r = 16 * half + rr;
+        const uint16_t* src = kvb + (size_t)__shfl_sync(0xFFFFFFFFu, my_row, rr) * kDqk;
+        const uint32_t rbase = st + r * 128;
+        const int x = r & 7;
+        cp_async_16(rbase + kb0 + (((c0 & 7) ^ x) << 4), src + c0 * 8, 16);
+        cp_async_16(rbase + kb1 + (((c1 & 7) ^ x) << 4), src + c1 * 8, 16);
+        if (c2 < kDqk / 8) cp_async_16(rbase + kb2 + (((c2 & 7) ^ x) << 4), src + c2 * 8, 16);
       }
       cp_async_commit();
       cp_async_wait<0>();
       fence_proxy_async();  // the copies are visible to the tensor core (async proxy)
-      mbar_arrive(full_bar(pw));
+      mbar_arrive(full_bar(ps));
     }
-    if (pw == 0 && lane == 0) mbar_wait_drain(qfull_bar, 0);
-  } else if (warp == 4) {
+    if (warp == 0 && lane == 0) mbar_wait_drain(qfull_bar, 0);
+  } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA issuer
     // the whole warp runs the loop (descriptor arithmetic stays warp-uniform); one
     // elected lane issues the tensor-core instructions
@@ -184,7 +199,6 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true, false);  // V^T (M-major) x P (K-major)
     bool ok = mbar_wait(qfull_bar, 0, err, 22);
     const uint64_t dq = sdesc_kmajor_sw128(sQ);
-    const uint64_t dp = sdesc_kmajor_sw128(sP);
     for (int i = 0; i <= ntiles && ok; ++i) {
       if (i < ntiles) {
         const int s = i % kStages, sb = i & 1;
@@ -205,11 +219,12 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         __syncwarp();
       }
       if (i >= 1) {
-        const int jt = i - 1, sj = jt % kStages;
-        ok = mbar_wait(pfull_bar, jt & 1, err, 25);
+        const int jt = i - 1, sj = jt % kStages, pb = jt & 1;
+        ok = mbar_wait(pfull_bar(pb), (jt >> 1) & 1, err, 25);
         if (!ok) break;
         tc_fence_after();
         const uint64_t da = sdesc_mnmajor_sw128(sStage + sj * kStageBytes, kBlockBytes, 1024);
+        const uint64_t dp = sdesc_kmajor_sw64(sP + pb * kPBytes);
         const uint32_t first = jt > 0 ? 1u : 0u;
         if (leader) {
 #pragma unroll
@@ -218,7 +233,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
             for (int ks = 0; ks < kKeys / 16; ++ks)
               mma_bf16(tmem + kTmemO + 64 * mb, da + (uint64_t)(((2 * mb) * kBlockBytes + ks * 16 * 128) >> 4),
                        dp + (uint64_t)((ks * 32) >> 4), idPV, first | (ks > 0 ? 1u : 0u));
-          mma_commit(pfree_bar);
+          mma_commit(pfree_bar(pb));
           mma_commit(empty_bar(sj));
         }
         __syncwarp();
@@ -232,7 +247,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   } else {
     // ------------------------------------------------------------------ softmax + read-out
     const int quarter = warp & 3;
-    const int st_tid = threadIdx.x - 160;         // 0..127
+    const int st_tid = threadIdx.x - 32 * kSoftmaxWarp0;  // 0..127
     const bool owner = lane < 16;                 // this thread's TMEM lane holds a head of S
     const int head = 16 * quarter + (lane & 15);
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
@@ -251,7 +266,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
       mbar_arrive(sfree_bar(sb));
       ok = mbar_wait(full_bar(s), (i / kStages) & 1, err, 28);  // orders the gather's mask write
       if (!ok) break;
-      const uint32_t mask = s_mask[s];
+      const uint32_t mask = (uint32_t)s_mask[2 * s] | ((uint32_t)s_mask[2 * s + 1] << 16);
       float* alpha = s_alpha + 64 * (i & 1);
       float mt = -INFINITY;
 #pragma unroll
@@ -272,29 +287,33 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
       ok = mbar_wait(grp_bar, grp_phase, err, 29);
       grp_phase ^= 1;
       if (!ok) break;
-      if (i > 0) {
-        ok = mbar_wait(pfree_bar, (i - 1) & 1, err, 30);  // O^T and P are no longer in use
+      bool any = false;
+#pragma unroll 8
+      for (int h = 0; h < 64; ++h) any |= h < H && alpha[h] != 1.f;
+      if (i > 0 && any) {
+        // O^T is rescaled only once the previous tile's PV has finished with it
+        ok = mbar_wait(pfree_bar((i - 1) & 1), ((i - 1) >> 1) & 1, err, 30);
         if (!ok) break;
         tc_fence_after();
-        bool any = false;
-#pragma unroll 8
-        for (int h = 0; h < 64; ++h) any |= h < H && alpha[h] != 1.f;
-        if (any) {
-          // rescale O^T: this thread's lane is one value dim, its columns the heads
+        // rescale O^T: this thread's lane is one value dim, its columns the heads
 #pragma unroll 1
-          for (int mb = 0; mb < 4; ++mb)
+        for (int mb = 0; mb < 4; ++mb)
 #pragma unroll 1
-            for (int half = 0; half < 2; ++half) {
-              uint32_t o[32];
-              const uint32_t ta = tmem + lane_addr + kTmemO + 64 * mb + 32 * half;
-              tmem_ld32(ta, o);
-              tmem_ld_wait();
+          for (int half = 0; half < 2; ++half) {
+            uint32_t o[32];
+            const uint32_t ta = tmem + lane_addr + kTmemO + 64 * mb + 32 * half;
+            tmem_ld32(ta, o);
+            tmem_ld_wait();
 #pragma unroll
-              for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha[32 * half + c]);
-              tmem_st32(ta, o);
-            }
-          tmem_st_wait();
-        }
+            for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha[32 * half + c]);
+            tmem_st32(ta, o);
+          }
+        tmem_st_wait();
+      }
+      if (i > 1) {
+        // P buffer i&1 was last read by PV(i-2)
+        ok = mbar_wait(pfree_bar(i & 1), ((i >> 1) & 1) ^ 1, err, 34);
+        if (!ok) break;
       }
       if (owner) {
         const float mu = m_used == -INFINITY ? 0.f : m_used;
@@ -308,16 +327,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
           packed[j / 2] = pack_bf16x2(p0, p1);
         }
         l_run += ls;
-        // P row `head`: 32 keys in the first 64 bytes of a 128-byte swizzled row (K-major)
-        unsigned char* prow = smem + kOffP + head * 128;
+        // P row `head` of buffer i&1: 32 keys = 64 bytes, K-major with the 64-byte swizzle
+        unsigned char* prow = smem + kOffP + (i & 1) * kPBytes + head * 64;
 #pragma unroll
         for (int c = 0; c < kKeys / 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ (head & 7)) << 4)) =
+          *reinterpret_cast<uint4*>(prow + ((c ^ ((head >> 1) & 3)) << 4)) =
               make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
         fence_proxy_async();
       }
       tc_fence_before();
-      mbar_arrive(pfull_bar);
+      mbar_arrive(pfull_bar(i & 1));
     }
     // ------------------------------------------------------------------ read-out
     if (ok && ntiles > 0) ok = mbar_wait(ofinal_bar, 0, err, 31);
@@ -372,20 +391,70 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         bulk_store(dst, smem_u32(s_out), (uint32_t)(H * kDv * 4));
         bulk_commit();
         bulk_wait_all();
+        fence_proxy_async_global();
       }
-      if (ok && nsplit > 1 && st_tid < H) {
-        float* pm = partial + unit * (size_t)H * (kDv + 2) + (size_t)H * kDv;
-        pm[2 * st_tid] = ntiles > 0 ? s_m[st_tid] : -INFINITY;
-        pm[2 * st_tid + 1] = ntiles > 0 ? s_l[st_tid] : 0.f;
+      if (ok && nsplit > 1) {
+        if (st_tid < H) {
+          float* pm = partial + unit * (size_t)H * (kDv + 2) + (size_t)H * kDv;
+          pm[2 * st_tid] = ntiles > 0 ? s_m[st_tid] : -INFINITY;
+          pm[2 * st_tid + 1] = ntiles > 0 ? s_l[st_tid] : 0.f;
+        }
+        // publish this split; the last split of the (row, layer) to arrive merges them all
+        __threadfence();
+        mbar_arrive(grp_bar);
+        grp_phase ^= 1;
+        ok = mbar_wait(grp_bar, grp_phase, err, 35);
+        if (ok && st_tid == 0) {
+          const uint32_t t = atomicAdd(&tickets[(size_t)layer * gridDim.y + row], 1u);
+          *s_last = (t == (uint32_t)nsplit - 1) ? 1u : 0u;
+        }
       }
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
+  }
+  if (nsplit > 1 && *s_last) {
+    // merge: out[h][:] = sum_s 2^(m_s - M) O_s[h][:] / sum_s 2^(m_s - M) l_s
+    __threadfence();
+    const size_t unit0 = ((size_t)layer * gridDim.y + row) * nsplit;
+    const size_t stride = (size_t)H * (kDv + 2);
+    float* coef = reinterpret_cast<float*>(smem + kOffStage);  // [nsplit][64], the stages are idle
+    if (threadIdx.x < H) {
+      const int h = threadIdx.x;
+      float M = -INFINITY;
+      for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(&partial[(unit0 + sp) * stride + (size_t)H * kDv + 2 * h]));
+      float den = 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float m = __ldcg(&partial[(unit0 + sp) * stride + (size_t)H * kDv + 2 * h]);
+        const float l = __ldcg(&partial[(unit0 + sp) * stride + (size_t)H * kDv + 2 * h + 1]);
+        const float wgt = m == -INFINITY ? 0.f : exp2f(m - M);
+        coef[sp * 64 + h] = wgt;
+        den += wgt * l;
+      }
+      const float inv = den > 0.f ? 1.f / den : 0.f;
+      for (int sp = 0; sp < nsplit; ++sp) coef[sp * 64 + h] *= inv;
+    }
+    __syncthreads();
+    float* out = layers.out[layer] + (size_t)row * H * kDv;
+    for (int e = threadIdx.x; e < H * (kDv / 4); e += kThreadsA) {
+      const int h = e / (kDv / 4), d = (e - h * (kDv / 4)) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const float c = coef[sp * 64 + h];
+        if (c == 0.f) continue;
+        const float4 o = __ldcg(reinterpret_cast<const float4*>(partial + (unit0 + sp) * stride + (size_t)h * kDv + d));
+        acc.x = fmaf(c, o.x, acc.x);
+        acc.y = fmaf(c, o.y, acc.y);
+        acc.z = fmaf(c, o.z, acc.z);
+        acc.w = fmaf(c, o.w, acc.w);
+      }
+      *reinterpret_cast<float4*>(out + (size_t)h * kDv + d) = acc;
+    }
   }
 }
 
@@ -436,6 +505,32 @@ ErrAddr g_err_addr;
 
 }  // namespace
 
+// Keys per split: a multiple of the 64-row granularity.
+int attn_split_chunk(int k, int nsplit) {
+  const int chunk = (k + nsplit - 1) / nsplit;
+  return (chunk + kAttnTile - 1) / kAttnTile * kAttnTile;
+}
+
+// Splits per (query row, layer): about one CTA per SM in total.
+int attn_num_splits(long long rows, int L, int k) {
+  const long long units = rows * L;
+  long long ns = kNumSMs / (units > 0 ? units : 1);
+  if (ns < 1) ns = 1;
+  const long long max_ns = (k + kAttnTile - 1) / kAttnTile;
+  if (ns > max_ns) ns = max_ns;
+  const int chunk = attn_split_chunk(k, (int)ns);
+  return (k + chunk - 1) / chunk;
+}
+
+size_t attn_ticket_bytes(long long rows, int L) { return ((size_t)L * rows * sizeof(uint32_t) + 255) & ~(size_t)255; }
+
+// Workspace of the split path: one ticket per (layer, row), then the split partials.
+size_t attn_workspace_bytes(long long rows, int L, int H, int k) {
+  const int ns = attn_num_splits(rows, L, k);
+  if (ns <= 1) return 0;
+  return attn_ticket_bytes(rows, L) + (size_t)L * rows * ns * H * (kDv + 2) * sizeof(float);
+}
+
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
                                   int k, float scale, void* ws, cudaStream_t stream) {
   const long long rows = (long long)B * T;
@@ -451,12 +546,13 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
     return e;
   const int nsplit = attn_num_splits(rows, L, k);
   const int chunk = attn_split_chunk(k, nsplit);
-  float* partial = static_cast<float*>(ws);
-  attn_tc_kernel<<<dim3(nsplit, (unsigned)rows, L), kThreadsA, kSmemA, stream>>>(maps, layers, idx, T, N, H, k, chunk,
-                                                                                 scale * 1.4426950408889634f, partial, err);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  if (nsplit > 1) e = launch_attn_combine(layers, L, rows, H, nsplit, partial, stream);
-  return e;
+  uint32_t* tickets = static_cast<uint32_t*>(ws);
+  float* partial = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + attn_ticket_bytes(rows, L));
+  if (nsplit > 1 && (e = cudaMemsetAsync(tickets, 0, (size_t)L * rows * sizeof(uint32_t), stream)) != cudaSuccess)
+    return e;
+  attn_tc_kernel<<<dim3(nsplit, (unsigned)rows, L), kThreadsA, kSmemA, stream>>>(
+      maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f, partial, tickets, err);
+  return cudaGetLastError();
 }
 
 cudaError_t attn_tc_device_error(int* code, bool clear) {

@@ -85,7 +85,7 @@ size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L) {
 dsa_status dsa_index_score(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
                            long long q_pos0, float* scores, cudaStream_t stream) {
   if (!q || !w || !k || !scores || !sizes_ok(B, T, N)) return DSA_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 4) || !aligned(scores, 4)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 16) || !aligned(scores, 4)) return DSA_ERR_INVALID_ARG;
   return cuda_status(launch_index_score_tc(q, w, k, B, T, N, q_pos0, scores, nullptr, stream));
 }
 
@@ -124,7 +124,7 @@ dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t*
     return DSA_ERR_INVALID_ARG;
   if (L > DSA_MAX_LAYERS || k > DSA_MAX_TOPK || !heads_supported(H)) return DSA_ERR_UNSUPPORTED;
   if (compute_indices && (!iq || !w || !ik)) return DSA_ERR_INVALID_ARG;
-  if (compute_indices && (!aligned(iq, 16) || !aligned(ik, 16) || !aligned(w, 4))) return DSA_ERR_INVALID_ARG;
+  if (compute_indices && (!aligned(iq, 16) || !aligned(ik, 16) || !aligned(w, 16))) return DSA_ERR_INVALID_ARG;
   if (!aligned(idx_shared, 4)) return DSA_ERR_INVALID_ARG;
   AttnLayers layers{};
   for (int l = 0; l < L; ++l) {

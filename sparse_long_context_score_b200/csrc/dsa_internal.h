@@ -40,13 +40,15 @@ constexpr int kHistBits = 12;
 constexpr int kHistBins = 1 << kHistBits;
 constexpr int kHistShift = 32 - kHistBits;
 constexpr int kTopkChunk = 8192;       // scores per CTA in the scan kernels
-constexpr int kCandCap = 8192;         // candidates kept per row for the in-SMEM resolve
+constexpr int kCandCap = 8192;         // candidates kept per row for the resolve
+constexpr int kHist2Bins = 1024;       // second radix digit: key bits 19..10
 constexpr int kRowStateWords = 16;
 
 struct TopkWorkspace {
   uint32_t* hist;        // [rows][kHistBins]
   uint32_t* row_state;   // [rows][kRowStateWords]
   uint32_t* chunk_sel;   // [rows][nchunks]  selected threshold-bin candidates per chunk
+  uint32_t* hist2;       // [rows][kHist2Bins] next 10 key bits of the threshold-bin elements
   uint32_t* chunk_above; // [rows][nchunks]  elements above the threshold bin per chunk
   uint32_t* chunk_off;   // [rows][nchunks]  output offset of each chunk
   uint64_t* cand;        // [rows][kCandCap] composite keys of threshold-bin elements
@@ -66,12 +68,8 @@ constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core atte
 
 int attn_num_splits(long long rows, int L, int k);
 int attn_split_chunk(int k, int nsplit);
-cudaError_t launch_attn_combine(const AttnLayers& layers, int L, long long rows, int H, int nsplit, const float* partial,
-                                cudaStream_t stream);
+size_t attn_ticket_bytes(long long rows, int L);
 size_t attn_workspace_bytes(long long rows, int L, int H, int k);
-
-cudaError_t launch_index_score(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
-                               long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream);
 
 // tcgen05 indexer (T == 1: decode, one query per MMA; T > 1: 8 queries per MMA).  With a
 // histogram pointer (decode only, B <= 148) the first radix digit of the select is counted.
@@ -83,11 +81,8 @@ cudaError_t indexer_tc_device_error(int* code, bool clear);
 cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
                         const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream);
 
-// tcgen05 attention (the product path) and the warp-level mma.sync one (kept for comparison)
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
                                   int k, float scale, void* ws, cudaStream_t stream);
-cudaError_t launch_sparse_attn_mma(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                                   int k, float scale, void* ws, cudaStream_t stream);
 cudaError_t attn_tc_device_error(int* code, bool clear);
 
 }  // namespace dsa

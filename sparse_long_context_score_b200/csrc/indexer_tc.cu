@@ -8,19 +8,21 @@
 // N = 32*QG, K = 128 (8 MMAs of K = 16).  QG = 1 for decode (the key stream is the whole
 // cost; the tensor core is ~10% busy), QG = 8 for chunked prefill (a dense contraction).
 //
-// Warp roles (192 threads, one CTA per SM, persistent over a contiguous range of
-// (query group, key tile) items):
+// Warp roles (one CTA per SM, persistent over a contiguous range of (query group, key
+// tile) items):
 //   warp 0      TMA producer: 128x128 bf16 key tiles (two 64-column boxes, 128-byte
 //               swizzle) into a ring of shared-memory stages; the query group once per
 //               group change;
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma into one of two TMEM
 //               accumulators (2 x 32*QG columns) and commits to the stage / accumulator
 //               barriers;
-//   warps 2..5  epilogue: each thread owns one key row of the accumulator (its warp's
-//               TMEM lane quarter), loads the 32 head columns of each query, applies
-//               ReLU and the head weights, sums, and stores the score (coalesced: a warp
-//               writes 32 consecutive keys).  In decode it can also count the first radix
-//               digit of each score into a per-row histogram for the top-k select.
+//   warps 2..   epilogue (4 warps in decode, 8 in prefill: two per TMEM lane quarter, each
+//               scoring 4 of the 8 queries): each thread owns one key row of the
+//               accumulator (its warp's TMEM lane quarter), loads the 32 head columns of a
+//               query, applies ReLU and the head weights, sums, and stores the score
+//               (coalesced: a warp writes 32 consecutive keys).  In decode it can also
+//               count the first radix digit of each score into a per-row histogram for the
+//               top-k select.
 // Every mbarrier wait is bounded (see sm100.cuh); a timeout sets the device error word.
 #include <cudaTypedefs.h>
 
@@ -37,12 +39,13 @@ using namespace sm100;
 static __device__ int g_indexer_tc_error;
 
 constexpr int kTileKeys = 128;
-constexpr int kThreadsTC = 192;
 constexpr int kHalfBytesA = kTileKeys * 128;  // 128 rows x 64 bf16 = 16 KB
 constexpr int kStageBytesA = 2 * kHalfBytesA;
 
 template <int QG, bool kHist>
 struct TcCfg {
+  static constexpr int kEpiWarps = QG == 1 ? 4 : 8;   // prefill: two warps per TMEM lane quarter
+  static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kN = 32 * QG;                  // MMA N
   static constexpr int kStages = QG == 1 ? 5 : 4;
   static constexpr int kHalfBytesB = kN * 128;
@@ -102,7 +105,7 @@ struct Cursor {
 };
 
 template <int QG, bool kHist>
-__global__ void __launch_bounds__(kThreadsTC, 1)
+__global__ void __launch_bounds__(TcCfg<QG, kHist>::kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                   const float* __restrict__ w, int B, int T, int N, long long q_pos0, long long total_items,
                   float* __restrict__ scores, uint32_t* __restrict__ hist, int* __restrict__ err) {
@@ -138,7 +141,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 128);
+      mbar_init(tempty_bar(b), 32 * C::kEpiWarps);
     }
     mbar_init(qfull_bar, 1);
     mbar_init(qfree_bar, 1);
@@ -152,7 +155,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     tmem_relinquish();
   }
   if (kHist)
-    for (int i = threadIdx.x; i < 2 * kHistBins; i += kThreadsTC) s_hist[i] = 0;
+    for (int i = threadIdx.x; i < 2 * kHistBins; i += C::kThreads) s_hist[i] = 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -207,34 +210,38 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = idesc_bf16_f32(kTileKeys, C::kN);
-      Cursor cur;
-      cur.start(it, begin, end);
-      int stage = 0;
-      uint32_t phase = 0, qfull_phase = 0;
-      long long acc = 0;
-      int cur_qg = -1;
-      bool ok = true;
-      while (cur.valid() && ok) {
-        if (cur.qg != cur_qg) {
-          if (cur_qg >= 0) mma_commit(qfree_bar);
-          ok = mbar_wait(qfull_bar, qfull_phase, err, 4);
-          qfull_phase ^= 1;
-          if (!ok) break;
-          cur_qg = cur.qg;
-        }
-        const int buf = (int)(acc & 1);
-        const uint32_t use = (uint32_t)(acc >> 1);
-        ok = mbar_wait(tempty_bar(buf), (use & 1) ^ 1, err, 5);
+    // the whole warp runs the loop (descriptor arithmetic stays warp-uniform); one
+    // elected lane issues the tensor-core instructions
+    const bool leader = elect_one();
+    constexpr uint32_t idesc = idesc_bf16_f32(kTileKeys, C::kN);
+    Cursor cur;
+    cur.start(it, begin, end);
+    int stage = 0;
+    uint32_t phase = 0, qfull_phase = 0;
+    long long acc = 0;
+    int cur_qg = -1;
+    bool ok = true;
+    const uint64_t bd0 = sdesc_kmajor_sw128(sB);
+    while (cur.valid() && ok) {
+      if (cur.qg != cur_qg) {
+        if (cur_qg >= 0 && leader) mma_commit(qfree_bar);
+        __syncwarp();
+        ok = mbar_wait(qfull_bar, qfull_phase, err, 4);
+        qfull_phase ^= 1;
         if (!ok) break;
-        tc_fence_after();
-        ok = mbar_wait(full_bar(stage), phase, err, 6);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t d = tmem_base + buf * C::kN;
-        const uint64_t ad0 = sdesc_kmajor_sw128(sA + stage * kStageBytesA);
-        const uint64_t bd0 = sdesc_kmajor_sw128(sB);
+        cur_qg = cur.qg;
+      }
+      const int buf = (int)(acc & 1);
+      const uint32_t use = (uint32_t)(acc >> 1);
+      ok = mbar_wait(tempty_bar(buf), (use & 1) ^ 1, err, 5);
+      if (!ok) break;
+      tc_fence_after();
+      ok = mbar_wait(full_bar(stage), phase, err, 6);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t d = tmem_base + buf * C::kN;
+      const uint64_t ad0 = sdesc_kmajor_sw128(sA + stage * kStageBytesA);
+      if (leader) {
 #pragma unroll
         for (int kh = 0; kh < 2; ++kh)
 #pragma unroll
@@ -243,20 +250,25 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                      bd0 + (uint64_t)((kh * C::kHalfBytesB + ks * 32) >> 4), idesc, (kh | ks) != 0);
         mma_commit(empty_bar(stage));
         mma_commit(tfull_bar(buf));
-        ++acc;
-        if (++stage == C::kStages) {
-          stage = 0;
-          phase ^= 1;
-        }
-        cur.next(it);
       }
-      // every MMA issued so far has finished before TMEM is released
+      __syncwarp();
+      ++acc;
+      if (++stage == C::kStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+      cur.next(it);
+    }
+    // every MMA issued so far has finished before TMEM is released
+    if (leader) {
       mma_commit(done_bar);
       if (!mbar_wait_drain(done_bar, 0)) atomicCAS(err, 0, 7);
     }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
+    const int qhalf = (warp - 2) >> 2;  // prefill: which half of the 8 queries this warp scores
     const int row_in_tile = 32 * quarter + lane;
     Cursor cur;
     cur.start(it, begin, end);
@@ -285,24 +297,42 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         slot = 1;
       }
       uint32_t* hslot = s_hist + slot * kHistBins;
-#pragma unroll 1
-      for (int g = 0; g < QG; ++g) {
+      (void)hslot;
+      if (QG == 1) {
         uint32_t r[32];
-        tmem_ld32(tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * C::kN + 32 * g, r);
+        tmem_ld32(tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * C::kN, r);
         tmem_ld_wait();
-        const int t = t0 + g;
         float sc = 0.f;
-        if (QG == 1) {
 #pragma unroll
-          for (int h = 0; h < 32; ++h) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
-        } else {
-          const float* wq = w + ((size_t)b * T + (t < T ? t : T - 1)) * 32;
-#pragma unroll
-          for (int h = 0; h < 32; ++h) sc = fmaf(__ldg(&wq[h]), fmaxf(__uint_as_float(r[h]), 0.f), sc);
-        }
-        if (t < T && key < visible_count(N, q_pos0, t)) {
-          scores[((size_t)b * T + t) * N + key] = sc;
+        for (int h = 0; h < 32; ++h) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
+        if (t0 < T && key < visible_count(N, q_pos0, t0)) {
+          scores[((size_t)b * T + t0) * N + key] = sc;
           if (kHist) atomicAdd(&hslot[order_key(sc) >> kHistShift], 1u);
+        }
+      } else {
+        // two queries (64 columns) per TMEM round trip; head weights as 16-byte loads
+#pragma unroll 1
+        for (int g = 4 * qhalf; g < 4 * qhalf + 4; g += 2) {
+          uint32_t r0[32], r1[32];
+          tmem_ld32(tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * C::kN + 32 * g, r0);
+          tmem_ld32(tmem_base + ((uint32_t)(32 * quarter) << 16) + buf * C::kN + 32 * g + 32, r1);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int t = t0 + g + u;
+            const float4* wq = reinterpret_cast<const float4*>(w + ((size_t)b * T + (t < T ? t : T - 1)) * 32);
+            float sc = 0.f;
+#pragma unroll
+            for (int h4 = 0; h4 < 8; ++h4) {
+              const float4 w4 = __ldg(&wq[h4]);
+              const uint32_t* rr = u ? r1 : r0;
+              sc = fmaf(w4.x, fmaxf(__uint_as_float(rr[4 * h4 + 0]), 0.f), sc);
+              sc = fmaf(w4.y, fmaxf(__uint_as_float(rr[4 * h4 + 1]), 0.f), sc);
+              sc = fmaf(w4.z, fmaxf(__uint_as_float(rr[4 * h4 + 2]), 0.f), sc);
+              sc = fmaf(w4.w, fmaxf(__uint_as_float(rr[4 * h4 + 3]), 0.f), sc);
+            }
+            if (t < T && key < visible_count(N, q_pos0, t)) scores[((size_t)b * T + t) * N + key] = sc;
+          }
         }
       }
       tc_fence_before();
@@ -323,7 +353,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     Cursor cur;
     cur.start(it, begin, end);
     const int b_first = cur.qg / it.G;
-    for (int i = threadIdx.x; i < 2 * kHistBins; i += kThreadsTC) {
+    for (int i = threadIdx.x; i < 2 * kHistBins; i += C::kThreads) {
       const uint32_t c = s_hist[i];
       const int row = b_first + i / kHistBins;
       if (c && row < B) atomicAdd(&hist[(size_t)row * kHistBins + (i % kHistBins)], c);
@@ -403,7 +433,7 @@ cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int 
   }
   if (total == 0) return cudaSuccess;
   const int grid = (int)(total < kNumSMs ? total : kNumSMs);
-  indexer_tc_kernel<QG, kHist><<<grid, kThreadsTC, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
+  indexer_tc_kernel<QG, kHist><<<grid, C::kThreads, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
                                                                        hist, err);
   return cudaGetLastError();
 }

@@ -14,12 +14,13 @@
 //   1. histogram of the top 12 bits (4096 bins) per row -- built here, or folded into
 //      the indexer epilogue;
 //   2. select kernel, grid (rows, chunks of 8192): every CTA finds the threshold bin b*
-//      from the histogram, counts its elements above b*, and appends the elements of
-//      bin b* to a per-row candidate list; the last CTA of a row (atomic ticket, no
-//      waiting) resolves the remaining 52 bits by 8-bit radix passes over the
-//      candidates in shared memory (or, if the bin holds more than kCandCap elements,
-//      over the row itself), giving the exact threshold composite, and turns per-chunk
-//      counts into output offsets;
+//      from the histogram, counts its elements above b*, appends the elements of bin b*
+//      to a per-row candidate list (one reservation per CTA) and histograms their next
+//      10 key bits into a per-row second-level histogram; the last CTA of a row (atomic
+//      ticket, no waiting) finds the second digit from that histogram, ranks the few
+//      elements of the final sub-bin directly (radix passes over the candidates, or over
+//      the row when bin b* overflows the list, are the fallbacks), which gives the exact
+//      threshold composite, and turns per-chunk counts into output offsets;
 //   3. compact kernel, grid (rows, chunks): every element with C(s) >= threshold is
 //      written at its chunk offset plus its warp-ballot rank, so the output comes out
 //      in ascending token order.
@@ -99,12 +100,19 @@ __device__ __forceinline__ uint32_t block_excl_scan(uint32_t v, uint32_t* s_warp
 
 constexpr int kRadixBins = 2048;  // digits of the resolve: 10, 10, 11, 11, 10 bits
 
+constexpr int kMaxSmemChunks = 4096;  // rows up to 32M scores keep their chunk counts in SMEM
+
+constexpr int kFinalCap = 1024;  // final sub-bin sizes ranked directly
+
 struct SelectSmem {
   uint32_t radix[kRadixBins];
+  uint32_t chunk_cnt[kMaxSmemChunks];
+  uint32_t hist2[kHist2Bins];
+  uint64_t fin[kFinalCap];
   uint32_t warp_tmp[32];
   uint32_t total;
-  uint32_t digit, digit_above, digit_count, is_last;
-  uint64_t cand[kCandCap];
+  uint32_t digit, digit_above, digit_count, is_last, cand_base, nfin;
+  unsigned long long thr;
 };
 
 // Digit search: with `bins` counts (bins <= 8 * kSelThreads), find the
@@ -187,7 +195,6 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   const int nchunks = gridDim.y;
   const long long V = visible_count(N, q_pos0, row_t(row, T));
   uint32_t* state = ws.row_state + (size_t)row * kRowStateWords;
-  const int lane = threadIdx.x & 31;
 
   if (V <= k) {
     // every visible position is kept; pad the rest of the row
@@ -203,51 +210,73 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   const uint32_t above = sm.digit_above;
   const uint32_t bcount = sm.digit_count;
   const bool use_cand = bcount <= (uint32_t)kCandCap;
+  for (int i = threadIdx.x; i < kHist2Bins; i += kSelThreads) sm.hist2[i] = 0;
 
-  // 2. scan this chunk: count the elements above b*, append the elements of b*
+  // 2. scan this chunk: count the elements above b*, append the elements of b* (one
+  //    reservation per CTA on the row's candidate counter, after a block scan)
   const float* sr = scores + (size_t)row * N;
   const long long s0 = (long long)chunk * kTopkChunk;
   const long long s1 = min(s0 + (long long)kTopkChunk, V);
   uint64_t* cand = ws.cand + (size_t)row * kCandCap;
-  uint32_t n_above = 0;
-  auto visit = [&](long long s, float v) {
-    const bool in = s < s1;
-    const uint32_t key = order_key(v);
-    const uint32_t bin = key >> kHistShift;
-    n_above += (in && bin > bstar) ? 1u : 0u;
-    const bool app = in && use_cand && bin == bstar;
-    const uint32_t m = __ballot_sync(0xFFFFFFFFu, app);
-    if (m) {
-      uint32_t base = 0;
-      if (lane == __ffs(m) - 1) base = atomicAdd(&state[RS_CAND], (uint32_t)__popc(m));
-      base = __shfl_sync(0xFFFFFFFFu, base, __ffs(m) - 1);
-      const uint32_t pos = base + __popc(m & ((1u << lane) - 1u));
-      if (app && pos < (uint32_t)kCandCap) cand[pos] = composite(key, (uint32_t)s);
-    }
+  constexpr int kPerThread = kTopkChunk / kSelThreads;  // 16
+  uint32_t keys[kPerThread];
+  uint32_t cand_bits = 0, n_above = 0;
+  auto elem = [&](int i) -> long long {
+    // element i of this thread: four consecutive scores per 16-byte group
+    return s0 + 4LL * (threadIdx.x + kSelThreads * (i >> 2)) + (i & 3);
   };
   if ((N & 3) == 0) {
-    // 16 scores per thread as four 16-byte loads, all issued before use
-    float4 v[4];
+    float4 v[kPerThread / 4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const long long e = s0 + 4LL * (threadIdx.x + kSelThreads * i);
-      v[i] = e + 3 < s1 ? __ldcg(reinterpret_cast<const float4*>(sr + e))
+    for (int g = 0; g < kPerThread / 4; ++g) {
+      const long long e = elem(4 * g);
+      v[g] = e + 3 < s1 ? __ldcg(reinterpret_cast<const float4*>(sr + e))
                         : make_float4(e < s1 ? sr[e] : 0.f, e + 1 < s1 ? sr[e + 1] : 0.f,
                                       e + 2 < s1 ? sr[e + 2] : 0.f, 0.f);
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const long long e = s0 + 4LL * (threadIdx.x + kSelThreads * i);
-      visit(e, v[i].x);
-      visit(e + 1, v[i].y);
-      visit(e + 2, v[i].z);
-      visit(e + 3, v[i].w);
+    for (int g = 0; g < kPerThread / 4; ++g) {
+      keys[4 * g + 0] = order_key(v[g].x);
+      keys[4 * g + 1] = order_key(v[g].y);
+      keys[4 * g + 2] = order_key(v[g].z);
+      keys[4 * g + 3] = order_key(v[g].w);
     }
   } else {
-    for (long long s = s0 + threadIdx.x; s < s0 + kTopkChunk; s += kSelThreads) visit(s, s < s1 ? sr[s] : 0.f);
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i) {
+      const long long e = elem(i);
+      keys[i] = e < s1 ? order_key(sr[e]) : 0u;
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const bool in = elem(i) < s1;
+    const uint32_t bin = keys[i] >> kHistShift;
+    n_above += (in && bin > bstar) ? 1u : 0u;
+    cand_bits |= (in && use_cand && bin == bstar) ? (1u << i) : 0u;
+  }
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i)
+    if (cand_bits & (1u << i)) atomicAdd(&sm.hist2[(keys[i] >> 10) & (kHist2Bins - 1)], 1u);
+  const uint32_t my_off = block_excl_scan((uint32_t)__popc(cand_bits), sm.warp_tmp, &sm.total);
+  if (threadIdx.x == 0) sm.cand_base = sm.total ? atomicAdd(&state[RS_CAND], sm.total) : 0u;
+  __syncthreads();
+  {
+    uint32_t pos = sm.cand_base + my_off;
+#pragma unroll
+    for (int i = 0; i < kPerThread; ++i)
+      if (cand_bits & (1u << i)) {
+        if (pos < (uint32_t)kCandCap) cand[pos] = composite(keys[i], (uint32_t)elem(i));
+        ++pos;
+      }
   }
   (void)block_excl_scan(n_above, sm.warp_tmp, &sm.total);
   if (threadIdx.x == 0) ws.chunk_above[(size_t)row * nchunks + chunk] = sm.total;
+  if (use_cand) {
+    uint32_t* g2 = ws.hist2 + (size_t)row * kHist2Bins;
+    for (int i = threadIdx.x; i < kHist2Bins; i += kSelThreads)
+      if (sm.hist2[i]) atomicAdd(&g2[i], sm.hist2[i]);
+  }
 
   // 3. the last CTA of the row resolves the threshold
   __threadfence();
@@ -258,35 +287,74 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   __threadfence();
 
   const uint32_t remaining = (uint32_t)k - above;  // 1 <= remaining <= bcount
-  uint64_t thr52;
-  if (use_cand) {
-    for (long long i = threadIdx.x; i < bcount; i += kSelThreads) sm.cand[i] = __ldcg(&cand[i]);
-    __syncthreads();
-    thr52 = resolve_threshold(sm, bcount, remaining, [&](long long i, uint64_t& c) {
-      c = sm.cand[i];
-      return true;
-    });
-  } else {
-    thr52 = resolve_threshold(sm, V, remaining, [&](long long s, uint64_t& c) {
-      const uint32_t key = order_key(__ldcg(&sr[s]));
-      if ((key >> kHistShift) != bstar) return false;
-      c = composite(key, (uint32_t)s);
-      return true;
-    });
-  }
-  const uint64_t thr = ((uint64_t)bstar << 52) | thr52;
-
-  // 4. threshold-bin elements selected per chunk
+  const bool smem_cnt = nchunks <= kMaxSmemChunks;
   uint32_t* csel = ws.chunk_sel + (size_t)row * nchunks;
+  uint32_t* cnt = smem_cnt ? sm.chunk_cnt : csel;
+  if (smem_cnt)
+    for (int c = threadIdx.x; c < nchunks; c += kSelThreads) sm.chunk_cnt[c] = 0;
+  if (threadIdx.x == 0) {
+    sm.nfin = 0;
+    sm.thr = 0;
+  }
+  uint64_t thr = 0;
+  bool resolved = false;
   if (use_cand) {
-    for (long long i = threadIdx.x; i < bcount; i += kSelThreads) {
-      const uint64_t c = sm.cand[i];
-      if (c >= thr) atomicAdd(&csel[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+    // 4a. second digit from the row's second-level histogram; the elements of the final
+    //     sub-bin (usually a handful) are ranked directly
+    const uint32_t* g2 = ws.hist2 + (size_t)row * kHist2Bins;
+    find_digit(sm, kHist2Bins, remaining, [&](int bin) { return __ldcg(&g2[bin]); });
+    const uint32_t d2 = sm.digit, r2 = remaining - sm.digit_above, n2 = sm.digit_count;
+    if (n2 <= (uint32_t)kFinalCap) {
+      for (long long i = threadIdx.x; i < bcount; i += kSelThreads) {
+        const uint64_t c = __ldcg(&cand[i]);
+        const uint32_t dg = (uint32_t)(c >> 42) & (kHist2Bins - 1);
+        if (dg > d2) atomicAdd(&cnt[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+        else if (dg == d2) {
+          const uint32_t pos = atomicAdd(&sm.nfin, 1u);
+          if (pos < (uint32_t)kFinalCap) sm.fin[pos] = c;
+        }
+      }
+      __syncthreads();
+      const uint32_t nf = min(sm.nfin, (uint32_t)kFinalCap);  // == n2
+      for (uint32_t i = threadIdx.x; i < nf; i += kSelThreads) {
+        const uint64_t c = sm.fin[i];
+        uint32_t rank = 0;
+        for (uint32_t j = 0; j < nf; ++j) rank += sm.fin[j] > c ? 1u : 0u;
+        if (rank == r2 - 1) sm.thr = c;  // composites are distinct: exactly one thread writes
+      }
+      __syncthreads();
+      thr = sm.thr;
+      for (uint32_t i = threadIdx.x; i < nf; i += kSelThreads) {
+        const uint64_t c = sm.fin[i];
+        if (c >= thr) atomicAdd(&cnt[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+      }
+      resolved = true;
+    } else {
+      // many equal high bits: radix passes over the candidate list
+      const uint64_t thr52 = resolve_threshold(sm, bcount, remaining, [&](long long i, uint64_t& c) {
+        c = __ldcg(&cand[i]);
+        return true;
+      });
+      thr = ((uint64_t)bstar << 52) | thr52;
+      for (long long i = threadIdx.x; i < bcount; i += kSelThreads) {
+        const uint64_t c = __ldcg(&cand[i]);
+        if (c >= thr) atomicAdd(&cnt[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+      }
+      resolved = true;
     }
-  } else {
-    for (long long s = threadIdx.x; s < V; s += kSelThreads) {
-      const uint32_t key = order_key(__ldcg(&sr[s]));
-      if ((key >> kHistShift) == bstar && composite(key, (uint32_t)s) >= thr) atomicAdd(&csel[s / kTopkChunk], 1u);
+  }
+  if (!resolved) {
+    // the threshold bin overflowed the candidate list: radix passes over the row itself
+    const uint64_t thr52 = resolve_threshold(sm, V, remaining, [&](long long s2, uint64_t& c) {
+      const uint32_t key = order_key(__ldcg(&sr[s2]));
+      if ((key >> kHistShift) != bstar) return false;
+      c = composite(key, (uint32_t)s2);
+      return true;
+    });
+    thr = ((uint64_t)bstar << 52) | thr52;
+    for (long long s2 = threadIdx.x; s2 < V; s2 += kSelThreads) {
+      const uint32_t key = order_key(__ldcg(&sr[s2]));
+      if ((key >> kHistShift) == bstar && composite(key, (uint32_t)s2) >= thr) atomicAdd(&cnt[s2 / kTopkChunk], 1u);
     }
   }
   __threadfence();
@@ -296,7 +364,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   uint32_t carry = 0;
   for (int c0 = 0; c0 < nchunks; c0 += kSelThreads) {
     const int c = c0 + threadIdx.x;
-    const uint32_t v = c < nchunks ? __ldcg(&ws.chunk_above[(size_t)row * nchunks + c]) + __ldcg(&csel[c]) : 0u;
+    const uint32_t v = c < nchunks ? __ldcg(&ws.chunk_above[(size_t)row * nchunks + c]) + (smem_cnt ? sm.chunk_cnt[c] : __ldcg(&csel[c])) : 0u;
     const uint32_t off = block_excl_scan(v, sm.warp_tmp, &sm.total);
     if (c < nchunks) ws.chunk_off[(size_t)row * nchunks + c] = carry + off;
     carry += sm.total;
@@ -418,6 +486,7 @@ size_t topk_workspace_bytes(long long rows, int N) {
   b += (size_t)rows * kHistBins * 4;
   b += (size_t)rows * kRowStateWords * 4;
   b += (size_t)rows * nchunks * 4 * 3;
+  b += (size_t)rows * kHist2Bins * 4;
   b = (b + 255) & ~(size_t)255;
   b += (size_t)rows * kCandCap * 8;
   return (b + 255) & ~(size_t)255;
@@ -433,6 +502,8 @@ TopkWorkspace topk_workspace(void* base, long long rows, int N) {
   p += (size_t)rows * kRowStateWords * 4;
   w.chunk_sel = reinterpret_cast<uint32_t*>(p);
   p += (size_t)rows * nchunks * 4;
+  w.hist2 = reinterpret_cast<uint32_t*>(p);
+  p += (size_t)rows * kHist2Bins * 4;
   w.zero_bytes = (size_t)(p - static_cast<unsigned char*>(base));
   w.chunk_above = reinterpret_cast<uint32_t*>(p);
   p += (size_t)rows * nchunks * 4;
