@@ -138,6 +138,28 @@ class ClockSampler:
         return {"sm_mhz": sms[len(sms) // 2], "sm_max_mhz": rows[0][1], "reasons": reasons, "samples": len(rows)}
 
 
+def rank_key(key: int, rank: int) -> int:
+    """Each rank decodes its own batch (weak scaling): its inputs use the workload's keys
+    XOR the rank, so no two ranks see the same tensors."""
+    return key ^ rank
+
+
+def max_over_ranks(values, world: int, device=None):
+    """Element-wise max of a list of floats over all ranks (the slowest rank sets the step
+    time).  Uses the initialised process group; a no-op for a single process."""
+    import torch
+    if world <= 1:
+        return list(values)
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_throughput(units_per_rank: int, world: int, max_ms: float) -> float:
+    """Whole-job units per second: the units all ranks processed over the slowest rank's time."""
+    return units_per_rank * world / (max_ms * 1e-3)
+
+
 def make_inputs(w, device, rank):
     import torch
     import synth
@@ -146,27 +168,27 @@ def make_inputs(w, device, rank):
     groups = []
     for g in range(w.groups):
         ik = torch.empty(w.B, w.N, 128, dtype=bf, device=device)
-        sd.int17_bf16(ik, w.key(synth.KIND_IK, g) ^ rank)
+        sd.int17_bf16(ik, rank_key(w.key(synth.KIND_IK, g), rank))
         kvs = []
         for l in range(w.L):
             kv = torch.empty(w.B, w.N, 576, dtype=bf, device=device)
-            sd.normal_bf16(kv, w.key(synth.KIND_KV, g, l) ^ rank)
+            sd.normal_bf16(kv, rank_key(w.key(synth.KIND_KV, g, l), rank))
             kvs.append(kv)
         iq = torch.empty(w.B, w.T, 32, 128, dtype=bf, device=device)
-        sd.int17_bf16(iq, w.key(synth.KIND_IQ, g) ^ rank)
+        sd.int17_bf16(iq, rank_key(w.key(synth.KIND_IQ, g), rank))
         wt = torch.empty(w.B, w.T, 32, dtype=torch.float32, device=device)
-        sd.pow2_f32(wt, w.key(synth.KIND_W, g) ^ rank)
+        sd.pow2_f32(wt, rank_key(w.key(synth.KIND_W, g), rank))
         qs = []
         for l in range(w.L):
             q = torch.empty(w.B, w.T, w.H, 576, dtype=bf, device=device)
-            sd.normal_bf16(q, w.key(synth.KIND_Q, g, l) ^ rank)
+            sd.normal_bf16(q, rank_key(w.key(synth.KIND_Q, g, l), rank))
             qs.append(q)
         idx = torch.empty(w.B, w.T, w.k, dtype=torch.int32, device=device)
         outs = [torch.empty(w.B, w.T, w.H, 512, dtype=torch.float32, device=device) for _ in range(w.L)]
         draft_qs = []
         for st in range(1, w.steps):
             qd = torch.empty(w.B, w.T, w.H, 576, dtype=bf, device=device)
-            sd.normal_bf16(qd, w.key(synth.KIND_Q, g, 0, st) ^ rank)
+            sd.normal_bf16(qd, rank_key(w.key(synth.KIND_Q, g, 0, st), rank))
             draft_qs.append(qd)
         groups.append(dict(ik=ik, kvs=kvs, iq=iq, wt=wt, qs=qs, idx=idx, outs=outs, draft_qs=draft_qs))
     return groups
@@ -253,6 +275,7 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     idx_ms = sum(idx_times) / len(idx_times)
 
     if not e2e:
+        step_ms, idx_ms = max_over_ranks([step_ms, idx_ms], world, device)
         del groups, ws, flush, flush_rd, scores, graph, igraph
         torch.cuda.empty_cache()
         return w, step_ms, idx_ms, None, 0, 0, clk.summary()
@@ -276,10 +299,7 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     e2e_times = timed(e2e_step, args.steps, args.warmup)
     e2e_ms = sum(e2e_times) / len(e2e_times)
 
-    if world > 1:
-        t = torch.tensor([step_ms, e2e_ms, idx_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        step_ms, e2e_ms, idx_ms = t.tolist()
+    step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms], world, device)
     return w, step_ms, idx_ms, e2e_ms, h2d, d2h, clk.summary()
 
 
@@ -358,7 +378,7 @@ def main():
     w, step_ms, idx_ms, e2e_ms, h2d, d2h, clocks = run_ours(args, rank, world, device)
     step_bytes, idx_bytes = algorithmic(w)
     tokens = w.B * w.T * world
-    value = tokens / (step_ms * 1e-3)
+    value = job_throughput(w.B * w.T, world, step_ms)
     peak, peak_kind = peaks()
     achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
     line = {

@@ -58,6 +58,7 @@ constexpr int kMmaWarp = kProducerWarps;
 constexpr int kSoftmaxWarp0 = kProducerWarps + 1;
 constexpr int kThreadsA = (kProducerWarps + 5) * 32;  // 416
 constexpr float kRescaleLog2 = 8.f;
+constexpr int kPrefetchRounds = 2;               // L2 prefetch distance, in rounds of kStages tiles
 
 constexpr int kOffQ = 0;
 constexpr int kOffStage = kOffQ + kQBytes;
@@ -163,6 +164,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     // column block and in-row offset of each are constants
     const int c0 = lane, c1 = lane + 32, c2 = lane + 64;
     const uint32_t kb0 = (c0 >> 3) * kBlockBytes, kb1 = (c1 >> 3) * kBlockBytes, kb2 = (c2 >> 3) * kBlockBytes;
+    // rows of this warp's tile i are pulled into L2 kPrefetchRounds rounds ahead, so the
+    // shared-memory gather of a tile mostly hits L2: L2 is the deep in-flight buffer the
+    // stage ring is too small to be
+    auto prefetch_tile = [&](int i) {
+      if (i < ntiles && lane < 16) {
+        const int key = i * kKeys + 16 * half + lane;
+        const int v = key < nkeys ? __ldg(&sel[key]) : -1;
+        if (v >= 0 && v < N) prefetch_l2(kvb + (size_t)v * kDqk, kDqk * 2);
+      }
+    };
     for (int i = ps; i < ntiles; i += kStages) {
       bool ok = true;
       if (lane == 0) ok = mbar_wait(empty_bar(ps), ((i / kStages) & 1) ^ 1, err, 21);
@@ -185,6 +196,12 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         if (c2 < kDqk / 8) cp_async_16(rbase + kb2 + (((c2 & 7) ^ x) << 4), src + c2 * 8, 16);
       }
       cp_async_commit();
+      // prefetch while this tile's copies are in flight: the first time the next
+      // kPrefetchRounds rounds, afterwards the round that comes kPrefetchRounds later
+      if (i == ps)
+        for (int r = 1; r <= kPrefetchRounds; ++r) prefetch_tile(ps + r * kStages);
+      else
+        prefetch_tile(i + kPrefetchRounds * kStages);
       cp_async_wait<0>();
       fence_proxy_async();  // the copies are visible to the tensor core (async proxy)
       mbar_arrive(full_bar(ps));
