@@ -141,6 +141,8 @@ dsa_status dsa_topk_noalloc(const float *scores, int B, int T, int N, long long 
  *   out  [B, T, H, 512] f32    softmax_j(scale * q . kv[idx_j]) weighted sum of values;
  *                              zero when a row selects nothing
  * bf16 operands, f32 accumulation and softmax.  H in {16, 32, 48, 64}.
+ * The key splits of a query row are reduced on chip, so this call needs no workspace:
+ * `workspace` may be NULL and `workspace_bytes` 0 (both are ignored).
  */
 dsa_status dsa_sparse_attn(const uint16_t *q, const uint16_t *kv, const int32_t *idx,
                            int B, int T, int N, int H, int k, float scale, float *out,

@@ -26,10 +26,13 @@
 //   warp 8      TMEM allocation; one elected lane issues S(i) and then O += P(i-1) V(i-1),
 //               so the softmax of one tile overlaps the next tile's logits;
 //   warps 9..12 softmax (threads on lanes 0..15 of each warp own a head), P as bf16 in
-//               shared memory, and at the end the read-out of O^T (lane = value dim) into
-//               shared memory and one bulk (TMA) store of the [H][512] output block --
-//               per-thread 4-byte global stores of that block ran at a few GB/s from an SM
-//               whose shared memory leaves almost no L1.
+//               shared memory.
+// The key splits of one (row, layer) run as one thread-block cluster and are reduced on
+// chip: each split scales its O^T by its share of the normaliser, stages it in its shared
+// memory, and sums one slice of the [H][512] output over the cluster's shared memories.
+// (A global-memory merge by the last split to finish -- 16 MB of partials written and
+// read back at the end of the 32-unit decode batch -- made the kernel's tail longer than
+// its whole main loop.)
 // All mbarrier waits are bounded (sm100.cuh).
 #include <cudaTypedefs.h>
 
@@ -57,8 +60,10 @@ constexpr int kProducerWarps = 8;                // two warps per stage, 16 rows
 constexpr int kMmaWarp = kProducerWarps;
 constexpr int kSoftmaxWarp0 = kProducerWarps + 1;
 constexpr int kThreadsA = (kProducerWarps + 5) * 32;  // 416
+static_assert(kSoftmaxWarp0 + 4 == kThreadsA / 32, "four softmax warps, one per TMEM lane quarter");
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kPrefetchRounds = 2;               // L2 prefetch distance, in rounds of kStages tiles
+constexpr int kMaxSplits = 8;                    // key splits of one (row, layer): one portable cluster
 
 constexpr int kOffQ = 0;
 constexpr int kOffStage = kOffQ + kQBytes;
@@ -67,9 +72,12 @@ constexpr int kOffAlpha = kOffP + 2 * kPBytes;   // [2][64] f32 (tile parity)
 constexpr int kOffL = kOffAlpha + 2 * 64 * 4;    // [64] f32
 constexpr int kOffM = kOffL + 64 * 4;            // [64] f32
 constexpr int kOffMask = kOffM + 64 * 4;         // [kStages][2] u16 (one half per producer warp)
-constexpr int kOffFlag = kOffMask + kStages * 4;   // u32: this CTA merges the splits
+constexpr int kOffVote = kOffMask + kStages * 4;  // [2] u32 (tile parity): one byte per softmax warp
+// after the main loop the P buffers hold [kMaxSplits][64] f32: each split's share of the normaliser
+constexpr int kOffCoef = kOffP;
+static_assert(kMaxSplits * 64 * 4 <= 2 * kPBytes, "coefficients fit the P buffers");
 constexpr int kNumBars = 2 * kStages + 11;
-constexpr int kOffBar = kOffFlag + 16;
+constexpr int kOffBar = kOffVote + 16;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmemA = kOffTmem + 16 + 1024;
 static_assert(kSmemA <= 232448, "shared memory budget");
@@ -84,8 +92,7 @@ struct AttnMaps {
 
 __global__ void __launch_bounds__(kThreadsA, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const int32_t* __restrict__ idx, int T, int N,
-               int H, int k, int chunk, float scale_log2, float* __restrict__ partial, uint32_t* __restrict__ tickets,
-               int* __restrict__ err) {
+               int H, int k, int chunk, float scale_log2, int* __restrict__ err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -96,7 +103,8 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   float* s_l = reinterpret_cast<float*>(smem + kOffL);
   float* s_m = reinterpret_cast<float*>(smem + kOffM);
   uint16_t* s_mask = reinterpret_cast<uint16_t*>(smem + kOffMask);
-  uint32_t* s_last = reinterpret_cast<uint32_t*>(smem + kOffFlag);
+  float* s_coef = reinterpret_cast<float*>(smem + kOffCoef);
+  uint32_t* s_vote = reinterpret_cast<uint32_t*>(smem + kOffVote);
   const uint32_t bar0 = sbase + kOffBar;
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (kStages + s); };
@@ -133,7 +141,6 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     mbar_init(ofinal_bar, 1);
     mbar_init(qfull_bar, 1);
     mbar_init(grp_bar, 128);
-    *s_last = 0;
     fence_mbar_init();
     tma_prefetch(&maps.q[layer]);
   }
@@ -264,7 +271,6 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   } else {
     // ------------------------------------------------------------------ softmax + read-out
     const int quarter = warp & 3;
-    const int st_tid = threadIdx.x - 32 * kSoftmaxWarp0;  // 0..127
     const bool owner = lane < 16;                 // this thread's TMEM lane holds a head of S
     const int head = 16 * quarter + (lane & 15);
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
@@ -299,14 +305,16 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         l_run *= a;
       }
       if (owner) alpha[head] = a;
+      // one vote per warp: does any of its heads need O rescaled?  (64 shared loads of
+      // the factors per thread, serialised, cost about a microsecond per tile)
+      const uint32_t vote = __ballot_sync(0xFFFFFFFFu, owner && head < H && a != 1.f);
+      if (lane == 0) reinterpret_cast<volatile unsigned char*>(s_vote + (i & 1))[quarter] = vote != 0u ? 1 : 0;
       // every head's factor is known before O is touched
       mbar_arrive(grp_bar);
       ok = mbar_wait(grp_bar, grp_phase, err, 29);
       grp_phase ^= 1;
       if (!ok) break;
-      bool any = false;
-#pragma unroll 8
-      for (int h = 0; h < 64; ++h) any |= h < H && alpha[h] != 1.f;
+      const bool any = *reinterpret_cast<volatile uint32_t*>(s_vote + (i & 1)) != 0u;
       if (i > 0 && any) {
         // O^T is rescaled only once the previous tile's PV has finished with it
         ok = mbar_wait(pfree_bar((i - 1) & 1), ((i - 1) >> 1) & 1, err, 30);
@@ -355,123 +363,114 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
       tc_fence_before();
       mbar_arrive(pfull_bar(i & 1));
     }
-    // ------------------------------------------------------------------ read-out
-    if (ok && ntiles > 0) ok = mbar_wait(ofinal_bar, 0, err, 31);
-    tc_fence_after();
     if (owner) {
       s_l[head] = l_run;
       s_m[head] = m_used;
     }
-    mbar_arrive(grp_bar);
-    if (ok) ok = mbar_wait(grp_bar, grp_phase, err, 32);
-    if (ok) {
-      // O^T (lane = value dim, column = head) -> shared [head][512] (the stage ring is idle
-      // now) -> one bulk store of the whole [H][512] block
-      float* s_out = reinterpret_cast<float*>(smem + kOffStage);
-      const int dim_lane = 32 * quarter + lane;
-      // the 64 normalisers in registers once: a dependent shared load per element,
-      // serialised against the shared stores below, made this loop ~20x slower
-      float inv[64];
+  }
+
+  // ------------------------------------------------------------------ split reduction
+  // The splits of one (row, layer) form a cluster.  Each split publishes its running max
+  // and sum per head and stages its unnormalised O in its own shared memory, in the
+  // output's [head][512] layout; split r then owns slice r of that block and sums it over
+  // the cluster through distributed shared memory,
+  //   out[h] = sum_s c_s[h] O_s[h],  c_s[h] = 2^(m_s[h] - M[h]) / sum_r 2^(m_r[h] - M[h]) l_r[h],
+  // M[h] = max_r m_r[h], writes the sum back over its own slice (no peer reads that
+  // slice) and stores it with one bulk copy.  Nothing but the result goes through global
+  // memory.  Every thread passes the three cluster barriers on every path (a failed wait
+  // above only skips work), so none of them can be left waiting.
+  tc_fence_before();
+  cluster_sync();  // #1: (m, l) of every split published; this CTA's MMAs have completed
+  tc_fence_after();
+  if (threadIdx.x < 64) {
+    const int h = threadIdx.x;
+    float mr[kMaxSplits], lr[kMaxSplits];
+    float M = -INFINITY;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float4 l4 = reinterpret_cast<const float4*>(s_l)[j];
-        inv[4 * j + 0] = nsplit > 1 ? 1.f : (l4.x > 0.f ? 1.f / l4.x : 0.f);
-        inv[4 * j + 1] = nsplit > 1 ? 1.f : (l4.y > 0.f ? 1.f / l4.y : 0.f);
-        inv[4 * j + 2] = nsplit > 1 ? 1.f : (l4.z > 0.f ? 1.f / l4.z : 0.f);
-        inv[4 * j + 3] = nsplit > 1 ? 1.f : (l4.w > 0.f ? 1.f / l4.w : 0.f);
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+      mr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_m + h), sp)) : -INFINITY;
+      lr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_l + h), sp)) : 0.f;
+      M = fmaxf(M, mr[sp]);
+    }
+    float den = 0.f;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp) {
+      mr[sp] = mr[sp] == -INFINITY ? 0.f : exp2f(mr[sp] - M);
+      den += mr[sp] * lr[sp];
+    }
+    const float inv = den > 0.f ? 1.f / den : 0.f;
+#pragma unroll
+    for (int sp = 0; sp < kMaxSplits; ++sp)
+      if (sp < nsplit) s_coef[sp * 64 + h] = mr[sp] * inv;
+  }
+  // O^T (TMEM lane = value dim, column = head) -> staging [64 heads][512] f32 over the idle
+  // Q and stage buffers.  Twelve warps, three per TMEM lane quarter, take the eight
+  // 32-column chunks (value block mb, head half) two loads at a time.
+  float* stg = reinterpret_cast<float*>(smem + kOffQ);
+  if (warp != kMmaWarp) {
+    const int quarter = warp & 3;
+    const int j = warp < kProducerWarps ? warp >> 2 : 2;
+    const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16) + kTmemO;
+    for (int c = j; c < 8; c += 6) {
+      const bool two = c + 3 < 8;
+      uint32_t o0[32], o1[32];
+      if (ntiles > 0) {
+        tmem_ld32(lane_base + 64 * (c >> 1) + 32 * (c & 1), o0);
+        if (two) tmem_ld32(lane_base + 64 * ((c + 3) >> 1) + 32 * ((c + 3) & 1), o1);
+        tmem_ld_wait();
+      } else {
+#pragma unroll
+        for (int c2 = 0; c2 < 32; ++c2) o0[c2] = o1[c2] = 0u;
       }
-#pragma unroll 1
-      for (int mb = 0; mb < 4; ++mb) {
+      float* d0 = stg + (32 * (c & 1)) * kDv + 128 * (c >> 1) + 32 * quarter + lane;
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t o[32];
-          if (ntiles > 0) {
-            tmem_ld32(tmem + lane_addr + kTmemO + 64 * mb + 32 * half, o);
-            tmem_ld_wait();
-          } else {
+      for (int c2 = 0; c2 < 32; ++c2) d0[c2 * kDv] = __uint_as_float(o0[c2]);
+      if (two) {
+        float* d1 = stg + (32 * ((c + 3) & 1)) * kDv + 128 * ((c + 3) >> 1) + 32 * quarter + lane;
 #pragma unroll
-            for (int c = 0; c < 32; ++c) o[c] = 0u;
-          }
-          const int dim = 128 * mb + dim_lane;
-          // rows h >= H are written too (the store below copies only the first H)
-#pragma unroll
-          for (int c = 0; c < 32; ++c) s_out[(32 * half + c) * kDv + dim] = __uint_as_float(o[c]) * inv[32 * half + c];
-        }
-      }
-      fence_proxy_async();
-      mbar_arrive(grp_bar);
-      grp_phase ^= 1;
-      ok = mbar_wait(grp_bar, grp_phase, err, 33);
-      const size_t unit = ((size_t)layer * gridDim.y + row) * nsplit + split;
-      if (ok && st_tid == 0) {
-        float* dst = nsplit == 1 ? layers.out[layer] + (size_t)row * H * kDv : partial + unit * (size_t)H * (kDv + 2);
-        bulk_store(dst, smem_u32(s_out), (uint32_t)(H * kDv * 4));
-        bulk_commit();
-        bulk_wait_all();
-        fence_proxy_async_global();
-      }
-      if (ok && nsplit > 1) {
-        if (st_tid < H) {
-          float* pm = partial + unit * (size_t)H * (kDv + 2) + (size_t)H * kDv;
-          pm[2 * st_tid] = ntiles > 0 ? s_m[st_tid] : -INFINITY;
-          pm[2 * st_tid + 1] = ntiles > 0 ? s_l[st_tid] : 0.f;
-        }
-        // publish this split; the last split of the (row, layer) to arrive merges them all
-        __threadfence();
-        mbar_arrive(grp_bar);
-        grp_phase ^= 1;
-        ok = mbar_wait(grp_bar, grp_phase, err, 35);
-        if (ok && st_tid == 0) {
-          const uint32_t t = atomicAdd(&tickets[(size_t)layer * gridDim.y + row], 1u);
-          *s_last = (t == (uint32_t)nsplit - 1) ? 1u : 0u;
-        }
+        for (int c2 = 0; c2 < 32; ++c2) d1[c2 * kDv] = __uint_as_float(o1[c2]);
       }
     }
   }
-
+  cluster_sync();  // #2: every split's O is staged and its coefficients are known
+  {
+    // this split's slice of the output: float4 e = h * 128 + d/4 of the [H][512] block,
+    // which is also its byte offset / 16 in every split's staging buffer
+    const int total = H * (kDv / 4);
+    const int e0 = (int)((long long)split * total / nsplit), e1 = (int)((long long)(split + 1) * total / nsplit);
+    const uint32_t stg_s = smem_u32(stg);
+#pragma unroll 2
+    for (int e = e0 + threadIdx.x; e < e1; e += kThreadsA) {
+      const int h = e >> 7;
+      const uint32_t off = stg_s + 16u * (uint32_t)e;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplits; ++sp) {
+        if (sp < nsplit) {
+          const float cf = s_coef[sp * 64 + h];
+          const float4 v = ld_cluster_v4(cluster_map(off, sp));
+          acc.x = fmaf(cf, v.x, acc.x);
+          acc.y = fmaf(cf, v.y, acc.y);
+          acc.z = fmaf(cf, v.z, acc.z);
+          acc.w = fmaf(cf, v.w, acc.w);
+        }
+      }
+      reinterpret_cast<float4*>(stg)[e] = acc;
+    }
+    fence_proxy_async();  // the sums are visible to the bulk copy (async proxy)
+    __syncthreads();
+    if (threadIdx.x == 0 && e1 > e0) {
+      bulk_store(layers.out[layer] + (size_t)row * H * kDv + 4 * (size_t)e0, stg_s + 16u * (uint32_t)e0,
+                 (uint32_t)(e1 - e0) * 16u);
+      bulk_commit();
+      bulk_wait_all();
+    }
+  }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();  // #3: the peers are done reading this CTA's staging buffer
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
-  }
-  if (nsplit > 1 && *s_last) {
-    // merge: out[h][:] = sum_s 2^(m_s - M) O_s[h][:] / sum_s 2^(m_s - M) l_s
-    __threadfence();
-    const size_t unit0 = ((size_t)layer * gridDim.y + row) * nsplit;
-    const size_t stride = (size_t)H * (kDv + 2);
-    float* coef = reinterpret_cast<float*>(smem + kOffStage);  // [nsplit][64], the stages are idle
-    if (threadIdx.x < H) {
-      const int h = threadIdx.x;
-      float M = -INFINITY;
-      for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, __ldcg(&partial[(unit0 + sp) * stride + (size_t)H * kDv + 2 * h]));
-      float den = 0.f;
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float m = __ldcg(&partial[(unit0 + sp) * stride + (size_t)H * kDv + 2 * h]);
-        const float l = __ldcg(&partial[(unit0 + sp) * stride + (size_t)H * kDv + 2 * h + 1]);
-        const float wgt = m == -INFINITY ? 0.f : exp2f(m - M);
-        coef[sp * 64 + h] = wgt;
-        den += wgt * l;
-      }
-      const float inv = den > 0.f ? 1.f / den : 0.f;
-      for (int sp = 0; sp < nsplit; ++sp) coef[sp * 64 + h] *= inv;
-    }
-    __syncthreads();
-    float* out = layers.out[layer] + (size_t)row * H * kDv;
-    for (int e = threadIdx.x; e < H * (kDv / 4); e += kThreadsA) {
-      const int h = e / (kDv / 4), d = (e - h * (kDv / 4)) * 4;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int sp = 0; sp < nsplit; ++sp) {
-        const float c = coef[sp * 64 + h];
-        if (c == 0.f) continue;
-        const float4 o = __ldcg(reinterpret_cast<const float4*>(partial + (unit0 + sp) * stride + (size_t)h * kDv + d));
-        acc.x = fmaf(c, o.x, acc.x);
-        acc.y = fmaf(c, o.y, acc.y);
-        acc.z = fmaf(c, o.z, acc.z);
-        acc.w = fmaf(c, o.w, acc.w);
-      }
-      *reinterpret_cast<float4*>(out + (size_t)h * kDv + d) = acc;
-    }
   }
 }
 
@@ -528,28 +527,23 @@ int attn_split_chunk(int k, int nsplit) {
   return (chunk + kAttnTile - 1) / kAttnTile * kAttnTile;
 }
 
-// Splits per (query row, layer): about one CTA per SM in total.
+// Splits per (query row, layer): about one CTA per SM in total, at most one cluster's worth.
 int attn_num_splits(long long rows, int L, int k) {
   const long long units = rows * L;
   long long ns = kNumSMs / (units > 0 ? units : 1);
   if (ns < 1) ns = 1;
+  if (ns > kMaxSplits) ns = kMaxSplits;
   const long long max_ns = (k + kAttnTile - 1) / kAttnTile;
   if (ns > max_ns) ns = max_ns;
   const int chunk = attn_split_chunk(k, (int)ns);
   return (k + chunk - 1) / chunk;
 }
 
-size_t attn_ticket_bytes(long long rows, int L) { return ((size_t)L * rows * sizeof(uint32_t) + 255) & ~(size_t)255; }
-
-// Workspace of the split path: one ticket per (layer, row), then the split partials.
-size_t attn_workspace_bytes(long long rows, int L, int H, int k) {
-  const int ns = attn_num_splits(rows, L, k);
-  if (ns <= 1) return 0;
-  return attn_ticket_bytes(rows, L) + (size_t)L * rows * ns * H * (kDv + 2) * sizeof(float);
-}
+// The splits are reduced on chip (cluster shared memory): no global workspace.
+size_t attn_workspace_bytes(long long, int, int, int) { return 0; }
 
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                                  int k, float scale, void* ws, cudaStream_t stream) {
+                                  int k, float scale, void*, cudaStream_t stream) {
   const long long rows = (long long)B * T;
   AttnMaps maps;
   for (int l = 0; l < L; ++l)
@@ -563,13 +557,21 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
     return e;
   const int nsplit = attn_num_splits(rows, L, k);
   const int chunk = attn_split_chunk(k, nsplit);
-  uint32_t* tickets = static_cast<uint32_t*>(ws);
-  float* partial = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + attn_ticket_bytes(rows, L));
-  if (nsplit > 1 && (e = cudaMemsetAsync(tickets, 0, (size_t)L * rows * sizeof(uint32_t), stream)) != cudaSuccess)
-    return e;
-  attn_tc_kernel<<<dim3(nsplit, (unsigned)rows, L), kThreadsA, kSmemA, stream>>>(
-      maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f, partial, tickets, err);
-  return cudaGetLastError();
+  // the splits of one (row, layer) are one cluster along x
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nsplit, (unsigned)rows, L);
+  cfg.blockDim = dim3(kThreadsA);
+  cfg.dynamicSmemBytes = kSmemA;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nsplit;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f,
+                            err);
 }
 
 cudaError_t attn_tc_device_error(int* code, bool clear) {

@@ -68,7 +68,6 @@ constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core atte
 
 int attn_num_splits(long long rows, int L, int k);
 int attn_split_chunk(int k, int nsplit);
-size_t attn_ticket_bytes(long long rows, int L);
 size_t attn_workspace_bytes(long long rows, int L, int H, int k);
 
 // tcgen05 indexer (T == 1: decode, one query per MMA; T > 1: 8 queries per MMA).  With a

@@ -70,7 +70,9 @@ def test_sparse_attn_rejects(L):
     assert L.dsa_sparse_attn(None, FAKE, FAKE, 1, 1, 16, 64, 4, 0.1, FAKE, FAKE, 1 << 30, None) == -1
     assert L.dsa_sparse_attn(FAKE, FAKE, FAKE, 1, 1, 16, 20, 4, 0.1, FAKE, FAKE, 1 << 30, None) == -2
     assert L.dsa_sparse_attn(FAKE, FAKE, FAKE, 1, 1, 16, 64, 4096, 0.1, FAKE, FAKE, 1 << 30, None) == -2
-    assert L.dsa_sparse_attn(FAKE, FAKE, FAKE, 4, 1, 16, 64, 2048, 0.1, FAKE, None, 0, None) == -3
+    # unaligned output
+    assert L.dsa_sparse_attn(FAKE, FAKE, FAKE, 4, 1, 16, 64, 2048, 0.1, ctypes.c_void_p((1 << 20) + 4), None, 0,
+                             None) == -1
 
 
 def test_group_forward_rejects(L):
