@@ -64,6 +64,8 @@ static_assert(kSoftmaxWarp0 + 4 == kThreadsA / 32, "four softmax warps, one per 
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kPrefetchRounds = 2;               // L2 prefetch distance, in rounds of kStages tiles
 constexpr int kMaxSplits = 8;                    // key splits of one (row, layer): one portable cluster
+// float4 elements of the [64][512] output slice a thread sums when there are >= 2 splits
+constexpr int kPullPerThread = (64 * 128 / 2 + kThreadsA - 1) / kThreadsA;
 
 constexpr int kOffQ = 0;
 constexpr int kOffStage = kOffQ + kQBytes;
@@ -405,8 +407,10 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   }
   // O^T (TMEM lane = value dim, column = head) -> staging [64 heads][512] f32 over the idle
   // Q and stage buffers.  Twelve warps, three per TMEM lane quarter, take the eight
-  // 32-column chunks (value block mb, head half) two loads at a time.
+  // 32-column chunks (value block mb, head half) two loads at a time.  A single split
+  // (no cluster peers) applies its normaliser here and stores the staging directly.
   float* stg = reinterpret_cast<float*>(smem + kOffQ);
+  if (nsplit == 1) __syncthreads();  // s_coef
   if (warp != kMmaWarp) {
     const int quarter = warp & 3;
     const int j = warp < kProducerWarps ? warp >> 2 : 2;
@@ -421,6 +425,22 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
       } else {
 #pragma unroll
         for (int c2 = 0; c2 < 32; ++c2) o0[c2] = o1[c2] = 0u;
+      }
+      if (nsplit == 1) {
+        // the normalisers of these columns' heads, in registers before the stores
+#pragma unroll
+        for (int c4 = 0; c4 < 8; ++c4) {
+          const float4 v0 = reinterpret_cast<const float4*>(s_coef + 32 * (c & 1))[c4];
+          o0[4 * c4] = __float_as_uint(__uint_as_float(o0[4 * c4]) * v0.x);
+          o0[4 * c4 + 1] = __float_as_uint(__uint_as_float(o0[4 * c4 + 1]) * v0.y);
+          o0[4 * c4 + 2] = __float_as_uint(__uint_as_float(o0[4 * c4 + 2]) * v0.z);
+          o0[4 * c4 + 3] = __float_as_uint(__uint_as_float(o0[4 * c4 + 3]) * v0.w);
+          const float4 v1 = reinterpret_cast<const float4*>(s_coef + 32 * ((c + 3) & 1))[c4];
+          o1[4 * c4] = __float_as_uint(__uint_as_float(o1[4 * c4]) * v1.x);
+          o1[4 * c4 + 1] = __float_as_uint(__uint_as_float(o1[4 * c4 + 1]) * v1.y);
+          o1[4 * c4 + 2] = __float_as_uint(__uint_as_float(o1[4 * c4 + 2]) * v1.z);
+          o1[4 * c4 + 3] = __float_as_uint(__uint_as_float(o1[4 * c4 + 3]) * v1.w);
+        }
       }
       float* d0 = stg + (32 * (c & 1)) * kDv + 128 * (c >> 1) + 32 * quarter + lane;
 #pragma unroll
@@ -439,25 +459,37 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     const int total = H * (kDv / 4);
     const int e0 = (int)((long long)split * total / nsplit), e1 = (int)((long long)(split + 1) * total / nsplit);
     const uint32_t stg_s = smem_u32(stg);
-#pragma unroll 2
-    for (int e = e0 + threadIdx.x; e < e1; e += kThreadsA) {
-      const int h = e >> 7;
-      const uint32_t off = stg_s + 16u * (uint32_t)e;
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (nsplit > 1) {
+      // all loads of this thread's elements (at most kPullPerThread) are issued before
+      // any result is written back
+      float4 acc[kPullPerThread];
 #pragma unroll
-      for (int sp = 0; sp < kMaxSplits; ++sp) {
-        if (sp < nsplit) {
-          const float cf = s_coef[sp * 64 + h];
-          const float4 v = ld_cluster_v4(cluster_map(off, sp));
-          acc.x = fmaf(cf, v.x, acc.x);
-          acc.y = fmaf(cf, v.y, acc.y);
-          acc.z = fmaf(cf, v.z, acc.z);
-          acc.w = fmaf(cf, v.w, acc.w);
+      for (int q = 0; q < kPullPerThread; ++q) {
+        const int e = e0 + (int)threadIdx.x + q * kThreadsA;
+        acc[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e < e1) {
+          const int h = e >> 7;
+          const uint32_t off = stg_s + 16u * (uint32_t)e;
+#pragma unroll
+          for (int sp = 0; sp < kMaxSplits; ++sp) {
+            if (sp < nsplit) {
+              const float cf = s_coef[sp * 64 + h];
+              const float4 v = ld_cluster_v4(cluster_map(off, sp));
+              acc[q].x = fmaf(cf, v.x, acc[q].x);
+              acc[q].y = fmaf(cf, v.y, acc[q].y);
+              acc[q].z = fmaf(cf, v.z, acc[q].z);
+              acc[q].w = fmaf(cf, v.w, acc[q].w);
+            }
+          }
         }
       }
-      reinterpret_cast<float4*>(stg)[e] = acc;
+#pragma unroll
+      for (int q = 0; q < kPullPerThread; ++q) {
+        const int e = e0 + (int)threadIdx.x + q * kThreadsA;
+        if (e < e1) reinterpret_cast<float4*>(stg)[e] = acc[q];
+      }
     }
-    fence_proxy_async();  // the sums are visible to the bulk copy (async proxy)
+    fence_proxy_async();  // the results are visible to the bulk copy (async proxy)
     __syncthreads();
     if (threadIdx.x == 0 && e1 > e0) {
       bulk_store(layers.out[layer] + (size_t)row * H * kDv + 4 * (size_t)e0, stg_s + 16u * (uint32_t)e0,
