@@ -66,6 +66,13 @@ typedef enum {
 /* Human-readable name of a dsa_status value. */
 const char *dsa_status_string(int status);
 
+/*
+ * The cudaError_t of the most recent call (on any thread) that returned DSA_ERR_CUDA, or 0
+ * if none has; and the runtime's description of such a code.
+ */
+int dsa_last_cuda_error(void);
+const char *dsa_cuda_error_string(int code);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int dsa_version(void);
 

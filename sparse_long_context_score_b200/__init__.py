@@ -29,7 +29,8 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
 
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_topk",
-           "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error")
+           "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error",
+           "dsa_last_cuda_error", "dsa_cuda_error_string")
 
 
 class DsaError(RuntimeError):
@@ -62,6 +63,10 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk_noalloc.argtypes = [P, I, I, I, LL, I, P, P]
         L.dsa_device_error.argtypes = [ctypes.POINTER(I), I]
         L.dsa_device_error.restype = I
+        L.dsa_last_cuda_error.argtypes = []
+        L.dsa_last_cuda_error.restype = I
+        L.dsa_cuda_error_string.argtypes = [I]
+        L.dsa_cuda_error_string.restype = ctypes.c_char_p
         for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc"):
             getattr(L, f).restype = I
         _lib = L
@@ -104,6 +109,9 @@ def _bf16_types():
 
 def _check(rc: int, where: str) -> None:
     if rc != DSA_OK:
+        if rc == -4:  # DSA_ERR_CUDA: name the CUDA error behind it
+            code = lib().dsa_last_cuda_error()
+            where = f"{where} (CUDA error {code}: {lib().dsa_cuda_error_string(code).decode()})"
         raise DsaError(rc, where)
 
 

@@ -13,6 +13,15 @@
 
 using namespace dsa;
 
+namespace dsa {
+std::atomic<int> g_last_cuda_error{0};
+dsa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return DSA_OK;
+  g_last_cuda_error.store((int)e, std::memory_order_relaxed);
+  return DSA_ERR_CUDA;
+}
+}  // namespace dsa
+
 namespace {
 
 inline bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -26,8 +35,6 @@ bool sizes_ok(int B, int T, int N) {
   if ((long long)N > 0x7FFFFFFFLL / 1) return false;
   return true;
 }
-
-dsa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA; }
 
 struct GroupLayout {
   size_t topk_off, topk_bytes, scores_off, scores_bytes, attn_off, attn_bytes, total;
@@ -52,6 +59,10 @@ bool heads_supported(int H) { return H == 16 || H == 32 || H == 48 || H == 64; }
 
 extern "C" {
 
+int dsa_last_cuda_error(void) { return g_last_cuda_error.load(std::memory_order_relaxed); }
+
+const char* dsa_cuda_error_string(int code) { return cudaGetErrorString((cudaError_t)code); }
+
 const char* dsa_status_string(int status) {
   switch (status) {
     case DSA_OK: return "DSA_OK";
@@ -71,8 +82,9 @@ dsa_status dsa_device_error(int* code, int clear) {
   if (!code) return DSA_ERR_INVALID_ARG;
   *code = 0;
   int a = 0;
-  if (indexer_tc_device_error(code, clear != 0) != cudaSuccess) return DSA_ERR_CUDA;
-  if (attn_tc_device_error(&a, clear != 0) != cudaSuccess) return DSA_ERR_CUDA;
+  cudaError_t e;
+  if ((e = indexer_tc_device_error(code, clear != 0)) != cudaSuccess) return cuda_status(e);
+  if ((e = attn_tc_device_error(&a, clear != 0)) != cudaSuccess) return cuda_status(e);
   if (!*code) *code = a;
   return *code ? DSA_ERR_TIMEOUT : DSA_OK;
 }
@@ -143,12 +155,13 @@ dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t*
     float* scores = reinterpret_cast<float*>(base + g.scores_off);
     // in decode the indexer folds the first radix digit of the select into its epilogue
     const bool fused_hist = T == 1 && B <= kNumSMs;
-    if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess) return DSA_ERR_CUDA;
+    if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess)
+      return cuda_status(e);
     if ((e = launch_index_score_tc(iq, w, ik, B, T, N, q_pos0, scores, fused_hist ? tws.hist : nullptr, stream)) !=
         cudaSuccess)
-      return DSA_ERR_CUDA;
+      return cuda_status(e);
     if ((e = launch_topk(scores, B, T, N, q_pos0, k, idx_shared, tws, fused_hist, stream)) != cudaSuccess)
-      return DSA_ERR_CUDA;
+      return cuda_status(e);
   }
   e = launch_sparse_attn_tc(layers, L, idx_shared, B, T, N, H, k, scale, base + g.attn_off, stream);
   return cuda_status(e);

@@ -28,6 +28,10 @@ struct DeviceOnce {
   }
 };
 
+// DSA_OK for cudaSuccess; otherwise records `e` as the last CUDA error (dsa_last_cuda_error)
+// and returns DSA_ERR_CUDA
+dsa_status cuda_status(cudaError_t e);
+
 constexpr int kIndexHeads = 32;   // index_n_heads
 constexpr int kIndexDim = 128;    // index_head_dim
 constexpr int kDqk = 576;         // compressed row: 512 latent + 64 rope
@@ -79,6 +83,12 @@ cudaError_t indexer_tc_device_error(int* code, bool clear);
 
 cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
                         const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream);
+// top-k of rows short enough for one cluster of CTAs (topk_cluster.cu); launch_topk
+// chooses it when topk_cluster_plan accepts the shape.  `hist` (nullable) holds the
+// first digit's histogram per row, counted by the indexer.
+bool topk_cluster_plan(long long rows, long long vmax, int* C, int* kpt);
+cudaError_t launch_topk_cluster(const float* scores, int B, int T, int N, long long q_pos0, int k, int C, int kpt,
+                                const uint32_t* hist, int32_t* idx, cudaStream_t stream);
 
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
                                   int k, float scale, void* ws, cudaStream_t stream);

@@ -53,8 +53,9 @@ extern "C" dsa_status dsa_topk_noalloc(const float* scores, int B, int T, int N,
   const long long rows = (long long)B * T;
   if (dsa::topk_workspace_bytes(rows, N) > kScratchBytes) return DSA_ERR_WORKSPACE;
   void* scratch = nullptr;
-  if (g_scratch_address.get(&scratch) != cudaSuccess) return DSA_ERR_CUDA;
+  const cudaError_t ea = g_scratch_address.get(&scratch);
+  if (ea != cudaSuccess) return dsa::cuda_status(ea);
   dsa::TopkWorkspace ws = dsa::topk_workspace(scratch, rows, N);
   const cudaError_t e = dsa::launch_topk(scores, B, T, N, q_pos0, k, idx, ws, false, stream);
-  return e == cudaSuccess ? DSA_OK : DSA_ERR_CUDA;
+  return dsa::cuda_status(e);
 }

@@ -187,7 +187,7 @@ __device__ uint64_t resolve_threshold(SelectSmem& sm, long long count, uint32_t 
 
 __global__ void __launch_bounds__(kSelThreads)
 topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, int k, TopkWorkspace ws,
-                   int32_t* __restrict__ idx_out) {
+                   int32_t* __restrict__ idx_out, int vec) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
   const int row = blockIdx.x;
@@ -225,7 +225,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
     // element i of this thread: four consecutive scores per 16-byte group
     return s0 + 4LL * (threadIdx.x + kSelThreads * (i >> 2)) + (i & 3);
   };
-  if ((N & 3) == 0) {
+  if (vec) {
     float4 v[kPerThread / 4];
 #pragma unroll
     for (int g = 0; g < kPerThread / 4; ++g) {
@@ -380,7 +380,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
 
 __global__ void __launch_bounds__(kCmpThreads)
 topk_compact_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, int k, TopkWorkspace ws,
-                    int32_t* __restrict__ idx_out) {
+                    int32_t* __restrict__ idx_out, int vec) {
   const int row = blockIdx.x;
   const int chunk = blockIdx.y;
   const int nchunks = gridDim.y;
@@ -409,7 +409,7 @@ topk_compact_kernel(const float* __restrict__ scores, int T, int N, long long q_
     return e < s1 && (take_all || composite(order_key(v), (uint32_t)e) >= thr);
   };
 
-  if ((N & 3) == 0) {
+  if (vec) {
     float4 v[kGroups];
 #pragma unroll
     for (int i = 0; i < kGroups; ++i) {
@@ -520,9 +520,10 @@ cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_po
   const long long rows = (long long)B * T;
   const long long vmax = visible_count(N, q_pos0, T - 1);
   const long long nchunks_all = ((long long)N + kTopkChunk - 1) / kTopkChunk;
-  const long long nchunks_vis = (vmax + kTopkChunk - 1) / kTopkChunk;
-  (void)nchunks_vis;
   cudaError_t e;
+  int C = 0, kpt = 0;
+  if (topk_cluster_plan(rows, vmax, &C, &kpt))
+    return launch_topk_cluster(scores, B, T, N, q_pos0, k, C, kpt, hist_ready ? ws.hist : nullptr, idx, stream);
   if (!hist_ready) {
     e = cudaMemsetAsync(ws.hist, 0, ws.zero_bytes, stream);
     if (e != cudaSuccess) return e;
@@ -530,6 +531,8 @@ cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_po
                                                                                                 ws.hist);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
+  // float4 loads need 16-byte aligned rows
+  const int vec = (N & 3) == 0 && (reinterpret_cast<uintptr_t>(scores) & 15) == 0;
   // the select kernel needs every chunk of the row to take a ticket, so it runs over all
   // chunks of N (chunks past the visible range count nothing)
   const size_t smem = sizeof(SelectSmem);
@@ -539,10 +542,10 @@ cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_po
        })) != cudaSuccess)
     return e;
   topk_select_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kSelThreads, smem, stream>>>(scores, T, N, q_pos0,
-                                                                                                  k, ws, idx);
+                                                                                                  k, ws, idx, vec);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   topk_compact_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kCmpThreads, 0, stream>>>(scores, T, N, q_pos0,
-                                                                                                k, ws, idx);
+                                                                                                k, ws, idx, vec);
   return cudaGetLastError();
 }
 

@@ -63,6 +63,10 @@ def _score_rows(seed, B, T, N, levels):
     (2, 1, 70000, 69999, 2048, 3000), (1, 1, 200, 199, 2048, 10), (1, 1, 1, 0, 1, 5), (2, 1, 8193, 8192, 7, 100),
     (1, 1, 33000, 32999, 1, 1 << 22), (1, 9, 3000, 2990, 2048, 1000), (1, 4, 20000, 2040, 2048, 1 << 20),
     (1, 1, 50000, 49999, 2048, 1),
+    # one cluster of 8 CTAs with 32 keys per thread; equal keys down to the index digits
+    (1, 1, 200000, 199999, 2048, 1 << 18), (2, 1, 150000, 149999, 2048, 3),
+    # shapes for the scan kernels: more rows than one wave of clusters, rows too long
+    (1, 160, 3000, 2900, 256, 1000), (1, 1, 300000, 299999, 2048, 1 << 20), (1, 1, 300000, 299999, 2048, 7),
 ])
 def test_topk_exact(dsa, orc, B, T, N, q_pos0, k, levels):
     sc = _score_rows(N + k + levels, B, T, N, levels)
