@@ -9,18 +9,23 @@
 // positions [r * chunk, (r + 1) * chunk) in shared memory (chunk = 1024 threads x kpt), so
 // the scores are read from memory once.  Radix select, most significant digit first, over
 // the 64-bit composite (digits of 12, 10, 10, 11, 11, 10 bits):
-//   - each CTA histograms the digit of its elements that still match the prefix found
-//     so far; the cluster adds the histograms through distributed shared memory (CTA r
-//     sums bins [r * bins / C, (r + 1) * bins / C) over the peers, then every CTA reads all
-//     the sums) and every CTA finds the same digit -- the bin where the count from the top
-//     reaches the rank still needed.  The first digit's histogram may come ready-made
-//     from the indexer epilogue;
-//   - once the bin holds at most kFinal elements, they are gathered into every CTA and
-//     ranked directly, which gives the threshold composite exactly;
-//   - every CTA counts its selected elements, takes the counts of the lower ranks as its
-//     output offset and writes its positions in order (warp ballots).
+//   - first digit (the top 12 key bits): its per-row histogram comes from the indexer
+//     epilogue, or the CTAs histogram their chunks and sum the histograms through
+//     distributed shared memory (CTA r adds up bins [r * 4096 / C, (r + 1) * 4096 / C) of
+//     every peer, then every CTA reads all the sums).  Every CTA finds the same threshold
+//     bin b*: the bin where the count from the top reaches k.  From then on a thread only
+//     looks at its elements with bin >= b* (a bit mask in a register): the selected
+//     elements are among them;
+//   - later digits: each CTA histograms the digit of its elements that still match the
+//     prefix and adds the non-empty bins into the bin's owner CTA (remote reductions into
+//     shared memory); one cluster barrier later every CTA reads the sums it needs;
+//   - the digits stop once every element of the bin is needed (at the latest when the
+//     64 bits are fixed: composites are distinct); the threshold is then the prefix;
+//   - every CTA sends its selected count to every peer, takes the counts of the lower
+//     ranks as its output offset and writes its positions in order (warp ballots).
 // No global workspace, no atomics on global memory and a single launch.  Every thread
-// passes every cluster barrier: the control flow depends only on cluster-wide sums.
+// passes every cluster barrier: the control flow depends only on cluster-wide sums, and
+// no CTA touches another's shared memory after the last barrier.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 #include "sm100.cuh"
@@ -34,45 +39,35 @@ using namespace sm100;
 constexpr int kCT = 1024;              // threads per CTA
 constexpr int kCWarps = kCT / 32;
 constexpr int kMaxBins = 1 << 12;
-constexpr int kFinal = 512;            // final-bin sizes ranked directly
+constexpr int kMaxC = 8;
 constexpr int kLevels = 6;
 __constant__ int kDigitWidth[kLevels] = {12, 10, 10, 11, 11, 10};
 
 struct ClusterSmem {
-  uint32_t h[kMaxBins];                // this CTA's histogram of the current digit
-  uint32_t part[kMaxBins];             // cluster sums of the bins this CTA owns
-  uint32_t full[kMaxBins];             // cluster sums of every bin (local copy)
-  unsigned long long fin[kFinal];      // this CTA's composites in the final bin
-  unsigned long long all[kFinal];      // the whole cluster's, gathered
+  uint32_t h[kMaxBins];                   // first digit counted here: this CTA's histogram
+  uint32_t part[kMaxBins];                // ... the cluster sums of the bins this CTA owns
+  uint32_t full0[kMaxBins];               // ... the cluster sums of every bin
+  uint32_t hl[2048];                      // this CTA's histogram of a later digit
+  uint32_t fullb[3][2048];                // cluster sums of the later-digit bins this CTA owns
+  uint32_t nsel[kMaxC];                   // selected counts per sending rank
   uint32_t warp_tmp[kCWarps];
-  uint32_t total;
-  uint32_t nfin;                       // read by the peers
-  uint32_t nsel;                       // read by the peers
-  uint32_t base;
-  uint32_t peer_cnt[8], peer_off[8];
-  uint32_t digit, above, count;
-  unsigned long long thr;
+  uint32_t res[3];                        // digit search: digit, above, count
 };
 
 // the keys follow the struct, 16-byte aligned (they are written as uint4)
 constexpr int kKeysOff = ((int)sizeof(ClusterSmem) + 127) & ~127;
 static_assert(kKeysOff % 16 == 0, "uint4 key stores");
 
-__device__ __forceinline__ uint32_t ld_cluster_u32(uint32_t addr) {
-  uint32_t v;
-  asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ unsigned long long ld_cluster_u64(uint32_t addr) {
-  unsigned long long v;
-  asm volatile("ld.shared::cluster.u64 %0, [%1];" : "=l"(v) : "r"(addr));
-  return v;
-}
-
-// Exclusive scan of one value per thread over the CTA (kCT threads); *total gets the sum.
-__device__ __forceinline__ uint32_t scan_excl(uint32_t v, ClusterSmem& sm) {
+// Thread t owns bins [bins - (t + 1) * per, bins - t * per) of a histogram (per = bins /
+// kCT, 1..4) and holds their counts in v[0..per), highest bin first.  Finds the bin d where
+// the count from the top reaches r: above(d) < r <= above(d) + count(d).  Two barriers.
+__device__ __forceinline__ void digit_search(const uint32_t (&v)[4], int per, int bins, uint32_t r, ClusterSmem& sm,
+                                             uint32_t& d, uint32_t& above, uint32_t& count) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t x = v;
+  uint32_t lsum = 0;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) lsum += i < per ? v[i] : 0u;
+  uint32_t x = lsum;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
@@ -80,59 +75,35 @@ __device__ __forceinline__ uint32_t scan_excl(uint32_t v, ClusterSmem& sm) {
   }
   if (lane == 31) sm.warp_tmp[warp] = x;
   __syncthreads();
-  if (warp == 0) {
-    const uint32_t wv = sm.warp_tmp[lane];
-    uint32_t z = wv;
+  const uint32_t wt = sm.warp_tmp[lane];
+  uint32_t z = wt;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, z, o);
-      if (lane >= o) z += y;
-    }
-    sm.warp_tmp[lane] = z - wv;
-    if (lane == 31) sm.total = z;
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, z, o);
+    if (lane >= o) z += y;
   }
-  __syncthreads();
-  const uint32_t r = sm.warp_tmp[warp] + x - v;
-  __syncthreads();
-  return r;
-}
-
-// In the histogram `hist` of `bins` bins (bins >= kCT / 8 ... kMaxBins), find the digit d
-// where the count from the top reaches r: above(d) < r <= above(d) + hist[d].  Results in
-// sm.digit / sm.above / sm.count.  Every thread of the CTA calls it.
-__device__ void digit_search(const uint32_t* hist, int bins, uint32_t r, ClusterSmem& sm) {
-  const int per = bins >= kCT ? bins / kCT : 1;
-  const int hi = bins - (int)threadIdx.x * per;  // this thread owns bins [hi - per, hi)
-  uint32_t local[4];
-  uint32_t lsum = 0;
+  uint32_t run = __shfl_sync(0xFFFFFFFFu, z - wt, warp) + x - lsum;
+  const int hi = bins - (int)threadIdx.x * per;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const int b = hi - 1 - i;
-    local[i] = (i < per && b >= 0) ? hist[b] : 0u;
-    lsum += local[i];
-  }
-  if (threadIdx.x == 0) {
-    sm.digit = 0;
-    sm.above = 0;
-    sm.count = 0;
-  }
-  uint32_t run = scan_excl(lsum, sm);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (i < per && hi - 1 - i >= 0 && run < r && run + local[i] >= r) {
-      sm.digit = (uint32_t)(hi - 1 - i);
-      sm.above = run;
-      sm.count = local[i];
+    if (i < per && run < r && run + v[i] >= r) {
+      sm.res[0] = (uint32_t)(hi - 1 - i);
+      sm.res[1] = run;
+      sm.res[2] = v[i];
     }
-    run += local[i];
+    run += i < per ? v[i] : 0u;
   }
   __syncthreads();
+  d = sm.res[0];
+  above = sm.res[1];
+  count = sm.res[2];
 }
 
-// Cluster-wide sum of every CTA's sm.h[0, bins) into every CTA's sm.full.
-__device__ void cluster_hist_sum(ClusterSmem& sm, int bins, int C, int me) {
+// First digit counted by the CTAs: cluster-wide sum of every CTA's sm.h into sm.full0.
+// CTA r adds up its share of the bins over all peers, then every CTA reads all the sums.
+__device__ void first_digit_sum(ClusterSmem& sm, int C, int me) {
   cluster_sync();  // every CTA's histogram is complete
-  const int bpc = bins / C;
+  const int bpc = kMaxBins / C;
   for (int b = threadIdx.x; b < bpc; b += kCT) {
     const uint32_t a = smem_u32(&sm.h[me * bpc + b]);
     uint32_t s = 0;
@@ -140,9 +111,9 @@ __device__ void cluster_hist_sum(ClusterSmem& sm, int bins, int C, int me) {
     sm.part[b] = s;
   }
   cluster_sync();  // every owner's sums are complete
-  for (int b = threadIdx.x; b < bins; b += kCT) {
+  for (int b = threadIdx.x; b < kMaxBins; b += kCT) {
     const int owner = b / bpc;
-    sm.full[b] = ld_cluster_u32(cluster_map(smem_u32(&sm.part[b - owner * bpc]), owner));
+    sm.full0[b] = ld_cluster_u32(cluster_map(smem_u32(&sm.part[b - owner * bpc]), owner));
   }
   __syncthreads();
 }
@@ -155,7 +126,8 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   ClusterSmem& sm = *reinterpret_cast<ClusterSmem*>(smem_raw);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kKeysOff);
   constexpr int kChunk = kCT * KPT;
-  constexpr int kSeg = 32 * KPT;  // positions of one warp, processed 32 at a time
+  constexpr int kSeg = 32 * KPT;  // positions of one warp, taken 32 at a time (bit `step` of a mask)
+  static_assert(KPT % 4 == 0 && KPT <= 32, "keys per thread");
   const int C = (int)gridDim.x, me = (int)blockIdx.x, row = (int)blockIdx.y;
   const long long V = visible_count(N, q_pos0, row % T);
   const long long c0 = (long long)me * kChunk;
@@ -163,24 +135,6 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   const int seg0 = warp * kSeg;
   const float* sr = scores + (size_t)row * N;
   int32_t* out = idx_out + (size_t)row * k;
-
-  // this CTA's scores, read once, as order keys (positions >= V are never used)
-#pragma unroll
-  for (int i = 0; i < KPT / 4; ++i) {
-    const int p = seg0 + 128 * i + 4 * lane;
-    const long long s = c0 + p;
-    float4 v;
-    if (vec && s + 3 < V) {
-      v = __ldcg(reinterpret_cast<const float4*>(sr + s));
-    } else {
-      v.x = s < V ? __ldcg(sr + s) : 0.f;
-      v.y = s + 1 < V ? __ldcg(sr + s + 1) : 0.f;
-      v.z = s + 2 < V ? __ldcg(sr + s + 2) : 0.f;
-      v.w = s + 3 < V ? __ldcg(sr + s + 3) : 0.f;
-    }
-    *reinterpret_cast<uint4*>(keys + p) = make_uint4(order_key(v.x), order_key(v.y), order_key(v.z), order_key(v.w));
-  }
-  __syncwarp();  // a warp only ever reads the keys of its own segment
 
   if (V <= k) {
     // every visible position is kept, in order; the rest of the row is padding
@@ -194,125 +148,157 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
     return;
   }
 
+  // loads in flight together: the first digit's histogram (this thread's four bins,
+  // highest first) and this CTA's scores
+  uint32_t hv[4] = {0u, 0u, 0u, 0u};
+  if (hist_g) {
+    const uint4 q = __ldcg(reinterpret_cast<const uint4*>(hist_g + (size_t)row * kHistBins + kHistBins -
+                                                          4 * (threadIdx.x + 1)));
+    hv[0] = q.w;
+    hv[1] = q.z;
+    hv[2] = q.y;
+    hv[3] = q.x;
+  }
+  float4 v[KPT / 4];
+#pragma unroll
+  for (int i = 0; i < KPT / 4; ++i) {
+    const long long s = c0 + seg0 + 128 * i + 4 * lane;
+    if (vec && s + 3 < V) {
+      v[i] = __ldcg(reinterpret_cast<const float4*>(sr + s));
+    } else {
+      v[i].x = s < V ? __ldcg(sr + s) : 0.f;
+      v[i].y = s + 1 < V ? __ldcg(sr + s + 1) : 0.f;
+      v[i].z = s + 2 < V ? __ldcg(sr + s + 2) : 0.f;
+      v[i].w = s + 3 < V ? __ldcg(sr + s + 3) : 0.f;
+    }
+  }
+  // the later-digit histograms the peers add into start at zero: barrier S0 (arrive now,
+  // wait before the first access to another CTA's shared memory)
+  for (int i = threadIdx.x; i < 2048; i += kCT) sm.fullb[1][i] = 0u;
+  cluster_arrive();
+  bool s0_pending = true;
+  auto wait_s0 = [&] {
+    if (s0_pending) {
+      cluster_wait();
+      s0_pending = false;
+    }
+  };
+#pragma unroll
+  for (int i = 0; i < KPT / 4; ++i)
+    *reinterpret_cast<uint4*>(keys + seg0 + 128 * i + 4 * lane) =
+        make_uint4(order_key(v[i].x), order_key(v[i].y), order_key(v[i].z), order_key(v[i].w));
+  __syncwarp();  // a warp only ever reads the keys of its own segment
+
   auto comp = [&](int p) -> unsigned long long {
     return ((unsigned long long)keys[p] << 32) | (unsigned long long)(0xFFFFFFFFu - (uint32_t)(c0 + p));
   };
 
-  // radix select over the composite, one digit per level, until the bin is small
-  unsigned long long prefix = 0;
-  int pos = 64;              // bits [pos, 64) of the threshold are fixed in `prefix`
-  uint32_t r = (uint32_t)k;  // rank still needed inside the current bin (1-based)
-  for (int level = 0; level < kLevels; ++level) {
+  // first digit: the threshold bin b*
+  uint32_t d, above, count;
+  if (!hist_g) {
+    for (int b = threadIdx.x; b < kMaxBins; b += kCT) sm.h[b] = 0u;
+    __syncthreads();
+#pragma unroll 4
+    for (int step = 0; step < KPT; ++step) {
+      const int p = seg0 + 32 * step + lane;
+      if (c0 + p < V) atomicAdd(&sm.h[keys[p] >> kHistShift], 1u);
+    }
+    wait_s0();
+    first_digit_sum(sm, C, me);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) hv[i] = sm.full0[kMaxBins - 1 - 4 * (int)threadIdx.x - i];
+  }
+  digit_search(hv, 4, kMaxBins, (uint32_t)k, sm, d, above, count);
+  uint32_t r = (uint32_t)k - above;  // rank still needed inside the current bin (1-based)
+  unsigned long long prefix = (unsigned long long)d << 52;
+  int pos = 52;                      // bits [pos, 64) of the threshold are fixed in `prefix`
+  const uint32_t bstar = d;
+
+  // the elements that can be selected: bin >= b*
+  uint32_t cand = 0;
+#pragma unroll
+  for (int step = 0; step < KPT; ++step) {
+    const int p = seg0 + 32 * step + lane;
+    if (c0 + p < V && (keys[p] >> kHistShift) >= bstar) cand |= 1u << step;
+  }
+
+  // later digits, until every element of the bin is needed: then the threshold is the
+  // prefix itself.  Each CTA adds its non-empty bins into the bin's owner (CTA
+  // bin / (bins / C), triple-buffered arrays), and after one barrier every CTA reads the
+  // sums of the bins it scans from their owners.
+  for (int level = 1; level < kLevels && count != r; ++level) {
     const int width = kDigitWidth[level];
     const int shift = pos - width;
     const int bins = 1 << width;
-    if (level == 0 && hist_g) {
-      for (int b = threadIdx.x; b < bins; b += kCT) sm.full[b] = __ldcg(&hist_g[(size_t)row * kHistBins + b]);
-      __syncthreads();
-    } else {
-      for (int b = threadIdx.x; b < bins; b += kCT) sm.h[b] = 0;
-      __syncthreads();
-#pragma unroll 4
-      for (int step = 0; step < KPT; ++step) {
-        const int p = seg0 + 32 * step + lane;
-        if (c0 + p < V) {
-          const unsigned long long c = comp(p);
-          if (pos == 64 || (c >> pos) == (prefix >> pos))
-            atomicAdd(&sm.h[(uint32_t)(c >> shift) & (uint32_t)(bins - 1)], 1u);
-        }
-      }
-      cluster_hist_sum(sm, bins, C, me);
-    }
-    digit_search(sm.full, bins, r, sm);
-    r -= sm.above;
-    prefix |= (unsigned long long)sm.digit << shift;
-    pos = shift;
-    if (sm.count <= (uint32_t)kFinal) break;  // the last level leaves one element
-  }
-
-  // the final bin: gather its elements from the whole cluster and rank them
-  if (threadIdx.x == 0) sm.nfin = 0;
-  __syncthreads();
-#pragma unroll 4
-  for (int step = 0; step < KPT; ++step) {
-    const int p = seg0 + 32 * step + lane;
-    if (c0 + p < V) {
+    const int bpc = bins / C;
+    uint32_t* fb = sm.fullb[level % 3];
+    for (int b = threadIdx.x; b < bins; b += kCT) sm.hl[b] = 0u;
+    __syncthreads();
+    for (uint32_t m = cand; m; m &= m - 1) {
+      const int p = seg0 + 32 * (__ffs(m) - 1) + lane;
       const unsigned long long c = comp(p);
-      if ((c >> pos) == (prefix >> pos)) {
-        const uint32_t slot = atomicAdd(&sm.nfin, 1u);
-        if (slot < (uint32_t)kFinal) sm.fin[slot] = c;
-      }
+      if ((c >> pos) == (prefix >> pos)) atomicAdd(&sm.hl[(uint32_t)(c >> shift) & (uint32_t)(bins - 1)], 1u);
     }
-  }
-  __syncthreads();
-  cluster_sync();  // every CTA's final-bin list is complete
-  if (threadIdx.x < 32) {
-    uint32_t cnt = lane < C ? ld_cluster_u32(cluster_map(smem_u32(&sm.nfin), lane)) : 0u;
-    cnt = min(cnt, (uint32_t)kFinal);
-    uint32_t incl = cnt;
+    __syncthreads();
+    wait_s0();
+    for (int b = threadIdx.x; b < bins; b += kCT) {
+      const uint32_t x = sm.hl[b];
+      if (x) red_cluster_add(cluster_map(smem_u32(&fb[b % bpc]), b / bpc), x);
+    }
+    // the owned part of the next level's array: its last readers were done two barriers ago
+    for (int i = threadIdx.x; i < bpc; i += kCT) sm.fullb[(level + 1) % 3][i] = 0u;
+    cluster_sync();  // every addition is in its owner
+    const int per = bins / kCT;
+    uint32_t lv[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-      if (lane >= o) incl += y;
+    for (int i = 0; i < 4; ++i) {
+      const int b = bins - 1 - per * (int)threadIdx.x - i;
+      if (i < per) lv[i] = ld_cluster_u32(cluster_map(smem_u32(&fb[b % bpc]), b / bpc));
     }
-    if (lane < 8) {
-      sm.peer_cnt[lane] = cnt;
-      sm.peer_off[lane] = incl - cnt;
-    }
-    if (lane == 31) sm.total = incl;
+    digit_search(lv, per, bins, r, sm, d, above, count);
+    r -= above;
+    prefix |= (unsigned long long)d << shift;
+    pos = shift;
   }
-  __syncthreads();
-  const uint32_t nall = min(sm.total, (uint32_t)kFinal);
-  for (int p = 0; p < C; ++p) {
-    const uint32_t cnt = sm.peer_cnt[p], off = sm.peer_off[p];
-    for (uint32_t i = threadIdx.x; i < cnt && off + i < (uint32_t)kFinal; i += kCT)
-      sm.all[off + i] = ld_cluster_u64(cluster_map(smem_u32(&sm.fin[i]), p));
-  }
-  if (threadIdx.x == 0) sm.thr = 0;
-  __syncthreads();
-  for (uint32_t i = threadIdx.x; i < nall; i += kCT) {
-    const unsigned long long c = sm.all[i];
-    uint32_t rank = 0;
-    for (uint32_t j = 0; j < nall; ++j) rank += sm.all[j] > c ? 1u : 0u;
-    if (rank == r - 1) sm.thr = c;  // composites are distinct: exactly one thread writes
-  }
-  __syncthreads();
-  const unsigned long long thr = sm.thr;
+  wait_s0();
+  const unsigned long long thr = prefix;  // every element of the final bin is selected
 
-  // selected = composite >= thr; output offset = selected count of the lower ranks
-  uint32_t wcnt = 0;
+  // selected = composite >= thr (all have bin >= b*); output offset = the selected count
+  // of the lower ranks, then of the lower warps
+  uint32_t sel = 0;
+  for (uint32_t m = cand; m; m &= m - 1) {
+    const int step = __ffs(m) - 1;
+    if (comp(seg0 + 32 * step + lane) >= thr) sel |= 1u << step;
+  }
+  uint32_t wcnt = __popc(sel);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) wcnt += __shfl_xor_sync(0xFFFFFFFFu, wcnt, o);
+  if (lane == 0) sm.warp_tmp[warp] = wcnt;
+  __syncthreads();
+  const uint32_t wt = sm.warp_tmp[lane];
+  uint32_t z = wt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, z, o);
+    if (lane >= o) z += y;
+  }
+  const uint32_t wbase = __shfl_sync(0xFFFFFFFFu, z - wt, warp);
+  const uint32_t cta_total = __shfl_sync(0xFFFFFFFFu, z, 31);
+  if (threadIdx.x < C) st_cluster_u32(cluster_map(smem_u32(&sm.nsel[me]), threadIdx.x), cta_total);
+  cluster_sync();  // every CTA's count is in every CTA; no shared-memory access across CTAs after this
+  uint32_t o = wbase;
+  for (int q = 0; q < me; ++q) o += sm.nsel[q];
 #pragma unroll 4
   for (int step = 0; step < KPT; ++step) {
-    const int p = seg0 + 32 * step + lane;
-    const bool sel = c0 + p < V && comp(p) >= thr;
-    wcnt += __popc(__ballot_sync(0xFFFFFFFFu, sel));
-  }
-  uint32_t wbase = scan_excl(lane == 0 ? wcnt : 0u, sm);
-  wbase = __shfl_sync(0xFFFFFFFFu, wbase, 0);
-  if (threadIdx.x == 0) sm.nsel = sm.total;
-  __syncthreads();
-  cluster_sync();  // every CTA's selected count is published
-  if (threadIdx.x == 0) {
-    uint32_t b = 0;
-    for (int p = 0; p < me; ++p) b += ld_cluster_u32(cluster_map(smem_u32(&sm.nsel), p));
-    sm.base = b;
-  }
-  __syncthreads();
-  uint32_t o = sm.base + wbase;
-#pragma unroll 4
-  for (int step = 0; step < KPT; ++step) {
-    const int p = seg0 + 32 * step + lane;
-    const bool sel = c0 + p < V && comp(p) >= thr;
-    const uint32_t m = __ballot_sync(0xFFFFFFFFu, sel);
-    if (sel) {
+    const bool b = (sel >> step) & 1u;
+    const uint32_t m = __ballot_sync(0xFFFFFFFFu, b);
+    if (b) {
       const uint32_t at = o + __popc(m & ((1u << lane) - 1u));
-      if (at < (uint32_t)k) out[at] = (int32_t)(c0 + p);
+      if (at < (uint32_t)k) out[at] = (int32_t)(c0 + seg0 + 32 * step + lane);
     }
     o += __popc(m);
   }
-  cluster_sync();  // the peers are done reading this CTA's shared memory
 }
-
 template <int KPT>
 cudaError_t launch_kpt(const float* scores, long long rows, int T, int N, long long q_pos0, int k, int C,
                        const uint32_t* hist, int32_t* idx, cudaStream_t stream) {
