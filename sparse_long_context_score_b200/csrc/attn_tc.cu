@@ -94,7 +94,7 @@ struct AttnMaps {
 
 __global__ void __launch_bounds__(kThreadsA, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const int32_t* __restrict__ idx, int T, int N,
-               int H, int k, int chunk, float scale_log2, int* __restrict__ err) {
+               int H, int k, int chunk, float scale_log2, int q_early, int* __restrict__ err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -162,10 +162,17 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     // four tiles are in flight and each is published as soon as it lands
     const int ps = warp >> 1, half = warp & 1;
     if (warp == 0 && lane == 0) {
+      // the queries may be read before the preceding kernel completes only when the caller
+      // knows that kernel does not write them (the top-k of the same group)
+      if (!q_early) grid_dep_wait();
       const CUtensorMap* qm = &maps.q[layer];
       mbar_arrive_expect_tx(qfull_bar, kQBytes);
       for (int kb = 0; kb < kBlocks; ++kb) tma_load_2d(sQ + kb * kQBlockBytes, qm, qfull_bar, 64 * kb, row * H);
     }
+    // the index list comes from the preceding kernel.  (Every other warp waits on the
+    // gather through the pipeline barriers, and the output is written only after the
+    // cluster barrier that follows this wait.)
+    grid_dep_wait();
     const int32_t* sel = idx + (size_t)row * k + j0;
     const uint16_t* kvb = layers.kv[layer] + (size_t)b * N * kDqk;
     const uint32_t st = sStage + ps * kStageBytes;
@@ -559,15 +566,49 @@ int attn_split_chunk(int k, int nsplit) {
   return (chunk + kAttnTile - 1) / kAttnTile * kAttnTile;
 }
 
-// Splits per (query row, layer): about one CTA per SM in total, at most one cluster's worth.
-int attn_num_splits(long long rows, int L, int k) {
-  const long long units = rows * L;
-  long long ns = kNumSMs / (units > 0 ? units : 1);
-  if (ns < 1) ns = 1;
-  if (ns > kMaxSplits) ns = kMaxSplits;
+namespace {
+// How many clusters of each size (1..kMaxSplits) of this kernel fit on the GPU at once,
+// per device; filled on the first launch on a device (before any stream capture).
+int g_cluster_fit[64][kMaxSplits + 1];
+
+cudaError_t query_cluster_fit() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  for (int c = 1; c <= kMaxSplits; ++c) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(c, 1, 1);
+    cfg.blockDim = dim3(kThreadsA);
+    cfg.dynamicSmemBytes = kSmemA;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = c;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if ((e = cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg)) != cudaSuccess) return e;
+    g_cluster_fit[dev][c] = n;
+  }
+  return cudaSuccess;
+}
+}  // namespace
+
+// Splits per (query row, layer): the most (<= kMaxSplits, about one CTA per SM in total)
+// whose clusters all fit on the GPU at once -- a second wave of clusters would double
+// the time.  Without the device's figures (fit == nullptr) the SM count alone decides.
+int attn_num_splits(long long rows, int L, int k, const int* fit) {
+  const long long units = rows * L > 0 ? rows * L : 1;
   const long long max_ns = (k + kAttnTile - 1) / kAttnTile;
-  if (ns > max_ns) ns = max_ns;
-  const int chunk = attn_split_chunk(k, (int)ns);
+  int best = 1;
+  for (int ns = 1; ns <= kMaxSplits && ns <= max_ns; ++ns) {
+    if (units * ns > kNumSMs) break;
+    if (fit && fit[ns] > 0 && units > fit[ns]) continue;
+    best = ns;
+  }
+  const int chunk = attn_split_chunk(k, best);
   return (k + chunk - 1) / chunk;
 }
 
@@ -575,7 +616,7 @@ int attn_num_splits(long long rows, int L, int k) {
 size_t attn_workspace_bytes(long long, int, int, int) { return 0; }
 
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                                  int k, float scale, void*, cudaStream_t stream) {
+                                  int k, float scale, void*, bool q_early, cudaStream_t stream) {
   const long long rows = (long long)B * T;
   AttnMaps maps;
   for (int l = 0; l < L; ++l)
@@ -584,10 +625,14 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
   cudaError_t e = g_err_addr.get(&err);
   if (e != cudaSuccess) return e;
   static DeviceOnce once;
-  if ((e = once.run([] { return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA); })) !=
-      cudaSuccess)
+  if ((e = once.run([] {
+         cudaError_t e2 = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA);
+         return e2 != cudaSuccess ? e2 : query_cluster_fit();
+       })) != cudaSuccess)
     return e;
-  const int nsplit = attn_num_splits(rows, L, k);
+  int dev = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  const int nsplit = attn_num_splits(rows, L, k, dev >= 0 && dev < 64 ? g_cluster_fit[dev] : nullptr);
   const int chunk = attn_split_chunk(k, nsplit);
   // the splits of one (row, layer) are one cluster along x
   cudaLaunchConfig_t cfg = {};
@@ -595,15 +640,17 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
   cfg.blockDim = dim3(kThreadsA);
   cfg.dynamicSmemBytes = kSmemA;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = nsplit;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // waits in-kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f,
-                            err);
+                            q_early ? 1 : 0, err);
 }
 
 cudaError_t attn_tc_device_error(int* code, bool clear) {

@@ -124,7 +124,7 @@ dsa_status dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const int32_t*
   layers.q[0] = q;
   layers.kv[0] = kv;
   layers.out[0] = out;
-  return cuda_status(launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, workspace, stream));
+  return cuda_status(launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, workspace, false, stream));
 }
 
 dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t* ik, const uint16_t* const* q,
@@ -163,7 +163,8 @@ dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t*
     if ((e = launch_topk(scores, B, T, N, q_pos0, k, idx_shared, tws, fused_hist, stream)) != cudaSuccess)
       return cuda_status(e);
   }
-  e = launch_sparse_attn_tc(layers, L, idx_shared, B, T, N, H, k, scale, base + g.attn_off, stream);
+  e = launch_sparse_attn_tc(layers, L, idx_shared, B, T, N, H, k, scale, base + g.attn_off,
+                            /*q_early=*/compute_indices != 0, stream);
   return cuda_status(e);
 }
 

@@ -70,7 +70,7 @@ struct AttnLayers {
 
 constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core attention
 
-int attn_num_splits(long long rows, int L, int k);
+int attn_num_splits(long long rows, int L, int k, const int* cluster_fit);
 int attn_split_chunk(int k, int nsplit);
 size_t attn_workspace_bytes(long long rows, int L, int H, int k);
 
@@ -90,8 +90,10 @@ bool topk_cluster_plan(long long rows, long long vmax, int* C, int* kpt);
 cudaError_t launch_topk_cluster(const float* scores, int B, int T, int N, long long q_pos0, int k, int C, int kpt,
                                 const uint32_t* hist, int32_t* idx, cudaStream_t stream);
 
+// q_early: the kernel before it in the stream does not write the queries (it is the
+// group's own top-k), so they are loaded before that kernel completes
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                                  int k, float scale, void* ws, cudaStream_t stream);
+                                  int k, float scale, void* ws, bool q_early, cudaStream_t stream);
 cudaError_t attn_tc_device_error(int* code, bool clear);
 
 }  // namespace dsa

@@ -110,6 +110,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
                   const float* __restrict__ w, int B, int T, int N, long long q_pos0, long long total_items,
                   float* __restrict__ scores, uint32_t* __restrict__ hist, int* __restrict__ err) {
   using C = TcCfg<QG, kHist>;
+  grid_dep_launch();  // the top-k may be scheduled as SMs free up; it waits for these scores
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);

@@ -124,6 +124,15 @@ __device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence
 // generic-proxy shared-memory writes become visible to the async proxy (tcgen05.mma)
 __device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
+// ------------------------------------------------------------------------- dependent launch
+// Programmatic dependent launch: the next kernel of the stream (launched with programmatic
+// stream serialization) may be scheduled once every CTA of this grid has issued this or
+// exited; it still waits, with grid_dep_wait, for this grid to complete.
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+// Wait until the preceding grid of the stream has completed and its memory operations are
+// visible (returns at once when this grid was launched without the attribute).
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ------------------------------------------------------------------------- cluster
 // Barrier over every thread of every CTA of the cluster; the release/acquire pair makes
 // shared-memory writes before it visible to peers' reads after it.

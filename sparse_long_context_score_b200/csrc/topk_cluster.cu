@@ -135,6 +135,8 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   const int seg0 = warp * kSeg;
   const float* sr = scores + (size_t)row * N;
   int32_t* out = idx_out + (size_t)row * k;
+  grid_dep_launch();  // the attention may be scheduled on free SMs; it waits for this grid
+  grid_dep_wait();    // the scores (and the histogram) of the preceding kernel
 
   if (V <= k) {
     // every visible position is kept, in order; the rest of the row is padding
@@ -314,13 +316,15 @@ cudaError_t launch_kpt(const float* scores, long long rows, int T, int N, long l
   cfg.blockDim = dim3(kCT);
   cfg.dynamicSmemBytes = (size_t)smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // waits in-kernel
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<KPT>, scores, T, N, q_pos0, k, vec, hist, idx);
 }
 
