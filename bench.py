@@ -41,6 +41,9 @@ def parse():
     p.add_argument("--cpu-sample", type=int, default=2, help="sequences in the CPU-oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra", action="store_true", help="skip the 1M / MTP / prefill workloads")
+    p.add_argument("--ncu-case", choices=["indexer", "topk", "attn"],
+                   help="run one kernel of the decode step a few times on a profiler-sized case and exit "
+                        "(for ncu captures; prints no benchmark line)")
     return p.parse_args()
 
 
@@ -340,8 +343,54 @@ def cpu_baseline(w, n_seq):
                       f"outside the timed region; {tokens} token-groups timed in {elapsed:.1f} s"}
 
 
+def ncu_case(kind: str) -> None:
+    """A few launches of one kernel of the decode128k step, sized for an ncu capture: the
+    indexer and the top-k on the full decode128k shapes (268 MB of keys, 4 MB of scores),
+    the attention on 32 (row, layer) units as in the step (4 key splits each) over caches of
+    65536 rows (2.4 GB, larger than L2) instead of 131072."""
+    import torch
+    import synth
+    import synth.device as sd
+    import sparse_long_context_score_b200 as dsa
+    from synth import configs as C
+    w = C.WORKLOADS["decode128k"]
+    bf = torch.bfloat16
+    launches = 3
+    if kind in ("indexer", "topk"):
+        iq = sd.int17_bf16(torch.empty(w.B, 1, 32, 128, dtype=bf, device="cuda"), w.key(synth.KIND_IQ))
+        wt = sd.pow2_f32(torch.empty(w.B, 1, 32, dtype=torch.float32, device="cuda"), w.key(synth.KIND_W))
+        ik = sd.int17_bf16(torch.empty(w.B, w.N, 128, dtype=bf, device="cuda"), w.key(synth.KIND_IK))
+        sc = torch.empty(w.B, 1, w.N, dtype=torch.float32, device="cuda")
+        idx = torch.empty(w.B, 1, w.k, dtype=torch.int32, device="cuda")
+        ws = dsa.workspace(w.B, 1, w.N, w.k, w.H, w.L)
+        dsa.dsa_index_score(iq, wt, ik, w.q_pos0, scores=sc)
+        for _ in range(launches):
+            if kind == "indexer":
+                dsa.dsa_index_score(iq, wt, ik, w.q_pos0, scores=sc)
+            else:
+                dsa.dsa_topk(sc, w.q_pos0, w.k, idx=idx, ws=ws)
+    else:
+        rows, n = 32, 65536
+        q = sd.normal_bf16(torch.empty(rows, 1, w.H, 576, dtype=bf, device="cuda"), w.key(synth.KIND_Q))
+        kv = sd.normal_bf16(torch.empty(rows, n, 576, dtype=bf, device="cuda"), w.key(synth.KIND_KV))
+        g = torch.Generator(device="cpu").manual_seed(w.key(synth.KIND_SCORES) & 0x7FFFFFFF)
+        idx = torch.stack([torch.sort(torch.randperm(n, generator=g)[:w.k]).values for _ in range(rows)])
+        idx = idx.view(rows, 1, w.k).to(torch.int32).cuda()
+        out = torch.empty(rows, 1, w.H, 512, dtype=torch.float32, device="cuda")
+        for _ in range(launches):
+            dsa.dsa_sparse_attn(q, kv, idx, C.SCALE, out=out)
+    torch.cuda.synchronize()
+    err = dsa.dsa_device_error()
+    print(f"ncu case {kind}: {launches} launches, device error word {err}")
+    if err:
+        sys.exit(1)
+
+
 def main():
     args = parse()
+    if args.ncu_case:
+        ncu_case(args.ncu_case)
+        return
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -396,7 +445,7 @@ def main():
         "gpu_launches": 5 * w.groups * args.steps,
         "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic("indexer.cu", w.name), "launch_us": idx_ms * 1e3,
+                     "traffic": profiled_traffic("indexer_tc.cu", w.name), "launch_us": idx_ms * 1e3,
                      "algorithmic_bytes_per_launch": idx_bytes},
     }
     if not args.no_extra and args.workload == "decode128k":
