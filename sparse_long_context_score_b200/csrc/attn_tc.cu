@@ -232,29 +232,25 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true, false);  // V^T (M-major) x P (K-major)
     bool ok = mbar_wait(qfull_bar, 0, err, 22);
     const uint64_t dq = sdesc_kmajor_sw128(sQ);
-    for (int i = 0; i <= ntiles && ok; ++i) {
-      if (i < ntiles) {
-        const int s = i % kStages, sb = i & 1;
-        ok = mbar_wait(full_bar(s), (i / kStages) & 1, err, 23);
-        if (ok) ok = mbar_wait(sfree_bar(sb), ((i >> 1) & 1) ^ 1, err, 24);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t dS = tmem + kTmemS + kKeys * sb;
-        // descriptors differ only in their start address: compile-time offsets from a base
-        const uint64_t dk = sdesc_kmajor_sw128(sStage + s * kStageBytes);
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < 4 * kBlocks; ++kk)
-            mma_bf16(dS, dq + (uint64_t)((((kk >> 2) * kQBlockBytes) + (kk & 3) * 32) >> 4),
-                     dk + (uint64_t)((((kk >> 2) * kBlockBytes) + (kk & 3) * 32) >> 4), idS, kk > 0);
-          mma_commit(sfull_bar(sb));
-        }
-        __syncwarp();
+    const int leader_lane = __ffs(__ballot_sync(0xFFFFFFFFu, leader)) - 1;
+    // S(i) needs tile i in its stage and a free S buffer; PV(j) needs P(j).  Each is issued
+    // as soon as it can be, PV first: a stage is released by its PV, and waiting for the
+    // next tile's data before issuing the previous tile's PV would keep one of the four
+    // stages from gathering.  The leader polls; the warp follows its decisions.
+    int is = 0, ipv = 0;
+    long long idle_since = clock64();
+    int spins = 0;
+    while (ok && ipv < ntiles) {
+      bool pv_ready = false, s_ready = false;
+      if (leader) {
+        pv_ready = ipv < is && mbar_try_wait(pfull_bar(ipv & 1), (ipv >> 1) & 1);
+        s_ready = is < ntiles && mbar_try_wait(full_bar(is % kStages), (is / kStages) & 1) &&
+                  mbar_try_wait(sfree_bar(is & 1), ((is >> 1) & 1) ^ 1);
       }
-      if (i >= 1) {
-        const int jt = i - 1, sj = jt % kStages, pb = jt & 1;
-        ok = mbar_wait(pfull_bar(pb), (jt >> 1) & 1, err, 25);
-        if (!ok) break;
+      pv_ready = __shfl_sync(0xFFFFFFFFu, pv_ready, leader_lane);
+      s_ready = __shfl_sync(0xFFFFFFFFu, s_ready, leader_lane);
+      if (pv_ready) {
+        const int jt = ipv, sj = jt % kStages, pb = jt & 1;
         tc_fence_after();
         const uint64_t da = sdesc_mnmajor_sw128(sStage + sj * kStageBytes, kBlockBytes, 1024);
         const uint64_t dp = sdesc_kmajor_sw64(sP + pb * kPBytes);
@@ -270,6 +266,35 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
           mma_commit(empty_bar(sj));
         }
         __syncwarp();
+        ++ipv;
+      }
+      if (s_ready) {
+        const int i = is, st = i % kStages, sb = i & 1;
+        tc_fence_after();
+        const uint32_t dS = tmem + kTmemS + kKeys * sb;
+        // descriptors differ only in their start address: compile-time offsets from a base
+        const uint64_t dk = sdesc_kmajor_sw128(sStage + st * kStageBytes);
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < 4 * kBlocks; ++kk)
+            mma_bf16(dS, dq + (uint64_t)((((kk >> 2) * kQBlockBytes) + (kk & 3) * 32) >> 4),
+                     dk + (uint64_t)((((kk >> 2) * kBlockBytes) + (kk & 3) * 32) >> 4), idS, kk > 0);
+          mma_commit(sfull_bar(sb));
+        }
+        __syncwarp();
+        ++is;
+      }
+      if (pv_ready || s_ready) {
+        idle_since = clock64();
+        spins = 0;
+      } else if (++spins == 64) {
+        // bounded like every other wait: give up after kWaitLimitCycles without progress,
+        // or when another thread has already failed
+        spins = 0;
+        const bool late = __any_sync(0xFFFFFFFFu, clock64() - idle_since > kWaitLimitCycles);
+        const bool failed = __any_sync(0xFFFFFFFFu, *reinterpret_cast<volatile int*>(err) != 0);
+        if (late && leader) atomicCAS(err, 0, 23);
+        ok = !(late || failed);
       }
     }
     if (leader) {
