@@ -343,6 +343,26 @@ def cpu_baseline(w, n_seq):
                       f"outside the timed region; {tokens} token-groups timed in {elapsed:.1f} s"}
 
 
+def launches_per_group(w) -> int:
+    """libdsa kernels one dsa_group_forward launches: the indexer, the top-k (one cluster
+    kernel for decode-shaped rows, else a select and a compact kernel, plus a histogram
+    kernel when the indexer does not count the first digit) and one attention launch for
+    all layers.  Mirrors the shape rules of the library (topk_cluster_plan)."""
+    rows = w.B * w.T
+    vmax = min(w.N, w.q_pos0 + w.T)
+    cluster = False
+    for c in (1, 2, 4, 8):
+        per = -(-vmax // (c * 1024))
+        kp = 4 if per <= 4 else 8 if per <= 8 else 16 if per <= 16 else 32 if per <= 32 else 0
+        if kp == 0 or (kp == 32 and c < 8):
+            continue
+        cluster = rows * c <= 148
+        break
+    fused_hist = w.T == 1 and w.B <= 148
+    topk = 1 if cluster else (2 if fused_hist else 3)
+    return 1 + topk + 1
+
+
 def ncu_case(kind: str) -> None:
     """A few launches of one kernel of the decode128k step, sized for an ncu capture: the
     indexer and the top-k on the full decode128k shapes (268 MB of keys, 4 MB of scores),
@@ -442,7 +462,7 @@ def main():
         "clocks": clocks,
         "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * w.groups * args.steps,
+        "gpu_launches": launches_per_group(w) * w.groups * args.steps,
         "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": profiled_traffic("indexer_tc.cu", w.name), "launch_us": idx_ms * 1e3,

@@ -62,7 +62,9 @@ constexpr int kSoftmaxWarp0 = kProducerWarps + 1;
 constexpr int kThreadsA = (kProducerWarps + 5) * 32;  // 416
 static_assert(kSoftmaxWarp0 + 4 == kThreadsA / 32, "four softmax warps, one per TMEM lane quarter");
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kPrefetchRounds = 2;               // L2 prefetch distance, in rounds of kStages tiles
+// rounds of kStages tiles in the largest split (k <= kMaxTopk keys): the row indices a
+// gather lane holds in registers
+constexpr int kRounds = (kMaxTopk + kKeys * kStages - 1) / (kKeys * kStages);
 constexpr int kMaxSplits = 8;                    // key splits of one (row, layer): one portable cluster
 // float4 elements of the [64][512] output slice a thread sums when there are >= 2 splits
 constexpr int kPullPerThread = (64 * 128 / 2 + kThreadsA - 1) / kThreadsA;
@@ -180,23 +182,22 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     // column block and in-row offset of each are constants
     const int c0 = lane, c1 = lane + 32, c2 = lane + 64;
     const uint32_t kb0 = (c0 >> 3) * kBlockBytes, kb1 = (c1 >> 3) * kBlockBytes, kb2 = (c2 >> 3) * kBlockBytes;
-    // rows of this warp's tile i are pulled into L2 kPrefetchRounds rounds ahead, so the
-    // shared-memory gather of a tile mostly hits L2: L2 is the deep in-flight buffer the
-    // stage ring is too small to be
-    auto prefetch_tile = [&](int i) {
-      if (i < ntiles && lane < 16) {
-        const int key = i * kKeys + 16 * half + lane;
-        const int v = key < nkeys ? __ldg(&sel[key]) : -1;
-        if (v >= 0 && v < N) prefetch_l2(kvb + (size_t)v * kDqk, kDqk * 2);
-      }
-    };
+    // the row indices of all this warp's tiles (ps, ps + kStages, ...), loaded at once before
+    // the first tile: no dependent index load sits in front of a tile's copies
+    int pre[kRounds];
+#pragma unroll
+    for (int j = 0; j < kRounds; ++j) {
+      const int key = (ps + kStages * j) * kKeys + 16 * half + (lane & 15);
+      pre[j] = key < nkeys ? __ldg(&sel[key]) : -1;
+    }
     for (int i = ps; i < ntiles; i += kStages) {
       bool ok = true;
       if (lane == 0) ok = mbar_wait(empty_bar(ps), ((i / kStages) & 1) ^ 1, err, 21);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
-      const int key = i * kKeys + 16 * half + (lane & 15);
-      const int v = key < nkeys ? __ldg(&sel[key]) : -1;
+      const int v = pre[0];
+#pragma unroll
+      for (int j = 0; j + 1 < kRounds; ++j) pre[j] = pre[j + 1];
       const bool valid = v >= 0 && v < N;
       const int my_row = valid ? v : 0;
       const uint32_t m = __ballot_sync(0xFFFFFFFFu, valid) & 0xFFFFu;
@@ -212,12 +213,6 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         if (c2 < kDqk / 8) cp_async_16(rbase + kb2 + (((c2 & 7) ^ x) << 4), src + c2 * 8, 16);
       }
       cp_async_commit();
-      // prefetch while this tile's copies are in flight: the first time the next
-      // kPrefetchRounds rounds, afterwards the round that comes kPrefetchRounds later
-      if (i == ps)
-        for (int r = 1; r <= kPrefetchRounds; ++r) prefetch_tile(ps + r * kStages);
-      else
-        prefetch_tile(i + kPrefetchRounds * kStages);
       cp_async_wait<0>();
       fence_proxy_async();  // the copies are visible to the tensor core (async proxy)
       mbar_arrive(full_bar(ps));
