@@ -176,7 +176,10 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   }
   // the later-digit histograms the peers add into start at zero: barrier S0 (arrive now,
   // wait before the first access to another CTA's shared memory)
-  for (int i = threadIdx.x; i < 2048; i += kCT) sm.fullb[1][i] = 0u;
+  for (int i = threadIdx.x; i < 2048; i += kCT) {
+    sm.fullb[1][i] = 0u;
+    sm.hl[i] = 0u;  // the second digit is counted in the candidate pass below
+  }
   cluster_arrive();
   bool s0_pending = true;
   auto wait_s0 = [&] {
@@ -216,12 +219,19 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   int pos = 52;                      // bits [pos, 64) of the threshold are fixed in `prefix`
   const uint32_t bstar = d;
 
-  // the elements that can be selected: bin >= b*
+  // the elements that can be selected: bin >= b*; those in b* also count their second
+  // digit (key bits 19..10) into this CTA's histogram when a second digit is needed
+  static_assert(kHistShift == 20, "second digit = key bits 19..10");
+  const bool second = count != r;
   uint32_t cand = 0;
 #pragma unroll
   for (int step = 0; step < KPT; ++step) {
     const int p = seg0 + 32 * step + lane;
-    if (c0 + p < V && (keys[p] >> kHistShift) >= bstar) cand |= 1u << step;
+    if (c0 + p < V) {
+      const uint32_t key = keys[p];
+      if ((key >> kHistShift) >= bstar) cand |= 1u << step;
+      if (second && (key >> kHistShift) == bstar) atomicAdd(&sm.hl[(key >> 10) & 1023u], 1u);
+    }
   }
 
   // later digits, until every element of the bin is needed: then the threshold is the
@@ -234,12 +244,14 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
     const int bins = 1 << width;
     const int bpc = bins / C;
     uint32_t* fb = sm.fullb[level % 3];
-    for (int b = threadIdx.x; b < bins; b += kCT) sm.hl[b] = 0u;
-    __syncthreads();
-    for (uint32_t m = cand; m; m &= m - 1) {
-      const int p = seg0 + 32 * (__ffs(m) - 1) + lane;
-      const unsigned long long c = comp(p);
-      if ((c >> pos) == (prefix >> pos)) atomicAdd(&sm.hl[(uint32_t)(c >> shift) & (uint32_t)(bins - 1)], 1u);
+    if (level > 1) {  // the second digit was counted in the candidate pass
+      for (int b = threadIdx.x; b < bins; b += kCT) sm.hl[b] = 0u;
+      __syncthreads();
+      for (uint32_t m = cand; m; m &= m - 1) {
+        const int p = seg0 + 32 * (__ffs(m) - 1) + lane;
+        const unsigned long long c = comp(p);
+        if ((c >> pos) == (prefix >> pos)) atomicAdd(&sm.hl[(uint32_t)(c >> shift) & (uint32_t)(bins - 1)], 1u);
+      }
     }
     __syncthreads();
     wait_s0();
