@@ -58,6 +58,7 @@ struct TcCfg {
   static constexpr int kNumBars = 2 * kStages + 4 + 3;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffTmem + 16 + 1024;  // + alignment slack
+  static_assert(kSmem <= 232448, "shared memory budget");
 };
 
 struct Items {
