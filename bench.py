@@ -163,11 +163,45 @@ def job_throughput(units_per_rank: int, world: int, max_ms: float) -> float:
     return units_per_rank * world / (max_ms * 1e-3)
 
 
+def _packed(specs, device):
+    """One device byte buffer holding tensors of the given (shape, dtype) at 256-byte
+    aligned offsets, and the tensors as views of it: a step's query-side inputs (and its
+    outputs) then cross PCIe in one copy each."""
+    import torch
+    offs, total = [], 0
+    for shape, dt in specs:
+        offs.append(total)
+        n = torch.tensor([], dtype=dt).element_size()
+        for d in shape:
+            n *= d
+        total = (total + n + 255) & ~255
+    buf = torch.empty(total, dtype=torch.uint8, device=device)
+    views = []
+    for (shape, dt), o in zip(specs, offs):
+        n = torch.tensor([], dtype=dt).element_size()
+        for d in shape:
+            n *= d
+        views.append(buf[o:o + n].view(dt).view(shape))
+    return buf, views
+
+
 def make_inputs(w, device, rank):
+    """Seeded synthetic inputs of every group.  The caches live in their own tensors; the
+    per-step query-side inputs of all groups (indexer queries, head weights, attention
+    queries, MTP draft queries) share one buffer, and so do the outputs (index lists and
+    attention outputs) -- groups[0]["in_buf"] / ["out_buf"]."""
     import torch
     import synth
     import synth.device as sd
     bf = torch.bfloat16
+    f32 = torch.float32
+    ins, outs_spec = [], []
+    for g in range(w.groups):
+        ins += [((w.B, w.T, 32, 128), bf), ((w.B, w.T, 32), f32)]
+        ins += [((w.B, w.T, w.H, 576), bf)] * (w.L + max(0, w.steps - 1))
+        outs_spec += [((w.B, w.T, w.k), torch.int32)] + [((w.B, w.T, w.H, 512), f32)] * w.L
+    in_buf, in_views = _packed(ins, device)
+    out_buf, out_views = _packed(outs_spec, device)
     groups = []
     for g in range(w.groups):
         ik = torch.empty(w.B, w.N, 128, dtype=bf, device=device)
@@ -177,23 +211,23 @@ def make_inputs(w, device, rank):
             kv = torch.empty(w.B, w.N, 576, dtype=bf, device=device)
             sd.normal_bf16(kv, rank_key(w.key(synth.KIND_KV, g, l), rank))
             kvs.append(kv)
-        iq = torch.empty(w.B, w.T, 32, 128, dtype=bf, device=device)
+        iq, wt = in_views.pop(0), in_views.pop(0)
         sd.int17_bf16(iq, rank_key(w.key(synth.KIND_IQ, g), rank))
-        wt = torch.empty(w.B, w.T, 32, dtype=torch.float32, device=device)
         sd.pow2_f32(wt, rank_key(w.key(synth.KIND_W, g), rank))
         qs = []
         for l in range(w.L):
-            q = torch.empty(w.B, w.T, w.H, 576, dtype=bf, device=device)
+            q = in_views.pop(0)
             sd.normal_bf16(q, rank_key(w.key(synth.KIND_Q, g, l), rank))
             qs.append(q)
-        idx = torch.empty(w.B, w.T, w.k, dtype=torch.int32, device=device)
-        outs = [torch.empty(w.B, w.T, w.H, 512, dtype=torch.float32, device=device) for _ in range(w.L)]
         draft_qs = []
         for st in range(1, w.steps):
-            qd = torch.empty(w.B, w.T, w.H, 576, dtype=bf, device=device)
+            qd = in_views.pop(0)
             sd.normal_bf16(qd, rank_key(w.key(synth.KIND_Q, g, 0, st), rank))
             draft_qs.append(qd)
+        idx = out_views.pop(0)
+        outs = [out_views.pop(0) for _ in range(w.L)]
         groups.append(dict(ik=ik, kvs=kvs, iq=iq, wt=wt, qs=qs, idx=idx, outs=outs, draft_qs=draft_qs))
+    groups[0]["in_buf"], groups[0]["out_buf"] = in_buf, out_buf
     return groups
 
 
@@ -284,21 +318,19 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         return w, step_ms, idx_ms, None, 0, 0, clk.summary()
 
     # end to end through the public API with host buffers: per step, the step's query-side
-    # inputs go host -> device from pinned memory and the outputs come back
-    pinned_in = [[t.cpu().pin_memory() for t in [g["iq"], g["wt"], *g["qs"], *g["draft_qs"]]] for g in groups]
-    pinned_out = [[torch.empty_like(t, device="cpu").pin_memory() for t in [g["idx"], *g["outs"]]] for g in groups]
+    # inputs (one packed buffer) go host -> device from pinned memory and the outputs (index
+    # lists and attention outputs, one packed buffer) come back
+    in_buf, out_buf = groups[0]["in_buf"], groups[0]["out_buf"]
+    pinned_in = in_buf.cpu().pin_memory()
+    pinned_out = torch.empty_like(out_buf, device="cpu").pin_memory()
 
     def e2e_step():
-        for g, pin, pout in zip(groups, pinned_in, pinned_out):
-            for dst, src in zip([g["iq"], g["wt"], *g["qs"], *g["draft_qs"]], pin):
-                dst.copy_(src, non_blocking=True)
+        in_buf.copy_(pinned_in, non_blocking=True)
         graph.replay()
-        for g, pout in zip(groups, pinned_out):
-            for dst, src in zip(pout, [g["idx"], *g["outs"]]):
-                dst.copy_(src, non_blocking=True)
+        pinned_out.copy_(out_buf, non_blocking=True)
 
-    h2d = sum(t.numel() * t.element_size() for pin in pinned_in for t in pin)
-    d2h = sum(t.numel() * t.element_size() for pout in pinned_out for t in pout)
+    h2d = in_buf.numel()
+    d2h = out_buf.numel()
     e2e_times = timed(e2e_step, args.steps, args.warmup)
     e2e_ms = sum(e2e_times) / len(e2e_times)
 

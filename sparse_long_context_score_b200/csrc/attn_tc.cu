@@ -625,7 +625,7 @@ int attn_num_splits(long long rows, int L, int k, const int* fit) {
   int best = 1;
   for (int ns = 1; ns <= kMaxSplits && ns <= max_ns; ++ns) {
     if (units * ns > kNumSMs) break;
-    if (fit && fit[ns] > 0 && units > fit[ns]) continue;
+    if (fit && ns > 1 && units > fit[ns]) continue;  // (a size that cannot run at all reports 0)
     best = ns;
   }
   const int chunk = attn_split_chunk(k, best);
