@@ -17,22 +17,26 @@
 // Warp roles (416 threads):
 //   warps 0..7  gather: the selected rows as 16-byte cp.async chunks written straight into
 //               the 128-byte-swizzled tensor-core layout; warps 2s, 2s+1 own stage s
-//               (16 rows each) and tiles s, s+4, ..., wait for their own copies, fence
-//               them to the async proxy and arrive on the stage barrier, so four tiles are
-//               in flight and each is published as soon as it lands (one TMA load brings
-//               the 64 query rows).  Issue parallelism matters: a random-row gather probe
-//               reached ~3.1 TB/s with 4 warps and ~3.9 TB/s with 6 on 128 SMs.  Random 1152-byte rows are too small for TMA: a
-//               4-row gather copy per 512 bytes ran latency-bound on B200.
-//   warp 8      TMEM allocation; one elected lane issues S(i) and then O += P(i-1) V(i-1),
-//               so the softmax of one tile overlaps the next tile's logits;
+//               (16 rows each) and tiles s, s+4, ... (their row indices loaded into
+//               registers up front), wait for their own copies, fence them to the async
+//               proxy and arrive on the stage barrier, so four tiles are in flight and each
+//               is published as soon as it lands (one TMA load brings the 64 query rows).
+//               Random 1152-byte rows are too small for TMA: measured on B200 with the same
+//               bytes in flight, a 128-byte box per row reached 0.57 TB/s, 4-row gather
+//               boxes 1.6 TB/s, one bulk copy per row 2.8 TB/s, 16-byte cp.async 4.9 TB/s.
+//   warp 8      TMEM allocation; one elected lane issues S(i) once tile i has landed and
+//               O += P(j) V(j) once P(j) is published, whichever is ready (PV first), so
+//               the softmax of one tile overlaps the next tile's logits and a stage is
+//               released as soon as its PV completes;
 //   warps 9..12 softmax (threads on lanes 0..15 of each warp own a head), P as bf16 in
 //               shared memory.
 // The key splits of one (row, layer) run as one thread-block cluster and are reduced on
-// chip: each split scales its O^T by its share of the normaliser, stages it in its shared
-// memory, and sums one slice of the [H][512] output over the cluster's shared memories.
+// chip: each split stages its unnormalised O in its shared memory, and split r sums slice r
+// of the [H][512] output over the cluster's shared memories with the normaliser shares.
 // (A global-memory merge by the last split to finish -- 16 MB of partials written and
 // read back at the end of the 32-unit decode batch -- made the kernel's tail longer than
-// its whole main loop.)
+// its whole main loop.)  The launch waits for the preceding kernel (programmatic dependent
+// launch) only where it reads that kernel's results.
 // All mbarrier waits are bounded (sm100.cuh).
 #include <cudaTypedefs.h>
 

@@ -10,6 +10,9 @@
 // which is distinct per element and orders exactly as required, so the selection is
 // "the k largest composites" and the answer is unique: bit-exact and deterministic.
 //
+// launch_topk sends rows that one cluster of CTAs can hold on chip (decode shapes) to
+// topk_cluster.cu; the kernels here take many rows or long rows.
+//
 // Radix select over C, most significant digit first:
 //   1. histogram of the top 12 bits (4096 bins) per row -- built here, or folded into
 //      the indexer epilogue;
