@@ -1,0 +1,37 @@
+"""Host-side helpers of bench.py, on CPU: the packed per-step buffers and the launch count
+the benchmark line claims."""
+import sys
+
+import pytest
+import torch
+
+sys.argv = sys.argv[:1]
+import bench  # noqa: E402
+from synth import configs as C  # noqa: E402
+
+
+def test_packed_views_are_aligned_disjoint_and_typed():
+    specs = [((3, 5, 7), torch.bfloat16), ((2, 9), torch.float32), ((4, 1, 11), torch.int32), ((1,), torch.bfloat16)]
+    buf, views = bench._packed(specs, "cpu")
+    spans = []
+    for (shape, dt), v in zip(specs, views):
+        assert tuple(v.shape) == shape and v.dtype == dt and v.is_contiguous()
+        off = v.data_ptr() - buf.data_ptr()
+        assert off % 256 == 0
+        spans.append((off, off + v.numel() * v.element_size()))
+    spans.sort()
+    assert all(a[1] <= b[0] for a, b in zip(spans, spans[1:]))
+    assert spans[-1][1] <= buf.numel()
+    # writing through one view changes only its own bytes
+    buf.zero_()
+    views[1].fill_(1.5)
+    assert float(views[1].sum()) == 1.5 * 18
+    assert float(views[0].float().abs().sum()) == 0.0 and int(views[2].abs().sum()) == 0
+    assert float(views[3].float().abs().sum()) == 0.0
+
+
+@pytest.mark.parametrize("name,expected", [("decode128k", 3), ("mtp", 3), ("tiny", 3), ("decode1m", 4), ("prefill", 5)])
+def test_launches_per_group(name, expected):
+    # indexer + top-k (one cluster kernel for decode-shaped rows; select + compact, plus a
+    # histogram kernel when the indexer does not count the first digit) + one attention launch
+    assert bench.launches_per_group(C.WORKLOADS[name]) == expected
