@@ -223,7 +223,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   uint64_t* cand = ws.cand + (size_t)row * kCandCap;
   constexpr int kPerThread = kTopkChunk / kSelThreads;  // 16
   uint32_t keys[kPerThread];
-  uint32_t cand_bits = 0, n_above = 0;
+  uint32_t cand_bits = 0, inb_bits = 0, n_above = 0;
   auto elem = [&](int i) -> long long {
     // element i of this thread: four consecutive scores per 16-byte group
     return s0 + 4LL * (threadIdx.x + kSelThreads * (i >> 2)) + (i & 3);
@@ -256,11 +256,13 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
     const bool in = elem(i) < s1;
     const uint32_t bin = keys[i] >> kHistShift;
     n_above += (in && bin > bstar) ? 1u : 0u;
-    cand_bits |= (in && use_cand && bin == bstar) ? (1u << i) : 0u;
+    inb_bits |= (in && bin == bstar) ? (1u << i) : 0u;
   }
+  if (use_cand) cand_bits = inb_bits;
+  // the second digit of every element of b* is counted, whether or not the candidates fit
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i)
-    if (cand_bits & (1u << i)) atomicAdd(&sm.hist2[(keys[i] >> 10) & (kHist2Bins - 1)], 1u);
+    if (inb_bits & (1u << i)) atomicAdd(&sm.hist2[(keys[i] >> 10) & (kHist2Bins - 1)], 1u);
   const uint32_t my_off = block_excl_scan((uint32_t)__popc(cand_bits), sm.warp_tmp, &sm.total);
   if (threadIdx.x == 0) sm.cand_base = sm.total ? atomicAdd(&state[RS_CAND], sm.total) : 0u;
   __syncthreads();
@@ -275,7 +277,7 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   }
   (void)block_excl_scan(n_above, sm.warp_tmp, &sm.total);
   if (threadIdx.x == 0) ws.chunk_above[(size_t)row * nchunks + chunk] = sm.total;
-  if (use_cand) {
+  {
     uint32_t* g2 = ws.hist2 + (size_t)row * kHist2Bins;
     for (int i = threadIdx.x; i < kHist2Bins; i += kSelThreads)
       if (sm.hist2[i]) atomicAdd(&g2[i], sm.hist2[i]);
@@ -301,13 +303,15 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
   }
   uint64_t thr = 0;
   bool resolved = false;
-  if (use_cand) {
-    // 4a. second digit from the row's second-level histogram; the elements of the final
-    //     sub-bin (usually a handful) are ranked directly
-    const uint32_t* g2 = ws.hist2 + (size_t)row * kHist2Bins;
-    find_digit(sm, kHist2Bins, remaining, [&](int bin) { return __ldcg(&g2[bin]); });
-    const uint32_t d2 = sm.digit, r2 = remaining - sm.digit_above, n2 = sm.digit_count;
-    if (n2 <= (uint32_t)kFinalCap) {
+  // 4. second digit from the row's second-level histogram (complete: every CTA counted all
+  //    its elements of b*); the elements of the final sub-bin (usually a handful) are
+  //    collected -- from the candidate list, or when that overflowed in one pass over the
+  //    row -- and ranked directly
+  const uint32_t* g2 = ws.hist2 + (size_t)row * kHist2Bins;
+  find_digit(sm, kHist2Bins, remaining, [&](int bin) { return __ldcg(&g2[bin]); });
+  const uint32_t d2 = sm.digit, r2 = remaining - sm.digit_above, n2 = sm.digit_count;
+  if (n2 <= (uint32_t)kFinalCap) {
+    if (use_cand) {
       for (long long i = threadIdx.x; i < bcount; i += kSelThreads) {
         const uint64_t c = __ldcg(&cand[i]);
         const uint32_t dg = (uint32_t)(c >> 42) & (kHist2Bins - 1);
@@ -317,37 +321,48 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
           if (pos < (uint32_t)kFinalCap) sm.fin[pos] = c;
         }
       }
-      __syncthreads();
-      const uint32_t nf = min(sm.nfin, (uint32_t)kFinalCap);  // == n2
-      for (uint32_t i = threadIdx.x; i < nf; i += kSelThreads) {
-        const uint64_t c = sm.fin[i];
-        uint32_t rank = 0;
-        for (uint32_t j = 0; j < nf; ++j) rank += sm.fin[j] > c ? 1u : 0u;
-        if (rank == r2 - 1) sm.thr = c;  // composites are distinct: exactly one thread writes
-      }
-      __syncthreads();
-      thr = sm.thr;
-      for (uint32_t i = threadIdx.x; i < nf; i += kSelThreads) {
-        const uint64_t c = sm.fin[i];
-        if (c >= thr) atomicAdd(&cnt[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
-      }
-      resolved = true;
     } else {
-      // many equal high bits: radix passes over the candidate list
-      const uint64_t thr52 = resolve_threshold(sm, bcount, remaining, [&](long long i, uint64_t& c) {
-        c = __ldcg(&cand[i]);
-        return true;
-      });
-      thr = ((uint64_t)bstar << 52) | thr52;
-      for (long long i = threadIdx.x; i < bcount; i += kSelThreads) {
-        const uint64_t c = __ldcg(&cand[i]);
-        if (c >= thr) atomicAdd(&cnt[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+      for (long long s2 = threadIdx.x; s2 < V; s2 += kSelThreads) {
+        const uint32_t key = order_key(__ldcg(&sr[s2]));
+        if ((key >> kHistShift) != bstar) continue;
+        const uint32_t dg = (key >> 10) & (kHist2Bins - 1);
+        if (dg > d2) atomicAdd(&cnt[s2 / kTopkChunk], 1u);
+        else if (dg == d2) {
+          const uint32_t pos = atomicAdd(&sm.nfin, 1u);
+          if (pos < (uint32_t)kFinalCap) sm.fin[pos] = composite(key, (uint32_t)s2);
+        }
       }
-      resolved = true;
     }
+    __syncthreads();
+    const uint32_t nf = min(sm.nfin, (uint32_t)kFinalCap);  // == n2
+    for (uint32_t i = threadIdx.x; i < nf; i += kSelThreads) {
+      const uint64_t c = sm.fin[i];
+      uint32_t rank = 0;
+      for (uint32_t j = 0; j < nf; ++j) rank += sm.fin[j] > c ? 1u : 0u;
+      if (rank == r2 - 1) sm.thr = c;  // composites are distinct: exactly one thread writes
+    }
+    __syncthreads();
+    thr = sm.thr;
+    for (uint32_t i = threadIdx.x; i < nf; i += kSelThreads) {
+      const uint64_t c = sm.fin[i];
+      if (c >= thr) atomicAdd(&cnt[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+    }
+    resolved = true;
+  } else if (use_cand) {
+    // many equal high bits: radix passes over the candidate list
+    const uint64_t thr52 = resolve_threshold(sm, bcount, remaining, [&](long long i, uint64_t& c) {
+      c = __ldcg(&cand[i]);
+      return true;
+    });
+    thr = ((uint64_t)bstar << 52) | thr52;
+    for (long long i = threadIdx.x; i < bcount; i += kSelThreads) {
+      const uint64_t c = __ldcg(&cand[i]);
+      if (c >= thr) atomicAdd(&cnt[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+    }
+    resolved = true;
   }
   if (!resolved) {
-    // the threshold bin overflowed the candidate list: radix passes over the row itself
+    // the final sub-bin is large and the candidates overflowed: radix passes over the row
     const uint64_t thr52 = resolve_threshold(sm, V, remaining, [&](long long s2, uint64_t& c) {
       const uint32_t key = order_key(__ldcg(&sr[s2]));
       if ((key >> kHistShift) != bstar) return false;
