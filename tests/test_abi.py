@@ -96,3 +96,11 @@ def test_binding_refuses_cpu_tensors():
     with pytest.raises((ValueError, ImportError)):
         dsa.dsa_index_score(torch.zeros(1, 1, 32, 128, dtype=torch.bfloat16), torch.zeros(1, 1, 32),
                             torch.zeros(1, 8, 128, dtype=torch.bfloat16), 7, scores=torch.zeros(1, 1, 8))
+
+
+def test_last_cuda_error_starts_clear_and_names_codes(L):
+    # argument errors are returned before any CUDA call, so they never set it
+    assert L.dsa_topk(None, 1, 1, 16, 15, 4, FAKE, FAKE, 1 << 30, None) == -1
+    assert L.dsa_last_cuda_error() == 0
+    assert L.dsa_cuda_error_string(0) == b"no error"
+    assert L.dsa_cuda_error_string(1)  # cudaErrorInvalidValue has a description
