@@ -26,9 +26,10 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-INDEXER_BYTES_PER_TOKEN = 128 * 2 + 4          # index key read + score write
+INDEXER_BYTES_PER_KEY = 128 * 2                  # one index key read per visible token
 INDEXER_BYTES_PER_QUERY = 32 * 128 * 2 + 32 * 4  # indexer query + head weights
-ROW_BYTES = 576 * 2                             # one gathered compressed row
+SCORE_BYTES_PER_KEY = 4                          # score write: reported, not algorithmic
+ROW_BYTES = 576 * 2                              # one gathered compressed row
 
 
 def parse():
@@ -48,13 +49,16 @@ def parse():
 
 
 def algorithmic(w):
-    """Algorithmic HBM bytes of one step, and of one indexer launch.  The indexer reads the
-    visible index keys once per query group and writes one score per visible key; the
-    attention gathers k rows per (query, layer, draft step) and writes the outputs."""
+    """Algorithmic HBM bytes of one step and of one indexer launch: the indexer reads the
+    visible index keys of each sequence once, plus its queries and head weights; the
+    attention gathers k compressed rows per (query, layer, draft step) and reads the
+    queries and writes the outputs; the index list is written once.  The score write
+    (4 B per visible key, L2-resident) is not algorithmic: it is returned separately."""
     vis = min(w.N, w.q_pos0 + w.T)
-    idx_launch = w.B * w.T * INDEXER_BYTES_PER_QUERY + w.B * w.T * vis * 4 + w.B * vis * 128 * 2
+    idx_launch = w.B * w.T * INDEXER_BYTES_PER_QUERY + w.B * vis * INDEXER_BYTES_PER_KEY
     attn = w.B * w.T * w.L * w.steps * (w.k * ROW_BYTES + w.H * 576 * 2 + w.H * 512 * 4)
-    return w.groups * (idx_launch + attn + w.B * w.T * w.k * 4), idx_launch
+    scores = w.B * w.T * vis * SCORE_BYTES_PER_KEY
+    return w.groups * (idx_launch + attn + w.B * w.T * w.k * 4), idx_launch, scores
 
 
 def prefill_indexer_flops(w):
@@ -232,6 +236,9 @@ def make_inputs(w, device, rank):
 
 
 def run_ours(args, rank, world, device, w=None, e2e=True):
+    """Times the workload's step on this rank's GPU.  Returns a dict: the step time (graph
+    replay, inputs resident in HBM), the indexer launch time, the end-to-end times (eager
+    and graph) with their host<->device bytes, and the clock record."""
     import torch
     import sparse_long_context_score_b200 as dsa
     from synth import configs as C
@@ -270,7 +277,10 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         step()
     torch.cuda.synchronize()
 
-    def timed(fn, K, W):
+    def timed(fn, K, W, host_in_region=False):
+        """K timed runs of fn after W warm-up runs, L2 flushed before each; CUDA events on
+        the launching stream.  With host_in_region the device is idle when the start event
+        is recorded, so the host's enqueue work of fn is inside the measured interval."""
         with torch.cuda.stream(stream):
             for _ in range(W):
                 flush_l2()
@@ -280,6 +290,8 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         with torch.cuda.stream(stream):
             for a, b in ev:
                 flush_l2()
+                if host_in_region:
+                    torch.cuda.synchronize()
                 a.record(stream)
                 fn()
                 b.record(stream)
@@ -294,7 +306,7 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    step_ms = sum(times) / len(times)
+    res = {"step_ms": sum(times) / len(times), "clocks": clk.summary()}
 
     # the dominant kernel alone: the indexer over the first group's cache, same launch shape
     g0 = groups[0]
@@ -309,70 +321,117 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         dsa.dsa_index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores, stream=stream)
     torch.cuda.synchronize()
     idx_times = timed(igraph.replay, args.steps, args.warmup)
-    idx_ms = sum(idx_times) / len(idx_times)
+    res["idx_ms"] = sum(idx_times) / len(idx_times)
+    status = dsa.dsa_check_device_status(stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed runs")
 
-    if not e2e:
-        step_ms, idx_ms = max_over_ranks([step_ms, idx_ms], world, device)
-        del groups, ws, flush, flush_rd, scores, graph, igraph
-        torch.cuda.empty_cache()
-        return w, step_ms, idx_ms, None, 0, 0, clk.summary()
+    if e2e:
+        # end to end through the public API with host buffers: per step, the step's
+        # query-side inputs (one packed buffer) go host -> device from pinned memory, the
+        # library calls run, and the outputs (index lists and attention outputs, one packed
+        # buffer) come back.  "eager" calls the C ABI per step (its host-side work included);
+        # "graph" replays the captured step between the two copies.
+        in_buf, out_buf = groups[0]["in_buf"], groups[0]["out_buf"]
+        pinned_in = in_buf.cpu().pin_memory()
+        pinned_out = torch.empty_like(out_buf, device="cpu").pin_memory()
 
-    # end to end through the public API with host buffers: per step, the step's query-side
-    # inputs (one packed buffer) go host -> device from pinned memory and the outputs (index
-    # lists and attention outputs, one packed buffer) come back
-    in_buf, out_buf = groups[0]["in_buf"], groups[0]["out_buf"]
-    pinned_in = in_buf.cpu().pin_memory()
-    pinned_out = torch.empty_like(out_buf, device="cpu").pin_memory()
+        def e2e_eager():
+            in_buf.copy_(pinned_in, non_blocking=True)
+            step()
+            pinned_out.copy_(out_buf, non_blocking=True)
 
-    def e2e_step():
-        in_buf.copy_(pinned_in, non_blocking=True)
-        graph.replay()
-        pinned_out.copy_(out_buf, non_blocking=True)
+        def e2e_graph():
+            in_buf.copy_(pinned_in, non_blocking=True)
+            graph.replay()
+            pinned_out.copy_(out_buf, non_blocking=True)
 
-    h2d = in_buf.numel()
-    d2h = out_buf.numel()
-    e2e_times = timed(e2e_step, args.steps, args.warmup)
-    e2e_ms = sum(e2e_times) / len(e2e_times)
+        eager = timed(e2e_eager, args.steps, args.warmup, host_in_region=True)
+        gr = timed(e2e_graph, args.steps, args.warmup, host_in_region=True)
+        res.update(e2e_ms=sum(eager) / len(eager), e2e_graph_ms=sum(gr) / len(gr), h2d=in_buf.numel(),
+                   d2h=out_buf.numel())
+        keys = ["step_ms", "idx_ms", "e2e_ms", "e2e_graph_ms"]
+    else:
+        keys = ["step_ms", "idx_ms"]
+    for k, v in zip(keys, max_over_ranks([res[k] for k in keys], world, device)):
+        res[k] = v
+    del groups, ws, flush, flush_rd, scores, graph, igraph
+    torch.cuda.empty_cache()
+    return w, res
 
-    step_ms, e2e_ms, idx_ms = max_over_ranks([step_ms, e2e_ms, idx_ms], world, device)
-    return w, step_ms, idx_ms, e2e_ms, h2d, d2h, clk.summary()
+
+def host_cpu() -> dict:
+    """The host CPU the oracle runs on: model name and logical core count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    import platform
+    return {"model": model or platform.processor() or "unknown", "logical_cores": os.cpu_count()}
 
 
-def cpu_baseline(w, n_seq):
-    """The oracle as it stands, on n_seq sequences of the workload (one IndexShare group,
-    all its layers), timed on this host; returns tokens/s and a description."""
+def oracle_sequence(w, b, o):
+    """The oracle over sequence b of the workload: for every IndexShare group the indexer
+    over its N keys, the top-k, and the attention of its L layers (and of every MTP draft
+    step, on the step-1 index list).  The inputs of each call are generated before it;
+    returns the seconds spent inside the oracle calls."""
     import numpy as np
-    import oracle
     import synth
     from synth import configs as C
-    o = oracle.default()
-    n_seq = max(1, min(n_seq, w.B))
     elapsed = 0.0
-    for b in range(n_seq):
-        iq = synth.int17_bf16(w.key(synth.KIND_IQ), (w.B, w.T, 32, 128))[b:b + 1]
-        wt = synth.pow2_f32(w.key(synth.KIND_W), (w.B, w.T, 32))[b:b + 1]
-        ik = synth.int17_bf16(w.key(synth.KIND_IK), index=synth.rows_index(
+    for g in range(w.groups):
+        iq = synth.int17_bf16(w.key(synth.KIND_IQ, g), (w.B, w.T, 32, 128))[b:b + 1]
+        wt = synth.pow2_f32(w.key(synth.KIND_W, g), (w.B, w.T, 32))[b:b + 1]
+        ik = synth.int17_bf16(w.key(synth.KIND_IK, g), index=synth.rows_index(
             np.arange(b * w.N, (b + 1) * w.N), 128)).reshape(1, w.N, 128)
         t0 = time.perf_counter()
         sc = o.index_score(iq, wt, ik, w.q_pos0).astype(np.float32)
         idx = o.topk(sc, w.q_pos0, w.k)
         elapsed += time.perf_counter() - t0
-        rows = idx[0, 0]
-        for l in range(w.L):
-            q = synth.normal_bf16(w.key(synth.KIND_Q, 0, l), (w.B, w.T, w.H, 576))[b:b + 1]
-            kv = synth.normal_bf16(w.key(synth.KIND_KV, 0, l), index=synth.rows_index(
-                b * w.N + rows.astype(np.uint64), 576)).reshape(1, w.k, 576)
-            local = np.arange(w.k, dtype=np.int32).reshape(1, 1, w.k)
-            t0 = time.perf_counter()
-            o.sparse_attn(q, kv, local, C.SCALE)
-            elapsed += time.perf_counter() - t0
-    tokens = n_seq * w.T * w.groups
-    per_group_s = elapsed / n_seq
-    value = 1.0 / (per_group_s * w.groups) * w.T
-    return {"value": value, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{n_seq} of {w.B} sequences, one IndexShare group (indexer over {w.N} keys, top-{w.k}, "
-                      f"{w.L} attention layers), scaled to {w.groups} group(s) per token; inputs generated "
-                      f"outside the timed region; {tokens} token-groups timed in {elapsed:.1f} s"}
+        for t in range(w.T):
+            rows = idx[0, t][idx[0, t] >= 0]
+            local = np.full((1, 1, w.k), -1, np.int32)
+            local[0, 0, :len(rows)] = np.arange(len(rows))
+            for l in range(w.L):
+                kv = synth.normal_bf16(w.key(synth.KIND_KV, g, l), index=synth.rows_index(
+                    b * w.N + rows.astype(np.uint64), 576)).reshape(1, len(rows), 576)
+                for st in range(w.steps):
+                    q = synth.normal_bf16(w.key(synth.KIND_Q, g, l, st), index=synth.rows_index(
+                        np.array([b * w.T + t]), w.H * 576)).reshape(1, 1, w.H, 576)
+                    t0 = time.perf_counter()
+                    o.sparse_attn(q, kv, local, C.SCALE)
+                    elapsed += time.perf_counter() - t0
+    return elapsed
+
+
+def cpu_baseline(w, n_seq):
+    """The oracle as it stands on n_seq whole sequences of the workload (every group,
+    layer and draft step), timed on this host with one thread; tokens/s."""
+    import oracle
+    o = oracle.default()
+    n_seq = max(1, min(n_seq, w.B))
+    elapsed = sum(oracle_sequence(w, b, o) for b in range(n_seq))
+    tokens = n_seq * w.T * w.steps
+    cpu = host_cpu()
+    return {"value": tokens / elapsed, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "host_cpu": cpu["model"], "host_logical_cores": cpu["logical_cores"],
+            "sample": f"{n_seq} of {w.B} sequences of {w.name}, whole (all {w.groups} IndexShare group(s): "
+                      f"indexer over {w.N} keys, top-{w.k}, {w.L} attention layer(s) x {w.steps} step(s)); "
+                      f"single-threaded C oracle in double precision; inputs generated outside the timed "
+                      f"region; {tokens} token(s) in {elapsed:.1f} s"}
+
+
+def workload_config(w, world: int) -> dict:
+    """The `config` object of the bench line: the workload and how it is run (the same in
+    both arms)."""
+    return {"workload": w.name, "B": w.B, "T": w.T, "N": w.N, "k": w.k, "H": w.H, "L": w.L, "groups": w.groups,
+            "draft_steps": w.steps, "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            "l2": "flushed before every timed step (512 MiB write, then a 512 MiB read so the write-back is not timed)"}
 
 
 def launches_per_group(w) -> int:
@@ -451,21 +510,26 @@ def main():
     metric = "DSA group decode tokens/s"
     if args.impl == "reference":
         if rank == 0:
-            K = args.steps
-            vals = []
-            cb = None
-            for _ in range(args.warmup + K):
-                cb = cpu_baseline(w, 1)
-                vals.append(cb["value"])
-            v = sum(vals[args.warmup:]) / max(1, K)
-            cb["value"] = v
+            import oracle
+            o = oracle.default()
+            times = []
+            for step in range(args.warmup + args.steps):
+                dt = oracle_sequence(w, step % w.B, o)
+                if step >= args.warmup:
+                    times.append(dt)
+            step_s = sum(times) / len(times)
+            v = w.T * w.steps / step_s
+            cpu = host_cpu()
             print(json.dumps({"impl": "reference", "metric": metric, "value": v, "unit": "tokens/s",
-                              "n_gpus": args.gpus, "steps": K, "warmup": args.warmup,
-                              "ms_per_step": 1e3 / v * w.B, "higher_is_better": True, "scaling": "weak",
+                              "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                              "ms_per_step": step_s * 1e3, "higher_is_better": True, "scaling": "weak",
                               "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                              "config": {"workload": w.name, "B": w.B, "N": w.N, "k": w.k, "H": w.H, "L": w.L,
-                                         "groups": w.groups},
-                              "cpu_baseline": cb,
+                              "config": workload_config(w, args.gpus),
+                              "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                                               "host_cpu": cpu["model"], "host_logical_cores": cpu["logical_cores"],
+                                               "sample": f"each step is one whole sequence of {w.name} (sequence "
+                                                         f"step mod {w.B}), the single-threaded C oracle in double "
+                                                         f"precision; inputs generated outside the timed region"},
                               "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                                       "d2h_bytes_per_step": 0}}))
         return
@@ -476,48 +540,46 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
-    w, step_ms, idx_ms, e2e_ms, h2d, d2h, clocks = run_ours(args, rank, world, device)
-    step_bytes, idx_bytes = algorithmic(w)
-    tokens = w.B * w.T * world
-    value = job_throughput(w.B * w.T, world, step_ms)
+    w, r = run_ours(args, rank, world, device)
+    step_bytes, idx_bytes, score_bytes = algorithmic(w)
+    tokens = w.B * w.T * w.steps * world
+    value = job_throughput(w.B * w.T * w.steps, world, r["step_ms"])
     peak, peak_kind = peaks()
-    achieved = idx_bytes / (idx_ms * 1e-3) / 1e9
+    achieved = idx_bytes / (r["idx_ms"] * 1e-3) / 1e9
+    step_gbs = step_bytes / (r["step_ms"] * 1e-3) / 1e9
     line = {
         "metric": metric, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": r["step_ms"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "T": w.T, "N": w.N, "k": w.k, "H": w.H, "L": w.L,
-                   "groups": w.groups, "l2": "flushed before every timed step (512 MiB write, then a 512 MiB read so the write-back is not timed)",
-                   "parallelism": f"dp{world}" if world > 1 else "single GPU",
-                   "step_hbm_gbs": step_bytes / (step_ms * 1e-3) / 1e9,
-                   "step_roofline_frac": step_bytes / (step_ms * 1e-3) / 1e9 / peak},
-        "clocks": clocks,
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
+        "config": workload_config(w, world),
+        "clocks": r["clocks"],
+        "e2e": {"value": tokens / (r["e2e_ms"] * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
+                "d2h_bytes_per_step": r["d2h"], "calls": "eager: the C ABI called per step",
+                "graph_replay_value": tokens / (r["e2e_graph_ms"] * 1e-3)},
         "gpu_launches": launches_per_group(w) * w.groups * args.steps,
         "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": profiled_traffic("indexer_tc.cu", w.name), "launch_us": idx_ms * 1e3,
-                     "algorithmic_bytes_per_launch": idx_bytes},
+                     "traffic": profiled_traffic("indexer_tc.cu", w.name), "launch_us": r["idx_ms"] * 1e3,
+                     "algorithmic_bytes_per_launch": idx_bytes, "score_write_bytes_per_launch": score_bytes},
+        "step": {"hbm_gbs": step_gbs, "roofline_frac": step_gbs / peak, "algorithmic_bytes": step_bytes},
     }
     if not args.no_extra and args.workload == "decode128k":
         extra = {}
         for name in ("decode1m", "mtp", "prefill"):
-            we = C.WORKLOADS[name]
-            _, ms, ims, _, _, _, clk2 = run_ours(args, rank, world, device, w=we, e2e=False)
-            b2, ib2 = algorithmic(we)
-            toks = we.B * we.T * (we.steps if we.steps > 1 else 1) * world
+            we, r2 = run_ours(args, rank, world, device, w=C.WORKLOADS[name], e2e=False)
+            b2, ib2, _ = algorithmic(we)
+            ms, ims = r2["step_ms"], r2["idx_ms"]
+            toks = we.B * we.T * we.steps * world
             ent = {"tokens_per_s": toks / (ms * 1e-3), "ms_per_step": ms, "step_hbm_gbs": b2 / (ms * 1e-3) / 1e9,
                    "step_roofline_frac": b2 / (ms * 1e-3) / 1e9 / peak, "indexer_launch_us": ims * 1e3,
-                   "indexer_hbm_gbs": ib2 / (ims * 1e-3) / 1e9, "clocks_sm_mhz": clk2.get("sm_mhz"),
-                   "clock_reasons": clk2.get("reasons")}
+                   "indexer_hbm_gbs": ib2 / (ims * 1e-3) / 1e9, "clocks_sm_mhz": r2["clocks"].get("sm_mhz"),
+                   "clock_reasons": r2["clocks"].get("reasons")}
             if name == "prefill":
                 fl = prefill_indexer_flops(we)
                 ent["indexer_tflops"] = fl / (ims * 1e-3) / 1e12
-                ent["indexer_tensor_frac_of_measured_bf16"] = ent["indexer_tflops"] / _bf16_peak()
-                ent["tokens_per_s"] = we.B * we.T * world / (ms * 1e-3)
+                ent["indexer_tflops_frac_of_bf16_peak"] = ent["indexer_tflops"] / _bf16_peak()
             extra[name] = ent
-        line["config"]["other_workloads"] = extra
+        line["other_workloads"] = extra
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, args.cpu_sample)
     if rank == 0:

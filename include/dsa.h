@@ -77,11 +77,21 @@ const char *dsa_cuda_error_string(int code);
 int dsa_version(void);
 
 /*
- * Device-side error word of the tensor-core kernels.  Their pipeline waits are bounded:
- * a wait that runs out records a nonzero code and the kernel returns early (its outputs
- * are then incomplete).  Synchronises with the device, writes the code (0 = none) to
- * *code and returns DSA_ERR_TIMEOUT if it is set, DSA_OK otherwise; clear != 0 resets it.
+ * Device-side error words.  The pipeline waits of the indexer and the attention kernels
+ * are bounded: a wait that runs out records a nonzero code and the kernel returns early
+ * (its outputs are then incomplete).  The top-k records a code when a selection invariant
+ * fails (a row did not select exactly k positions), which would be a bug.
+ *
+ * dsa_check_device_status: synchronises `stream` (the work enqueued on it so far), reads
+ * the error words and resets the ones that are set.  Returns DSA_ERR_TIMEOUT if a bounded
+ * wait ran out, DSA_ERR_DEVICE if the top-k recorded a broken invariant, DSA_ERR_CUDA if
+ * the stream itself reports a CUDA error, DSA_OK otherwise.  The words are per device and
+ * shared by all streams: an error recorded by work on another stream shows here too.
+ *
+ * dsa_device_error: the same check after synchronising the whole device, also giving the
+ * first nonzero code in *code (0 = none); clear != 0 resets the words.
  */
+dsa_status dsa_check_device_status(cudaStream_t stream);
 dsa_status dsa_device_error(int *code, int clear);
 
 /*
@@ -120,20 +130,23 @@ dsa_status dsa_topk(const float *scores, int B, int T, int N, long long q_pos0, 
 
 /*
  * Top-k select that allocates nothing -- for callers that cannot allocate device memory
- * (an inference engine's plugin enqueue step, a serving loop held to a fixed memory
- * plan, code being recorded into a CUDA graph where cudaMalloc is not allowed).  The
- * pages have no counterpart of this entry point; it is the same select as dsa_topk with
- * the same bit-exact output, taking dsa_topk's arguments minus the workspace: its
- * scratch is a fixed DSA_NOALLOC_SCRATCH_BYTES array inside the library, held on every
- * GPU that loads the library until the process exits.
- *   - Sizes whose select needs more scratch than that return DSA_ERR_WORKSPACE: at most
- *     23 query rows (B*T) for N up to 1,048,576 (fewer for longer rows); use dsa_topk
- *     beyond that.
+ * when they run the select: an inference engine's plugin whose enqueue step must not
+ * allocate (the engine owns every buffer), a serving loop held to a fixed memory plan, or
+ * a latency-critical host thread that must not call cudaMalloc (it can synchronise the
+ * device).  The pages have no counterpart of this entry point; it is the same select as
+ * dsa_topk with the same bit-exact output, taking dsa_topk's arguments minus the
+ * workspace.  Its scratch is a fixed DSA_NOALLOC_SCRATCH_BYTES array inside the library,
+ * held on every GPU that loads the library until the process exits.
+ *   - Shapes whose rows each fit one thread-block cluster on chip (decode shapes: rows of
+ *     up to 262,144 visible positions, as many rows as the GPU runs clusters for at once)
+ *     use no scratch.  The other shapes take the scan kernels, whose scratch must fit the
+ *     array: at most 23 query rows (B*T) for N up to 1,048,576 (fewer for longer rows);
+ *     beyond that the call returns DSA_ERR_WORKSPACE -- use dsa_topk.
  *   - The first call on a device looks up the array's device address (a runtime call,
  *     not an allocation); make that first call before any stream capture.
  *   - All calls share the array and it keeps the last call's contents; the parts that
- *     must start at zero are cleared on `stream` by every call.  Calls that overlap on
- *     the GPU (unordered streams) race on the array and must not be issued.
+ *     must start at zero are cleared on `stream` by every call that uses them.  Calls that
+ *     overlap on the GPU (unordered streams) race on the array and must not be issued.
  *   - It calls no cudaMalloc, cudaFree or allocating library routine.
  */
 #define DSA_NOALLOC_SCRATCH_BYTES (2u << 20)

@@ -30,7 +30,7 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_topk",
            "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error",
-           "dsa_last_cuda_error", "dsa_cuda_error_string")
+           "dsa_check_device_status", "dsa_last_cuda_error", "dsa_cuda_error_string")
 
 
 class DsaError(RuntimeError):
@@ -63,6 +63,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_topk_noalloc.argtypes = [P, I, I, I, LL, I, P, P]
         L.dsa_device_error.argtypes = [ctypes.POINTER(I), I]
         L.dsa_device_error.restype = I
+        L.dsa_check_device_status.argtypes = [P]
+        L.dsa_check_device_status.restype = I
         L.dsa_last_cuda_error.argtypes = []
         L.dsa_last_cuda_error.restype = I
         L.dsa_cuda_error_string.argtypes = [I]
@@ -122,6 +124,12 @@ def dsa_device_error(clear: bool = False) -> int:
     if rc not in (DSA_OK, -5):
         raise DsaError(rc, "dsa_device_error")
     return code.value
+
+
+def dsa_check_device_status(stream=None) -> int:
+    """Synchronise `stream` and return the device-side status of the work on it (0 = OK,
+    -5 a bounded wait ran out, -6 a top-k invariant failed); resets the error words."""
+    return int(lib().dsa_check_device_status(_stream(stream)))
 
 
 def dsa_workspace_size(B: int, T: int, N: int, k: int, H: int, L: int) -> int:

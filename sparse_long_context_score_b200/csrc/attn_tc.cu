@@ -562,25 +562,7 @@ bool make_map_576(CUtensorMap* map, const void* base, long long rows, int box_ro
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-struct ErrAddr {
-  std::atomic<int*> ptr[64] = {};
-  cudaError_t get(int** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int* p = ptr[dev].load();
-    if (!p) {
-      void* v = nullptr;
-      if ((e = cudaGetSymbolAddress(&v, g_attn_tc_error)) != cudaSuccess) return e;
-      p = static_cast<int*>(v);
-      ptr[dev].store(p);
-    }
-    *out = p;
-    return cudaSuccess;
-  }
-};
-ErrAddr g_err_addr;
+SymbolAddress g_err_addr;
 
 }  // namespace
 
@@ -623,12 +605,12 @@ cudaError_t query_cluster_fit() {
 // Splits per (query row, layer): the most (<= kMaxSplits, about one CTA per SM in total)
 // whose clusters all fit on the GPU at once -- a second wave of clusters would double
 // the time.  Without the device's figures (fit == nullptr) the SM count alone decides.
-int attn_num_splits(long long rows, int L, int k, const int* fit) {
+int attn_num_splits(long long rows, int L, int k, int sm_budget, const int* fit) {
   const long long units = rows * L > 0 ? rows * L : 1;
   const long long max_ns = (k + kAttnTile - 1) / kAttnTile;
   int best = 1;
   for (int ns = 1; ns <= kMaxSplits && ns <= max_ns; ++ns) {
-    if (units * ns > kNumSMs) break;
+    if (units * ns > sm_budget) break;
     if (fit && ns > 1 && units > fit[ns]) continue;  // (a size that cannot run at all reports 0)
     best = ns;
   }
@@ -646,7 +628,7 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
   for (int l = 0; l < L; ++l)
     if (!make_map_576(&maps.q[l], layers.q[l], rows * H, 64)) return cudaErrorInvalidValue;
   int* err = nullptr;
-  cudaError_t e = g_err_addr.get(&err);
+  cudaError_t e = g_err_addr.get(g_attn_tc_error, &err);
   if (e != cudaSuccess) return e;
   static DeviceOnce once;
   if ((e = once.run([] {
@@ -656,7 +638,9 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
     return e;
   int dev = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
-  const int nsplit = attn_num_splits(rows, L, k, dev >= 0 && dev < 64 ? g_cluster_fit[dev] : nullptr);
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int nsplit = attn_num_splits(rows, L, k, sms, dev >= 0 && dev < 64 ? g_cluster_fit[dev] : nullptr);
   const int chunk = attn_split_chunk(k, nsplit);
   // the splits of one (row, layer) are one cluster along x
   cudaLaunchConfig_t cfg = {};
@@ -677,13 +661,6 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
                             q_early ? 1 : 0, err);
 }
 
-cudaError_t attn_tc_device_error(int* code, bool clear) {
-  int* p = nullptr;
-  cudaError_t e = g_err_addr.get(&p);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaMemcpy(code, p, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess) return e;
-  if (clear && *code) e = cudaMemset(p, 0, sizeof(int));
-  return e;
-}
+cudaError_t attn_error_word(int** p) { return g_err_addr.get(g_attn_tc_error, p); }
 
 }  // namespace dsa

@@ -20,6 +20,20 @@ dsa_status cuda_status(cudaError_t e) {
   g_last_cuda_error.store((int)e, std::memory_order_relaxed);
   return DSA_ERR_CUDA;
 }
+
+int device_sm_count() {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) {
+    const int c = cache[dev].load(std::memory_order_relaxed);
+    if (c > 0) return c;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 0;
+  if (dev >= 0 && dev < 64) cache[dev].store(n, std::memory_order_relaxed);
+  return n;
+}
 }  // namespace dsa
 
 namespace {
@@ -55,6 +69,34 @@ GroupLayout group_layout(int B, int T, int N, int k, int H, int L) {
 
 bool heads_supported(int H) { return H == 16 || H == 32 || H == 48 || H == 64; }
 
+// The error words of the indexer, the attention and the top-k, in that order.
+struct ErrorWords {
+  int code[3] = {0, 0, 0};
+  int first() const { return code[0] ? code[0] : code[1] ? code[1] : code[2]; }
+  // a wait that ran out (indexer, attention) is a timeout; a broken top-k invariant a
+  // device error
+  dsa_status status() const { return (code[0] || code[1]) ? DSA_ERR_TIMEOUT : code[2] ? DSA_ERR_DEVICE : DSA_OK; }
+};
+
+// Reads the error words on `stream` (the caller has synchronised whatever it wants
+// covered) and, with `clear`, resets the ones that are set.
+cudaError_t read_error_words(cudaStream_t stream, bool clear, ErrorWords* w) {
+  int* p[3] = {nullptr, nullptr, nullptr};
+  cudaError_t e;
+  if ((e = indexer_error_word(&p[0])) != cudaSuccess) return e;
+  if ((e = attn_error_word(&p[1])) != cudaSuccess) return e;
+  if ((e = topk_error_word(&p[2])) != cudaSuccess) return e;
+  for (int i = 0; i < 3; ++i)
+    if ((e = cudaMemcpyAsync(&w->code[i], p[i], sizeof(int), cudaMemcpyDeviceToHost, stream)) != cudaSuccess) return e;
+  if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) return e;
+  if (clear) {
+    for (int i = 0; i < 3; ++i)
+      if (w->code[i] && (e = cudaMemsetAsync(p[i], 0, sizeof(int), stream)) != cudaSuccess) return e;
+    if ((e = cudaStreamSynchronize(stream)) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
 
 extern "C" {
@@ -81,12 +123,20 @@ int dsa_version(void) { return 10000; }
 dsa_status dsa_device_error(int* code, int clear) {
   if (!code) return DSA_ERR_INVALID_ARG;
   *code = 0;
-  int a = 0;
-  cudaError_t e;
-  if ((e = indexer_tc_device_error(code, clear != 0)) != cudaSuccess) return cuda_status(e);
-  if ((e = attn_tc_device_error(&a, clear != 0)) != cudaSuccess) return cuda_status(e);
-  if (!*code) *code = a;
-  return *code ? DSA_ERR_TIMEOUT : DSA_OK;
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e);
+  ErrorWords w;
+  if ((e = read_error_words(0, clear != 0, &w)) != cudaSuccess) return cuda_status(e);
+  *code = w.first();
+  return w.status();
+}
+
+dsa_status dsa_check_device_status(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_status(e);
+  ErrorWords w;
+  if ((e = read_error_words(stream, true, &w)) != cudaSuccess) return cuda_status(e);
+  return w.status();
 }
 
 size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L) {
@@ -154,7 +204,9 @@ dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t*
     TopkWorkspace tws = topk_workspace(base + g.topk_off, rows, N);
     float* scores = reinterpret_cast<float*>(base + g.scores_off);
     // in decode the indexer folds the first radix digit of the select into its epilogue
-    const bool fused_hist = T == 1 && B <= kNumSMs;
+    const int sms = device_sm_count();
+    if (sms <= 0) return cuda_status(cudaErrorInvalidDevice);
+    const bool fused_hist = T == 1 && B <= sms;
     if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess)
       return cuda_status(e);
     if ((e = launch_index_score_tc(iq, w, ik, B, T, N, q_pos0, scores, fused_hist ? tws.hist : nullptr, stream)) !=

@@ -28,6 +28,31 @@ struct DeviceOnce {
   }
 };
 
+// Device address of a file-scope __device__ int (an error word), looked up once per device
+// with that device current.  Instantiate it in the file that defines the variable.
+struct SymbolAddress {
+  std::atomic<int*> ptr[64] = {};
+  template <class Sym>
+  cudaError_t get(const Sym& symbol, int** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    int* p = ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+      void* v = nullptr;
+      if ((e = cudaGetSymbolAddress(&v, symbol)) != cudaSuccess) return e;
+      p = static_cast<int*>(v);
+      ptr[dev].store(p, std::memory_order_release);
+    }
+    *out = p;
+    return cudaSuccess;
+  }
+};
+
+// SM count of the current device, read once per device (0 if it cannot be read)
+int device_sm_count();
+
 // DSA_OK for cudaSuccess; otherwise records `e` as the last CUDA error (dsa_last_cuda_error)
 // and returns DSA_ERR_CUDA
 dsa_status cuda_status(cudaError_t e);
@@ -70,7 +95,7 @@ struct AttnLayers {
 
 constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core attention
 
-int attn_num_splits(long long rows, int L, int k, const int* cluster_fit);
+int attn_num_splits(long long rows, int L, int k, int sm_budget, const int* cluster_fit);
 int attn_split_chunk(int k, int nsplit);
 size_t attn_workspace_bytes(long long rows, int L, int H, int k);
 
@@ -78,22 +103,29 @@ size_t attn_workspace_bytes(long long rows, int L, int H, int k);
 // histogram pointer (decode only, B <= 148) the first radix digit of the select is counted.
 cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
                                   long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream);
-// error word of the tensor-core kernels' bounded waits (0 = none)
-cudaError_t indexer_tc_device_error(int* code, bool clear);
+// Device addresses of the error words: the indexer's and the attention's bounded waits
+// record a code when they run out; the top-k records one when a selection invariant
+// fails (the selected count is not k).  0 = none.
+cudaError_t indexer_error_word(int** p);
+cudaError_t attn_error_word(int** p);
+cudaError_t topk_error_word(int** p);
+
+// Whether launch_topk takes the scan kernels for this shape (and so reads and writes the
+// workspace): false when every row fits one cluster of CTAs on chip.
+bool topk_uses_workspace(long long rows, long long vmax);
 
 cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
                         const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream);
 // top-k of rows short enough for one cluster of CTAs (topk_cluster.cu); launch_topk
 // chooses it when topk_cluster_plan accepts the shape.  `hist` (nullable) holds the
 // first digit's histogram per row, counted by the indexer.
-bool topk_cluster_plan(long long rows, long long vmax, int* C, int* kpt);
+bool topk_cluster_plan(long long rows, long long vmax, int sms, int* C, int* kpt);
 cudaError_t launch_topk_cluster(const float* scores, int B, int T, int N, long long q_pos0, int k, int C, int kpt,
-                                const uint32_t* hist, int32_t* idx, cudaStream_t stream);
+                                const uint32_t* hist, int32_t* idx, int* err, cudaStream_t stream);
 
 // q_early: the kernel before it in the stream does not write the queries (it is the
 // group's own top-k), so they are loaded before that kernel completes
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
                                   int k, float scale, void* ws, bool q_early, cudaStream_t stream);
-cudaError_t attn_tc_device_error(int* code, bool clear);
 
 }  // namespace dsa

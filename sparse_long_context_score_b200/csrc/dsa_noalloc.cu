@@ -1,17 +1,21 @@
 // dsa_noalloc.cu -- top-k select for callers that cannot allocate device memory.
 //
 // Some callers of this library may not allocate GPU memory at the point where they run
-// the select: a plugin inside an inference engine whose enqueue step must not allocate,
-// a serving loop that works inside a fixed, pre-planned memory budget, or code being
-// recorded into a CUDA graph, where cudaMalloc is not allowed.  dsa_topk_noalloc serves
-// them: its scratch memory is a fixed array compiled into the library (below), so the
-// caller passes only the scores and the output buffer.
+// the select: a plugin inside an inference engine whose enqueue step must not allocate
+// (the engine owns every buffer), a serving loop that works inside a fixed, pre-planned
+// memory budget, or a latency-critical host thread that must not call cudaMalloc, which
+// can synchronise the whole device.  dsa_topk_noalloc serves them: its scratch memory is
+// a fixed array compiled into the library (below), so the caller passes only the scores
+// and the output buffer.  Shapes whose rows each fit one cluster of CTAs on chip use no
+// scratch at all; the others (many rows, or rows longer than a cluster holds) take the
+// scan kernels, whose scratch must fit the array.
 //
 // The array lives in every GPU that loads the library until the process exits.  All
 // calls share it and it keeps the last call's contents; the parts that must start at
 // zero are cleared on the stream at the start of every call.  Two calls that overlap on
 // the GPU (different streams, no ordering between them) race on it.
 #include "dsa.h"
+#include "dsa_common.cuh"
 #include "dsa_internal.h"
 
 namespace {
@@ -51,7 +55,9 @@ extern "C" dsa_status dsa_topk_noalloc(const float* scores, int B, int T, int N,
   if (k > DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
   if ((reinterpret_cast<uintptr_t>(scores) | reinterpret_cast<uintptr_t>(idx)) % 4) return DSA_ERR_INVALID_ARG;
   const long long rows = (long long)B * T;
-  if (dsa::topk_workspace_bytes(rows, N) > kScratchBytes) return DSA_ERR_WORKSPACE;
+  const long long vmax = dsa::visible_count(N, q_pos0, T - 1);
+  if (dsa::topk_uses_workspace(rows, vmax) && dsa::topk_workspace_bytes(rows, N) > kScratchBytes)
+    return DSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   const cudaError_t ea = g_scratch_address.get(&scratch);
   if (ea != cudaSuccess) return dsa::cuda_status(ea);

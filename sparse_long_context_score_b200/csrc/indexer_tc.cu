@@ -389,25 +389,7 @@ bool make_map(CUtensorMap* map, const void* base, long long d1, long long d2, in
   return r == CUDA_SUCCESS;
 }
 
-struct ErrAddr {
-  std::atomic<int*> ptr[64] = {};
-  cudaError_t get(int** out) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    int* p = ptr[dev].load();
-    if (!p) {
-      void* v = nullptr;
-      if ((e = cudaGetSymbolAddress(&v, g_indexer_tc_error)) != cudaSuccess) return e;
-      p = static_cast<int*>(v);
-      ptr[dev].store(p);
-    }
-    *out = p;
-    return cudaSuccess;
-  }
-};
-ErrAddr g_err_addr;
+SymbolAddress g_err_addr;
 
 template <int QG, bool kHist>
 cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N, long long q_pos0,
@@ -417,7 +399,7 @@ cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int 
   if (!make_map(&kmap, k, N, B, kTileKeys) || !make_map(&qmap, q, (long long)T * 32, B, C::kN))
     return cudaErrorInvalidValue;
   int* err = nullptr;
-  cudaError_t e = g_err_addr.get(&err);
+  cudaError_t e = g_err_addr.get(g_indexer_tc_error, &err);
   if (e != cudaSuccess) return e;
   static DeviceOnce once;
   if ((e = once.run([] {
@@ -434,7 +416,9 @@ cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int 
     total += (v + kTileKeys - 1) / kTileKeys;
   }
   if (total == 0) return cudaSuccess;
-  const int grid = (int)(total < kNumSMs ? total : kNumSMs);
+  const int sms = device_sm_count();
+  if (sms <= 0) return cudaErrorInvalidDevice;
+  const int grid = (int)(total < sms ? total : sms);
   indexer_tc_kernel<QG, kHist><<<grid, C::kThreads, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
                                                                        hist, err);
   return cudaGetLastError();
@@ -445,8 +429,8 @@ cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int 
 cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
                                   long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream) {
   // the fused histogram keeps two row slots per CTA: with contiguous item ranges over
-  // at most 148 CTAs a range spans at most two sequences when B <= 148
-  if (hist && (T != 1 || B > kNumSMs)) return cudaErrorNotSupported;
+  // at most one CTA per SM a range spans at most two sequences when B <= the SM count
+  if (hist && (T != 1 || B > device_sm_count())) return cudaErrorNotSupported;
   if (T == 1) {
     return hist ? launch_tc<1, true>(q, w, k, B, T, N, q_pos0, scores, hist, stream)
                 : launch_tc<1, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, stream);
@@ -454,13 +438,6 @@ cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint1
   return launch_tc<8, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, stream);
 }
 
-cudaError_t indexer_tc_device_error(int* code, bool clear) {
-  int* p = nullptr;
-  cudaError_t e = g_err_addr.get(&p);
-  if (e != cudaSuccess) return e;
-  if ((e = cudaMemcpy(code, p, sizeof(int), cudaMemcpyDeviceToHost)) != cudaSuccess) return e;
-  if (clear && *code) e = cudaMemset(p, 0, sizeof(int));
-  return e;
-}
+cudaError_t indexer_error_word(int** p) { return g_err_addr.get(g_indexer_tc_error, p); }
 
 }  // namespace dsa

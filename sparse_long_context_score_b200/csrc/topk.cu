@@ -36,6 +36,9 @@ namespace dsa {
 
 namespace {
 
+static __device__ int g_topk_error;
+SymbolAddress g_topk_err_addr;
+
 constexpr int kHistThreads = 256;
 constexpr int kSelThreads = 512;
 constexpr int kCmpThreads = 256;
@@ -190,7 +193,7 @@ __device__ uint64_t resolve_threshold(SelectSmem& sm, long long count, uint32_t 
 
 __global__ void __launch_bounds__(kSelThreads)
 topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, int k, TopkWorkspace ws,
-                   int32_t* __restrict__ idx_out, int vec) {
+                   int32_t* __restrict__ idx_out, int vec, int* __restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   SelectSmem& sm = *reinterpret_cast<SelectSmem*>(smem_raw);
   const int row = blockIdx.x;
@@ -388,6 +391,8 @@ topk_select_kernel(const float* __restrict__ scores, int T, int N, long long q_p
     carry += sm.total;
     __syncthreads();
   }
+  // every row selects exactly k elements (k < V here); anything else is a broken invariant
+  if (threadIdx.x == 0 && carry != (uint32_t)k) atomicCAS(err, 0, 42);
   if (threadIdx.x == 0) {
     state[RS_THR_LO] = (uint32_t)thr;
     state[RS_THR_HI] = (uint32_t)(thr >> 32);
@@ -498,6 +503,8 @@ topk_compact_kernel(const float* __restrict__ scores, int T, int N, long long q_
 
 }  // namespace
 
+cudaError_t topk_error_word(int** p) { return g_topk_err_addr.get(g_topk_error, p); }
+
 size_t topk_workspace_bytes(long long rows, int N) {
   const long long nchunks = ((long long)N + kTopkChunk - 1) / kTopkChunk;
   size_t b = 0;
@@ -533,6 +540,11 @@ TopkWorkspace topk_workspace(void* base, long long rows, int N) {
   return w;
 }
 
+bool topk_uses_workspace(long long rows, long long vmax) {
+  int C = 0, kpt = 0;
+  return !topk_cluster_plan(rows, vmax, device_sm_count(), &C, &kpt);
+}
+
 cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
                         const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream) {
   const long long rows = (long long)B * T;
@@ -540,8 +552,10 @@ cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_po
   const long long nchunks_all = ((long long)N + kTopkChunk - 1) / kTopkChunk;
   cudaError_t e;
   int C = 0, kpt = 0;
-  if (topk_cluster_plan(rows, vmax, &C, &kpt))
-    return launch_topk_cluster(scores, B, T, N, q_pos0, k, C, kpt, hist_ready ? ws.hist : nullptr, idx, stream);
+  int* err = nullptr;
+  if ((e = g_topk_err_addr.get(g_topk_error, &err)) != cudaSuccess) return e;
+  if (topk_cluster_plan(rows, vmax, device_sm_count(), &C, &kpt))
+    return launch_topk_cluster(scores, B, T, N, q_pos0, k, C, kpt, hist_ready ? ws.hist : nullptr, idx, err, stream);
   if (!hist_ready) {
     e = cudaMemsetAsync(ws.hist, 0, ws.zero_bytes, stream);
     if (e != cudaSuccess) return e;
@@ -560,7 +574,7 @@ cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_po
        })) != cudaSuccess)
     return e;
   topk_select_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kSelThreads, smem, stream>>>(scores, T, N, q_pos0,
-                                                                                                  k, ws, idx, vec);
+                                                                                                  k, ws, idx, vec, err);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   topk_compact_kernel<<<dim3((unsigned)rows, (unsigned)nchunks_all), kCmpThreads, 0, stream>>>(scores, T, N, q_pos0,
                                                                                                 k, ws, idx, vec);

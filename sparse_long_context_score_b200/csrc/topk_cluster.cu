@@ -121,7 +121,7 @@ __device__ void first_digit_sum(ClusterSmem& sm, int C, int me) {
 template <int KPT>
 __global__ void __launch_bounds__(kCT, 1)
 topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, int k, int vec,
-                    const uint32_t* __restrict__ hist_g, int32_t* __restrict__ idx_out) {
+                    const uint32_t* __restrict__ hist_g, int32_t* __restrict__ idx_out, int* __restrict__ err) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   ClusterSmem& sm = *reinterpret_cast<ClusterSmem*>(smem_raw);
   uint32_t* keys = reinterpret_cast<uint32_t*>(smem_raw + kKeysOff);
@@ -302,6 +302,12 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   cluster_sync();  // every CTA's count is in every CTA; no shared-memory access across CTAs after this
   uint32_t o = wbase;
   for (int q = 0; q < me; ++q) o += sm.nsel[q];
+  if (me == 0 && threadIdx.x == 0) {
+    // every row selects exactly k elements (k < V here); anything else is a broken invariant
+    uint32_t total = 0;
+    for (int q = 0; q < C; ++q) total += sm.nsel[q];
+    if (total != (uint32_t)k) atomicCAS(err, 0, 41);
+  }
 #pragma unroll 4
   for (int step = 0; step < KPT; ++step) {
     const bool b = (sel >> step) & 1u;
@@ -315,7 +321,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
 }
 template <int KPT>
 cudaError_t launch_kpt(const float* scores, long long rows, int T, int N, long long q_pos0, int k, int C,
-                       const uint32_t* hist, int32_t* idx, cudaStream_t stream) {
+                       const uint32_t* hist, int32_t* idx, int* err, cudaStream_t stream) {
   const int smem = kKeysOff + kCT * KPT * 4;
   static DeviceOnce once;
   cudaError_t e = once.run([&] {
@@ -337,7 +343,7 @@ cudaError_t launch_kpt(const float* scores, long long rows, int T, int N, long l
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<KPT>, scores, T, N, q_pos0, k, vec, hist, idx);
+  return cudaLaunchKernelEx(&cfg, topk_cluster_kernel<KPT>, scores, T, N, q_pos0, k, vec, hist, idx, err);
 }
 
 }  // namespace
@@ -346,12 +352,12 @@ cudaError_t launch_kpt(const float* scores, long long rows, int T, int N, long l
 // smallest C (1, 2, 4, 8) whose chunk of 1024 x kpt positions, kpt <= 16, covers a row,
 // else C = 8 with kpt = 32.  False when a row is longer than that, or when the clusters
 // would not fit the GPU in about one wave (many rows: the scan kernels do better).
-bool topk_cluster_plan(long long rows, long long vmax, int* C, int* kpt) {
+bool topk_cluster_plan(long long rows, long long vmax, int sms, int* C, int* kpt) {
   for (int c = 1; c <= 8; c *= 2) {
     const long long per = (vmax + (long long)c * kCT - 1) / ((long long)c * kCT);
     int kp = per <= 4 ? 4 : per <= 8 ? 8 : per <= 16 ? 16 : per <= 32 ? 32 : 0;
     if (kp == 0 || (kp == 32 && c < 8)) continue;
-    if (rows * c > kNumSMs) return false;
+    if (rows * c > sms) return false;
     *C = c;
     *kpt = kp;
     return true;
@@ -360,13 +366,13 @@ bool topk_cluster_plan(long long rows, long long vmax, int* C, int* kpt) {
 }
 
 cudaError_t launch_topk_cluster(const float* scores, int B, int T, int N, long long q_pos0, int k, int C, int kpt,
-                                const uint32_t* hist, int32_t* idx, cudaStream_t stream) {
+                                const uint32_t* hist, int32_t* idx, int* err, cudaStream_t stream) {
   const long long rows = (long long)B * T;
   switch (kpt) {
-    case 4: return launch_kpt<4>(scores, rows, T, N, q_pos0, k, C, hist, idx, stream);
-    case 8: return launch_kpt<8>(scores, rows, T, N, q_pos0, k, C, hist, idx, stream);
-    case 16: return launch_kpt<16>(scores, rows, T, N, q_pos0, k, C, hist, idx, stream);
-    case 32: return launch_kpt<32>(scores, rows, T, N, q_pos0, k, C, hist, idx, stream);
+    case 4: return launch_kpt<4>(scores, rows, T, N, q_pos0, k, C, hist, idx, err, stream);
+    case 8: return launch_kpt<8>(scores, rows, T, N, q_pos0, k, C, hist, idx, err, stream);
+    case 16: return launch_kpt<16>(scores, rows, T, N, q_pos0, k, C, hist, idx, err, stream);
+    case 32: return launch_kpt<32>(scores, rows, T, N, q_pos0, k, C, hist, idx, err, stream);
     default: return cudaErrorInvalidValue;
   }
 }
