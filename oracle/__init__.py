@@ -17,7 +17,7 @@ import subprocess
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRC = os.path.join(_HERE, "dsa_oracle.c")
+_SRCS = [os.path.join(_HERE, "dsa_oracle.c"), os.path.join(_HERE, "verify_oracle.c")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 OR_OK = 0
@@ -26,19 +26,22 @@ OR_ERR_NOMEM = -2
 OR_ERR_INVARIANT = -3
 
 
-def compile_c(src: str, out: str) -> str:
-    """gcc -O2 (no fast-math) of one oracle source into a shared library."""
+def compile_c(srcs, out: str) -> str:
+    """gcc -O2 (no fast-math) of the oracle sources into one shared library."""
+    srcs = [srcs] if isinstance(srcs, str) else list(srcs)
     tmp = out + ".tmp%d" % os.getpid()
-    subprocess.check_call(["gcc", "-O2", "-std=c11", "-Wall", "-Wextra", "-fPIC", "-shared",
-                           "-o", tmp, src, "-lm"])
+    subprocess.check_call(["gcc", "-O2", "-std=gnu11", "-Wall", "-Wextra", "-fPIC", "-shared",
+                           "-o", tmp, *srcs, "-lm"])
     os.replace(tmp, out)
     return out
 
 
 def build(force: bool = False) -> str:
-    """Compile dsa_oracle.c into liboracle.so next to it (rebuilt when the source is newer)."""
-    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        compile_c(_SRC, _LIB)
+    """Compile the oracle sources into liboracle.so next to them (rebuilt when a source is
+    newer)."""
+    newest = max(os.path.getmtime(x) for x in _SRCS)
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < newest:
+        compile_c(_SRCS, _LIB)
     return _LIB
 
 
@@ -54,8 +57,9 @@ class Oracle:
         L.oracle_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P]
         L.oracle_dense_masked_attn.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P]
         L.oracle_group_forward.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Lg, I, I, I, I, D, I, P, P]
+        L.oracle_verify.argtypes = [P, P, P, P, P, I, I, I, P, P, P, P]
         for f in ("oracle_index_score", "oracle_topk", "oracle_sparse_attn",
-                  "oracle_dense_masked_attn", "oracle_group_forward"):
+                  "oracle_dense_masked_attn", "oracle_group_forward", "oracle_verify"):
             getattr(L, f).restype = I
         self.L = L
 
@@ -126,6 +130,26 @@ class Oracle:
         return idx_shared, outs
 
 
+    def verify(self, p: np.ndarray, q: np.ndarray, draft: np.ndarray, u: np.ndarray, u2: np.ndarray):
+        """MTP verify step (rejection sampling), verify_oracle.c.  p, q [B, S, V] float32
+        target / draft probabilities; draft, u, u2 [B, S].  Returns (alpha [B,S] f64,
+        accept [B,S] i32, token [B,S] i32, accepted_len [B] i32)."""
+        p = np.ascontiguousarray(p, dtype=np.float32)
+        q = np.ascontiguousarray(q, dtype=np.float32)
+        B, S, V = p.shape
+        assert q.shape == p.shape
+        draft = np.ascontiguousarray(draft, dtype=np.int32).reshape(B, S)
+        u = np.ascontiguousarray(u, dtype=np.float32).reshape(B, S)
+        u2 = np.ascontiguousarray(u2, dtype=np.float32).reshape(B, S)
+        alpha = np.empty((B, S), np.float64)
+        accept = np.empty((B, S), np.int32)
+        token = np.empty((B, S), np.int32)
+        alen = np.empty((B,), np.int32)
+        _check(self.L.oracle_verify(_ptr(p), _ptr(q), _ptr(draft), _ptr(u), _ptr(u2), B, S, V, _ptr(alpha),
+                                    _ptr(accept), _ptr(token), _ptr(alen)), "oracle_verify")
+        return alpha, accept, token, alen
+
+
 def _ptr(a: np.ndarray) -> int:
     return a.ctypes.data
 
@@ -166,3 +190,7 @@ def sparse_attn(*a, **kw):
 
 def group_forward(*a, **kw):
     return default().group_forward(*a, **kw)
+
+
+def verify(*a, **kw):
+    return default().verify(*a, **kw)

@@ -356,4 +356,108 @@ def pin_mtp_draft_rows_never_attended(o):
         assert np.array_equal(oa[0], ob[0])
 
 
+# ------------------------------------------------------------------ MTP verify step
+# "GLM-5.2 MTP IndexShare inference", Rejection Sampling: the acceptance rate is the sum
+# over the vocabulary of the smaller of the two probabilities.  The accept / resample rule
+# read from it is the standard speculative-sampling rule; its defining property is that
+# the token it emits is distributed as the target distribution p.
+
+def _dist(seed, V, rows, temp=1.0):
+    """rows float32 probability vectors of length V (softmax of Gaussian logits, f32)."""
+    r = _rng(seed)
+    z = (r.standard_normal((rows, V)) * temp).astype(np.float32)
+    e = np.exp(z - z.max(axis=1, keepdims=True), dtype=np.float32)
+    return (e / e.sum(axis=1, keepdims=True, dtype=np.float32)).astype(np.float32)
+
+
+def pin_verify_identical_distributions(o):
+    """p == q: the acceptance rate is 1 and every draft token is kept."""
+    p = _dist(5, 300, 6).reshape(2, 3, 300)
+    draft = np.array([[3, 77, 299], [0, 150, 12]], np.int32)
+    u = np.full((2, 3), 0.999, np.float32)
+    a, acc, tok, alen = o.verify(p, p, draft, u, np.full((2, 3), 0.5, np.float32))
+    assert np.allclose(a, 1.0, atol=1e-6)
+    assert np.all(acc == 1) and np.array_equal(tok, draft) and np.all(alen == 3)
+
+
+def pin_verify_disjoint_supports(o):
+    """Disjoint supports: the acceptance rate is 0, every draft token is rejected and the
+    replacement comes from the target's support."""
+    V = 10
+    p = np.zeros((1, 2, V), np.float32)
+    q = np.zeros((1, 2, V), np.float32)
+    p[..., :5] = 0.2
+    q[..., 5:] = 0.2
+    a, acc, tok, alen = o.verify(p, q, np.array([[7, 9]], np.int32), np.array([[0.0, 0.5]], np.float32),
+                                 np.array([[0.1, 0.95]], np.float32))
+    assert np.allclose(a, 0.0) and np.all(acc == 0) and alen[0] == 0
+    assert tok[0, 0] == 0 and tok[0, 1] == 4  # inverse CDF of the uniform residual over 0..4
+
+
+def pin_verify_alpha_is_one_minus_tv(o):
+    """sum_v min(p_v, q_v) = (sum p + sum q)/2 - (1/2) sum |p - q| for any vectors, which is
+    1 - TV(p, q) for normalised ones."""
+    p = _dist(6, 4096, 8).reshape(2, 4, 4096)
+    q = _dist(7, 4096, 8, temp=1.5).reshape(2, 4, 4096)
+    a, _, _, _ = o.verify(p, q, np.zeros((2, 4), np.int32), np.zeros((2, 4), np.float32),
+                          np.zeros((2, 4), np.float32))
+    pd, qd = p.astype(np.float64), q.astype(np.float64)
+    assert np.allclose(a, 0.5 * (pd.sum(axis=2) + qd.sum(axis=2)) - 0.5 * np.abs(pd - qd).sum(axis=2), atol=1e-12)
+    assert np.allclose(a, 1.0 - 0.5 * np.abs(pd - qd).sum(axis=2), atol=2e-5)
+    assert np.all((a > 0.0) & (a < 1.0))
+
+
+def _grid(m):
+    return ((np.arange(m) + 0.5) / m).astype(np.float32)
+
+
+def pin_verify_accept_probability(o):
+    """Over a fine grid of u, the draft token x is accepted with frequency min(1, p_x/q_x)."""
+    p = np.array([0.4, 0.1, 0.3, 0.15, 0.05], np.float32)
+    q = np.array([0.2, 0.3, 0.3, 0.05, 0.15], np.float32)
+    M = 1000
+    u = _grid(M)
+    for x in range(5):
+        P = np.broadcast_to(p, (1, M, 5)).copy()
+        Q = np.broadcast_to(q, (1, M, 5)).copy()
+        _, acc, _, _ = o.verify(P, Q, np.full((1, M), x, np.int32), u.reshape(1, M), np.zeros((1, M), np.float32))
+        assert abs(acc.mean() - min(1.0, float(p[x]) / float(q[x]))) <= 2.0 / M, x
+
+
+def pin_verify_output_is_distributed_as_target(o):
+    """Speculative sampling's defining property: with x ~ q, u and u2 uniform, the emitted
+    token is distributed as p.  Enumerated on a tiny vocabulary: x weighted by q_x, u and
+    u2 on fine grids."""
+    p = np.array([0.05, 0.35, 0.2, 0.25, 0.15], np.float32)
+    q = np.array([0.3, 0.1, 0.2, 0.05, 0.35], np.float32)
+    M = 200
+    uu, vv = np.meshgrid(_grid(M), _grid(M), indexing="ij")
+    n = M * M
+    out = np.zeros(5)
+    for x in range(5):
+        P = np.broadcast_to(p, (1, n, 5)).copy()
+        Q = np.broadcast_to(q, (1, n, 5)).copy()
+        _, acc, tok, _ = o.verify(P, Q, np.full((1, n), x, np.int32), uu.reshape(1, n), vv.reshape(1, n))
+        out += float(q[x]) * np.bincount(tok.ravel(), minlength=5) / n
+        # a resampled token always has p > q
+        rej = tok[acc == 0]
+        assert np.all(p[rej] > q[rej])
+    assert np.allclose(out, p, atol=0.01), out
+
+
+def pin_verify_accepted_length_is_leading_run(o):
+    """The sequence is cut at its first rejection: accepted_len counts the leading
+    accepted positions only."""
+    V = 4
+    p = np.tile(np.array([0.7, 0.1, 0.1, 0.1], np.float32), (3, 5, 1))
+    q = np.tile(np.array([0.1, 0.7, 0.1, 0.1], np.float32), (3, 5, 1))
+    # token 0 (p > q) is always accepted; token 1 with u near 1 is rejected
+    draft = np.array([[0, 0, 1, 0, 0], [1, 0, 0, 0, 0], [0, 0, 0, 0, 0]], np.int32)
+    u = np.full((3, 5), 0.99, np.float32)
+    _, acc, tok, alen = o.verify(p, q, draft, u, np.full((3, 5), 0.3, np.float32))
+    assert alen.tolist() == [2, 0, 5]
+    assert acc.sum() == 13 and tok[0, 2] == 0 and tok[1, 0] == 0
+    del V
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

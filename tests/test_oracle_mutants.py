@@ -9,7 +9,10 @@ import pytest
 import oracle
 import pins
 
-SRC = os.path.join(os.path.dirname(oracle.__file__), "dsa_oracle.c")
+HERE = os.path.dirname(oracle.__file__)
+SRC = os.path.join(HERE, "dsa_oracle.c")
+VERIFY_SRC = os.path.join(HERE, "verify_oracle.c")
+SOURCES = [SRC, VERIFY_SRC]
 
 MUTANTS = {
     "relu_dropped": ("double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
@@ -29,18 +32,29 @@ MUTANTS = {
                      "for (int d = 0; d < dv; ++d) o[d] += p * bf16_to_double(c[d + 64]);"),
     "not_normalised": ("double p = exp(z[j] - zmax) / denom;", "double p = exp(z[j] - zmax);"),
     "reuse_ignored": ("if (compute_indices) {", "if (1) {"),
+    # MTP verify step (verify_oracle.c)
+    "verify_max_not_min": ("a += (double)(p[v] < q[v] ? p[v] : q[v]);", "a += (double)(p[v] > q[v] ? p[v] : q[v]);",
+                           VERIFY_SRC),
+    "verify_accept_reversed": ("accept[r] = uq < pr[x] ? 1 : 0;", "accept[r] = uq > pr[x] ? 1 : 0;", VERIFY_SRC),
+    "verify_residual_sign": ("float r = p[v] - q[v];\n        if (r > 0.0f) run",
+                             "float r = q[v] - p[v];\n        if (r > 0.0f) run", VERIFY_SRC),
+    "verify_resample_from_p": (": resample(pr, qr, V, u2[r], x)", ": resample(pr, pr, V, u2[r], x)",
+                               VERIFY_SRC),
+    "verify_len_counts_all": ("while (n < S && accept[(long)b * S + n]) ++n;",
+                              "for (int j = 0; j < S; ++j) n += accept[(long)b * S + j];", VERIFY_SRC),
 }
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(tmp_path, name):
-    old, new = MUTANTS[name]
-    text = open(SRC).read()
+    old, new, target = (MUTANTS[name] + (SRC,))[:3]
+    text = open(target).read()
     assert text.count(old) >= 1, f"mutation site for {name} not found"
     mutated = text.replace(old, new, 1)
     src = tmp_path / f"mutant_{name}.c"
     src.write_text(mutated)
-    so = oracle.compile_c(str(src), str(tmp_path / f"mutant_{name}.so"))
+    others = [x for x in SOURCES if x != target]
+    so = oracle.compile_c([str(src)] + others, str(tmp_path / f"mutant_{name}.so"))
     m = oracle.Oracle(so)
     caught = []
     for pin in pins.ALL_PINS:
