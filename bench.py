@@ -42,7 +42,10 @@ def parse():
     p.add_argument("--cpu-sample", type=int, default=2, help="sequences in the CPU-oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra", action="store_true", help="skip the 1M / MTP / prefill workloads")
-    p.add_argument("--ncu-case", choices=["indexer", "topk", "attn"],
+    p.add_argument("--schedule", default="micro", choices=["micro", "sequential"],
+                   help="decode workloads: dsa_decode_step (two micro-batches on two streams) or one "
+                        "dsa_group_forward per group in order on one stream")
+    p.add_argument("--ncu-case", choices=["indexer", "topk", "attn", "indexer_prefill", "attn_mtp", "topk_1m"],
                    help="run one kernel of the decode step a few times on a profiler-sized case and exit "
                         "(for ncu captures; prints no benchmark line)")
     return p.parse_args()
@@ -247,8 +250,13 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     torch.cuda.set_device(device)
     dsa.lib()
     groups = make_inputs(w, device, rank)
-    ws = dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, device)
+    micro = args.schedule == "micro" and w.T == 1 and w.steps == 1 and w.B >= 2
+    ws = dsa.decode_workspace(w.B, w.N, w.k, w.H, w.L, device) if micro else \
+        dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, device)
     stream = torch.cuda.Stream(device)
+    side = torch.cuda.Stream(device)
+    dgroups = [dict(iq=g["iq"], w=g["wt"], ik=g["ik"], qs=g["qs"], kvs=g["kvs"], idx=g["idx"], outs=g["outs"])
+               for g in groups]
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
     flush_rd = torch.zeros(512 << 20, dtype=torch.uint8, device=device)
 
@@ -259,6 +267,9 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         flush_rd.view(torch.int64).sum()
 
     def step():
+        if micro:
+            dsa.dsa_decode_step(dgroups, w.k, C.SCALE, ws=ws, stream=stream, side=side)
+            return
         for g in groups:
             dsa.dsa_group_forward(g["iq"], g["wt"], g["ik"], g["qs"], g["kvs"], w.q_pos0, w.k, C.SCALE,
                                   idx_shared=g["idx"], outs=g["outs"], ws=ws, stream=stream)
@@ -306,7 +317,8 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    res = {"step_ms": sum(times) / len(times), "clocks": clk.summary()}
+    res = {"step_ms": sum(times) / len(times), "clocks": clk.summary(),
+           "schedule": "two micro-batches (dsa_decode_step)" if micro else "groups in order (dsa_group_forward)"}
 
     # the dominant kernel alone: the indexer over the first group's cache, same launch shape
     g0 = groups[0]
@@ -355,9 +367,62 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         keys = ["step_ms", "idx_ms"]
     for k, v in zip(keys, max_over_ranks([res[k] for k in keys], world, device)):
         res[k] = v
-    del groups, ws, flush, flush_rd, scores, graph, igraph
+    del groups, dgroups, ws, flush, flush_rd, scores, graph, igraph
     torch.cuda.empty_cache()
     return w, res
+
+
+VERIFY_VOCAB = 151552  # a GLM-sized vocabulary (the pages do not fix it)
+
+
+def run_verify(args, device, peak):
+    """The MTP verify step (dsa_verify) for the mtp workload's 16 sequences x 7 draft
+    positions over a 151552-entry vocabulary: graph-captured, L2 flushed before each of
+    K timed runs; HBM-bound (8 B read per vocabulary entry and position)."""
+    import torch
+    import sparse_long_context_score_b200 as dsa
+    import synth
+    import synth.device as sd
+    from synth import configs as C
+    w = C.WORKLOADS["mtp"]
+    B, S, V = w.B, w.steps, VERIFY_VOCAB
+    torch.cuda.set_device(device)
+    zp = sd.normal_bf16(torch.empty(B, S, V, dtype=torch.bfloat16, device=device), w.key(synth.KIND_Q, 1, 0))
+    zq = sd.normal_bf16(torch.empty(B, S, V, dtype=torch.bfloat16, device=device), w.key(synth.KIND_Q, 1, 1))
+    p = torch.softmax(zp.float() * 2.0, dim=-1).contiguous()
+    q = torch.softmax(zq.float() * 2.6 + zp.float(), dim=-1).contiguous()
+    draft = torch.argmax(q, dim=-1).to(torch.int32).contiguous()
+    u = sd.unit_f32(torch.empty(B, S, dtype=torch.float32, device=device), w.key(synth.KIND_SCORES, 1, 0)) + 0.5
+    u2 = sd.unit_f32(torch.empty(B, S, dtype=torch.float32, device=device), w.key(synth.KIND_SCORES, 1, 1)) + 0.5
+    stream = torch.cuda.Stream(device)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(512 << 20, dtype=torch.uint8, device=device)
+    with torch.cuda.stream(stream):
+        dsa.dsa_verify(p, q, draft, u, u2, stream=stream)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        dsa.dsa_verify(p, q, draft, u, u2, stream=stream)
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            flush.zero_()
+            flush_rd.view(torch.int64).sum()
+            graph.replay()
+        for a, b in ev:
+            flush.zero_()
+            flush_rd.view(torch.int64).sum()
+            a.record(stream)
+            graph.replay()
+            b.record(stream)
+    torch.cuda.synchronize()
+    ms = sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+    nbytes = 2 * B * S * V * 4
+    del zp, zq, p, q, flush, flush_rd, graph
+    torch.cuda.empty_cache()
+    return {"B": B, "draft_steps": S, "vocab": V, "us_per_step": ms * 1e3, "hbm_gbs": nbytes / (ms * 1e-3) / 1e9,
+            "roofline_frac": nbytes / (ms * 1e-3) / 1e9 / peak, "algorithmic_bytes": nbytes}
 
 
 def host_cpu() -> dict:
@@ -434,11 +499,13 @@ def workload_config(w, world: int) -> dict:
             "l2": "flushed before every timed step (512 MiB write, then a 512 MiB read so the write-back is not timed)"}
 
 
-def launches_per_group(w) -> int:
-    """libdsa kernels one dsa_group_forward launches: the indexer, the top-k (one cluster
-    kernel for decode-shaped rows, else a select and a compact kernel, plus a histogram
-    kernel when the indexer does not count the first digit) and one attention launch for
-    all layers.  Mirrors the shape rules of the library (topk_cluster_plan)."""
+def launches_per_group(w, sms: int = 148, long_per_sm: int = 4) -> int:
+    """libdsa kernels one dsa_group_forward launches: the indexer, the top-k and one
+    attention launch for all layers.  The top-k is one kernel for rows a cluster holds
+    (decode shapes) and for long rows whose CTAs (one per 8192 scores) all fit the GPU at
+    once (a cooperative launch: `long_per_sm` of them per SM); otherwise a select and a
+    compact kernel, plus a histogram kernel when the indexer does not count the first
+    digit.  Mirrors the shape rules of the library (topk_cluster_plan, launch_topk)."""
     rows = w.B * w.T
     vmax = min(w.N, w.q_pos0 + w.T)
     cluster = False
@@ -447,18 +514,38 @@ def launches_per_group(w) -> int:
         kp = 4 if per <= 4 else 8 if per <= 8 else 16 if per <= 16 else 32 if per <= 32 else 0
         if kp == 0 or (kp == 32 and c < 8):
             continue
-        cluster = rows * c <= 148
+        cluster = rows * c <= sms
         break
-    fused_hist = w.T == 1 and w.B <= 148
-    topk = 1 if cluster else (2 if fused_hist else 3)
+    nchunks = -(-w.N // 8192)
+    long_rows = nchunks <= 512 and rows * nchunks <= long_per_sm * sms
+    fused_hist = w.T == 1 and w.B <= sms
+    topk = 1 if (cluster or long_rows) else (2 if fused_hist else 3)
     return 1 + topk + 1
 
 
+def step_launches(w, micro: bool) -> int:
+    """libdsa kernels of one step: per group, per micro-batch (two halves of the batch when
+    the step is micro-batched), launches_per_group of that micro-batch; every MTP draft
+    step after the first adds one attention launch."""
+    from synth import configs as C
+    if not micro:
+        return (launches_per_group(w) + (w.steps - 1)) * w.groups
+    b0 = (w.B + 1) // 2
+    halves = [C.scaled(w, B=b0), C.scaled(w, B=w.B - b0)]
+    return sum(launches_per_group(h, sms=148 // 3) for h in halves if h.B > 0) * w.groups
+
+
 def ncu_case(kind: str) -> None:
-    """A few launches of one kernel of the decode128k step, sized for an ncu capture: the
-    indexer and the top-k on the full decode128k shapes (268 MB of keys, 4 MB of scores),
-    the attention on 32 (row, layer) units as in the step (4 key splits each) over caches of
-    65536 rows (2.4 GB, larger than L2) instead of 131072."""
+    """A few launches of one kernel, sized for an ncu capture (a few GB on the device):
+      indexer, topk   the decode128k shapes (268 MB of keys, 4 MB of scores);
+      attn            32 (row, layer) units as in the decode128k step (4 key splits each)
+                      over caches of 65536 rows (2.4 GB, larger than L2);
+      attn_mtp        16 units as in an MTP draft step, run once first so that the 37.7 MB
+                      of selected rows are in L2, as in draft steps 2..7;
+      indexer_prefill 512 prefill queries (causal, after 126976 cached tokens) over the
+                      131072-token key cache, QG = 8 tensor-core tiles;
+      topk_1m         the decode1m select: 2 rows of 1,048,576 scores, first digit counted
+                      by the indexer as in the step."""
     import torch
     import synth
     import synth.device as sd
@@ -480,16 +567,36 @@ def ncu_case(kind: str) -> None:
                 dsa.dsa_index_score(iq, wt, ik, w.q_pos0, scores=sc)
             else:
                 dsa.dsa_topk(sc, w.q_pos0, w.k, idx=idx, ws=ws)
+    elif kind == "indexer_prefill":
+        wp = C.WORKLOADS["prefill"]
+        T = 512
+        iq = sd.int17_bf16(torch.empty(1, T, 32, 128, dtype=bf, device="cuda"), wp.key(synth.KIND_IQ))
+        wt = sd.pow2_f32(torch.empty(1, T, 32, dtype=torch.float32, device="cuda"), wp.key(synth.KIND_W))
+        ik = sd.int17_bf16(torch.empty(1, wp.N, 128, dtype=bf, device="cuda"), wp.key(synth.KIND_IK))
+        sc = torch.empty(1, T, wp.N, dtype=torch.float32, device="cuda")
+        for _ in range(launches):
+            dsa.dsa_index_score(iq, wt, ik, wp.q_pos0, scores=sc)
+    elif kind == "topk_1m":
+        w1 = C.WORKLOADS["decode1m"]
+        iq = sd.int17_bf16(torch.empty(w1.B, 1, 32, 128, dtype=bf, device="cuda"), w1.key(synth.KIND_IQ))
+        wt = sd.pow2_f32(torch.empty(w1.B, 1, 32, dtype=torch.float32, device="cuda"), w1.key(synth.KIND_W))
+        ik = sd.int17_bf16(torch.empty(w1.B, w1.N, 128, dtype=bf, device="cuda"), w1.key(synth.KIND_IK))
+        q = sd.normal_bf16(torch.empty(w1.B, 1, w1.H, 576, dtype=bf, device="cuda"), w1.key(synth.KIND_Q))
+        kv = sd.normal_bf16(torch.empty(w1.B, w1.N, 576, dtype=bf, device="cuda"), w1.key(synth.KIND_KV))
+        ws = dsa.workspace(w1.B, 1, w1.N, w1.k, w1.H, 1)
+        for _ in range(launches):  # the group call: indexer (with the first digit) -> top-k -> attention
+            dsa.dsa_group_forward(iq, wt, ik, [q], [kv], w1.q_pos0, w1.k, C.SCALE, ws=ws)
     else:
-        rows, n = 32, 65536
+        rows, n = (32, 65536) if kind == "attn" else (16, 262151)
         q = sd.normal_bf16(torch.empty(rows, 1, w.H, 576, dtype=bf, device="cuda"), w.key(synth.KIND_Q))
         kv = sd.normal_bf16(torch.empty(rows, n, 576, dtype=bf, device="cuda"), w.key(synth.KIND_KV))
         g = torch.Generator(device="cpu").manual_seed(w.key(synth.KIND_SCORES) & 0x7FFFFFFF)
-        idx = torch.stack([torch.sort(torch.randperm(n, generator=g)[:w.k]).values for _ in range(rows)])
+        idx = torch.stack([torch.sort(torch.randperm(n - 7, generator=g)[:w.k]).values for _ in range(rows)])
         idx = idx.view(rows, 1, w.k).to(torch.int32).cuda()
         out = torch.empty(rows, 1, w.H, 512, dtype=torch.float32, device="cuda")
+        ws = dsa.workspace(rows, 1, n, w.k, w.H, 1)
         for _ in range(launches):
-            dsa.dsa_sparse_attn(q, kv, idx, C.SCALE, out=out)
+            dsa.dsa_sparse_attn(q, kv, idx, C.SCALE, out=out, ws=ws)
     torch.cuda.synchronize()
     err = dsa.dsa_device_error()
     print(f"ncu case {kind}: {launches} launches, device error word {err}")
@@ -556,15 +663,16 @@ def main():
         "e2e": {"value": tokens / (r["e2e_ms"] * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": r["h2d"],
                 "d2h_bytes_per_step": r["d2h"], "calls": "eager: the C ABI called per step",
                 "graph_replay_value": tokens / (r["e2e_graph_ms"] * 1e-3)},
-        "gpu_launches": launches_per_group(w) * w.groups * args.steps,
+        "gpu_launches": step_launches(w, r["schedule"].startswith("two")) * args.steps,
         "roofline": {"kernel": "indexer", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "peak_kind": peak_kind, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": profiled_traffic("indexer_tc.cu", w.name), "launch_us": r["idx_ms"] * 1e3,
                      "algorithmic_bytes_per_launch": idx_bytes, "score_write_bytes_per_launch": score_bytes},
-        "step": {"hbm_gbs": step_gbs, "roofline_frac": step_gbs / peak, "algorithmic_bytes": step_bytes},
+        "step": {"hbm_gbs": step_gbs, "roofline_frac": step_gbs / peak, "algorithmic_bytes": step_bytes,
+                 "schedule": r["schedule"]},
     }
     if not args.no_extra and args.workload == "decode128k":
-        extra = {}
+        extra = {"mtp_verify": run_verify(args, device, peak)}
         for name in ("decode1m", "mtp", "prefill"):
             we, r2 = run_ours(args, rank, world, device, w=C.WORKLOADS[name], e2e=False)
             b2, ib2, _ = algorithmic(we)
@@ -572,7 +680,8 @@ def main():
             toks = we.B * we.T * we.steps * world
             ent = {"tokens_per_s": toks / (ms * 1e-3), "ms_per_step": ms, "step_hbm_gbs": b2 / (ms * 1e-3) / 1e9,
                    "step_roofline_frac": b2 / (ms * 1e-3) / 1e9 / peak, "indexer_launch_us": ims * 1e3,
-                   "indexer_hbm_gbs": ib2 / (ims * 1e-3) / 1e9, "clocks_sm_mhz": r2["clocks"].get("sm_mhz"),
+                   "indexer_hbm_gbs": ib2 / (ims * 1e-3) / 1e9, "schedule": r2["schedule"],
+                   "clocks_sm_mhz": r2["clocks"].get("sm_mhz"),
                    "clock_reasons": r2["clocks"].get("reasons")}
             if name == "prefill":
                 fl = prefill_indexer_flops(we)

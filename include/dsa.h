@@ -96,9 +96,10 @@ dsa_status dsa_device_error(int *code, int clear);
 
 /*
  * Bytes of workspace needed by dsa_topk, dsa_sparse_attn and dsa_group_forward for these
- * sizes (the largest of the three; one workspace serves all calls of that size).
- * B sequences, T queries per sequence, N cached rows, k top-k, H attention heads,
- * L layers per group.  Returns 0 for invalid sizes.
+ * sizes (one workspace serves all calls of that size).  B sequences, T queries per
+ * sequence, N cached rows, k top-k, H attention heads, L layers per group.  The attention
+ * part depends on the current device's SM count (how many CTAs share a query row), so
+ * query it with the device that will run the calls current.  Returns 0 for invalid sizes.
  */
 size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L);
 
@@ -140,7 +141,7 @@ dsa_status dsa_topk(const float *scores, int B, int T, int N, long long q_pos0, 
  *   - Shapes whose rows each fit one thread-block cluster on chip (decode shapes: rows of
  *     up to 262,144 visible positions, as many rows as the GPU runs clusters for at once)
  *     use no scratch.  The other shapes take the scan kernels, whose scratch must fit the
- *     array: at most 23 query rows (B*T) for N up to 1,048,576 (fewer for longer rows);
+ *     array: at most 21 query rows (B*T) for N up to 1,048,576 (fewer for longer rows);
  *     beyond that the call returns DSA_ERR_WORKSPACE -- use dsa_topk.
  *   - The first call on a device looks up the array's device address (a runtime call,
  *     not an allocation); make that first call before any stream capture.
@@ -161,8 +162,10 @@ dsa_status dsa_topk_noalloc(const float *scores, int B, int T, int N, long long 
  *   out  [B, T, H, 512] f32    softmax_j(scale * q . kv[idx_j]) weighted sum of values;
  *                              zero when a row selects nothing
  * bf16 operands, f32 accumulation and softmax.  H in {16, 32, 48, 64}.
- * The key splits of a query row are reduced on chip, so this call needs no workspace:
- * `workspace` may be NULL and `workspace_bytes` 0 (both are ignored).
+ * When few (row, layer) units are launched, each one's keys are split over up to 8 CTAs
+ * whose partial outputs meet in `workspace` (one [64][512] f32 block per split, 128 KB);
+ * dsa_workspace_size(B, T, N, k, H, 1) covers it.  Otherwise (e.g. long prefill chunks)
+ * no workspace is read and it may be NULL.
  */
 dsa_status dsa_sparse_attn(const uint16_t *q, const uint16_t *kv, const int32_t *idx,
                            int B, int T, int N, int H, int k, float scale, float *out,
@@ -185,6 +188,59 @@ dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t 
                              int B, int T, int N, long long q_pos0, int H, int k, float scale,
                              int compute_indices, int32_t *idx_shared, float *const *out,
                              void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * A decode step over G IndexShare groups, micro-batched.  Per group: the indexer and the
+ * top-k once, then the attention of L layers with the same index list (T = 1 query per
+ * sequence at the newest cached position, q_pos0 = N - 1), exactly as dsa_group_forward
+ * computes them.  The batch is split into two micro-batches -- sequences [0, ceil(B/2))
+ * and the rest -- whose chains run on two streams: micro-batch 0 on `stream`, 1 on `side`
+ * (a second stream of the caller; its work is joined back into `stream` before the call
+ * returns, so the call completes on `stream` like any other).  Each micro-batch runs its
+ * groups in order (group g+1's indexer after group g's attention, as in a model).  The
+ * HBM-bound indexers of the two micro-batches take turns (each waits for the other's
+ * previous one) on about two thirds of the SMs, and each micro-batch's top-k and
+ * attention run beside the other's indexer on the remaining third.  With B = 1 the groups
+ * run in order on `stream`.
+ *   groups[g]   the group's tensors for all B sequences, in the layouts of
+ *               dsa_group_forward with T = 1 (q, kv, out: L entries each)
+ *   workspace   dsa_decode_workspace_size(B, N, k, H, L) bytes, 256-byte aligned
+ * Uses events created once per device and host thread.
+ */
+typedef struct {
+    const uint16_t *iq, *ik; /* [B, 1, 32, 128] and [B, N, 128] bf16                        */
+    const float *w;          /* [B, 1, 32] f32                                                */
+    const uint16_t *q[DSA_MAX_LAYERS];  /* [B, 1, H, 576] bf16 per layer                     */
+    const uint16_t *kv[DSA_MAX_LAYERS]; /* [B, N, 576] bf16 per layer                        */
+    int32_t *idx;                       /* [B, 1, k] out: the group's index list            */
+    float *out[DSA_MAX_LAYERS];         /* [B, 1, H, 512] f32 per layer                     */
+} dsa_group_io;
+
+size_t dsa_decode_workspace_size(int B, int N, int k, int H, int L);
+dsa_status dsa_decode_step(const dsa_group_io *groups, int G, int L, int B, int N, int H, int k, float scale,
+                           void *workspace, size_t workspace_bytes, cudaStream_t stream, cudaStream_t side);
+
+/*
+ * MTP verify step -- rejection sampling of the draft tokens ("GLM-5.2 MTP IndexShare
+ * inference", Rejection Sampling: the acceptance rate is sum_v min(p_v, q_v); the MTP
+ * pages verify the draft tokens in order and cut the sequence at the first rejection).
+ *   p, q    [B, S, V] f32  target and draft probabilities of each draft position
+ *                          (row b*S + j is position j of sequence b); V < 2^24
+ *   draft   [B, S] i32     the draft tokens
+ *   u, u2   [B, S] f32     uniform numbers in [0, 1): the accept test and the resample
+ *   alpha   [B, S] f32 out the acceptance rate sum_v min(p_v, q_v)
+ *   accept  [B, S] i32 out 1 iff u * q[x] < p[x] (float32), x the draft token
+ *   token   [B, S] i32 out x when accepted, else a draw from max(0, p - q): integer
+ *                          weights floor(max(0, p_v - q_v) * 2^40), target
+ *                          floor(floor(u2 * 2^24) * sum / 2^24), the first token whose
+ *                          inclusive prefix sum exceeds it (x when the residual is empty;
+ *                          -1 for a draft token outside [0, V))
+ *   accepted_len [B] i32 out the leading accepted positions of each sequence
+ * Bit-exact decisions (accept, token, accepted_len); alpha within float32 summation error.
+ */
+dsa_status dsa_verify(const float *p, const float *q, const int32_t *draft, const float *u, const float *u2,
+                      int B, int S, int V, float *alpha, int32_t *accept, int32_t *token, int32_t *accepted_len,
+                      cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -30,7 +30,15 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_topk",
            "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error",
-           "dsa_check_device_status", "dsa_last_cuda_error", "dsa_cuda_error_string")
+           "dsa_check_device_status", "dsa_last_cuda_error", "dsa_cuda_error_string", "dsa_verify",
+           "dsa_decode_workspace_size", "dsa_decode_step")
+
+
+class GroupIO(ctypes.Structure):
+    """dsa_group_io: one IndexShare group's tensors for dsa_decode_step."""
+    _fields_ = [("iq", ctypes.c_void_p), ("ik", ctypes.c_void_p), ("w", ctypes.c_void_p),
+                ("q", ctypes.c_void_p * MAX_LAYERS), ("kv", ctypes.c_void_p * MAX_LAYERS), ("idx", ctypes.c_void_p),
+                ("out", ctypes.c_void_p * MAX_LAYERS)]
 
 
 class DsaError(RuntimeError):
@@ -69,7 +77,13 @@ def lib() -> ctypes.CDLL:
         L.dsa_last_cuda_error.restype = I
         L.dsa_cuda_error_string.argtypes = [I]
         L.dsa_cuda_error_string.restype = ctypes.c_char_p
-        for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc"):
+        L.dsa_verify.argtypes = [P, P, P, P, P, I, I, I, P, P, P, P, P]
+        L.dsa_decode_workspace_size.argtypes = [I, I, I, I, I]
+        L.dsa_decode_workspace_size.restype = S
+        L.dsa_decode_step.argtypes = [P, I, I, I, I, I, I, F, P, S, P, P]
+        L.dsa_decode_step.restype = I
+        for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc",
+                  "dsa_verify"):
             getattr(L, f).restype = I
         _lib = L
     return _lib
@@ -241,3 +255,62 @@ def dsa_topk_noalloc(scores, q_pos0: int, k: int, idx=None, stream=None):
                                 _ptr(idx, (torch.int32,), "idx", (B, T, k)), _stream(stream))
     _check(rc, "dsa_topk_noalloc")
     return idx
+
+
+def dsa_verify(p, q, draft, u, u2, stream=None):
+    """MTP verify step.  p, q [B,S,V] f32 probabilities; draft [B,S] int32; u, u2 [B,S] f32.
+    Returns (alpha [B,S] f32, accept [B,S] int32, token [B,S] int32, accepted_len [B] int32)."""
+    torch = _torch()
+    B, S, V = p.shape
+    dev = p.device
+    alpha = torch.empty((B, S), dtype=torch.float32, device=dev)
+    accept = torch.empty((B, S), dtype=torch.int32, device=dev)
+    token = torch.empty((B, S), dtype=torch.int32, device=dev)
+    alen = torch.empty((B,), dtype=torch.int32, device=dev)
+    rc = lib().dsa_verify(_ptr(p, (torch.float32,), "p", (B, S, V)), _ptr(q, (torch.float32,), "q", (B, S, V)),
+                          _ptr(draft, (torch.int32,), "draft", (B, S)), _ptr(u, (torch.float32,), "u", (B, S)),
+                          _ptr(u2, (torch.float32,), "u2", (B, S)), B, S, V, _ptr(alpha, (torch.float32,), "alpha"),
+                          _ptr(accept, (torch.int32,), "accept"), _ptr(token, (torch.int32,), "token"),
+                          _ptr(alen, (torch.int32,), "accepted_len"), _stream(stream))
+    _check(rc, "dsa_verify")
+    return alpha, accept, token, alen
+
+
+def decode_workspace(B: int, N: int, k: int, H: int, L: int, device=None):
+    """A workspace tensor of dsa_decode_workspace_size bytes (torch allocation)."""
+    torch = _torch()
+    n = int(lib().dsa_decode_workspace_size(B, N, k, H, L))
+    if n == 0:
+        raise ValueError("invalid sizes for dsa_decode_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def dsa_decode_step(groups, k: int, scale: float, ws=None, stream=None, side=None):
+    """A micro-batched decode step over IndexShare groups (see include/dsa.h).  `groups` is
+    a list of dicts with iq, w, ik, qs (L tensors), kvs (L tensors), idx, outs (L tensors);
+    `side` a second CUDA stream (created when None)."""
+    torch = _torch()
+    G = len(groups)
+    L = len(groups[0]["qs"])
+    B, _, H, _ = groups[0]["qs"][0].shape
+    N = groups[0]["kvs"][0].shape[1]
+    if ws is None:
+        ws = decode_workspace(B, N, k, H, L, groups[0]["qs"][0].device)
+    if side is None:
+        side = torch.cuda.Stream(groups[0]["qs"][0].device)
+    arr = (GroupIO * G)()
+    for g, d in enumerate(groups):
+        io = arr[g]
+        io.iq = _ptr(d["iq"], _bf16_types(), "iq", (B, 1, INDEX_HEADS, INDEX_DIM))
+        io.w = _ptr(d["w"], (torch.float32,), "w", (B, 1, INDEX_HEADS))
+        io.ik = _ptr(d["ik"], _bf16_types(), "ik", (B, N, INDEX_DIM))
+        io.idx = _ptr(d["idx"], (torch.int32,), "idx", (B, 1, k))
+        if len(d["qs"]) != L or len(d["kvs"]) != L or len(d["outs"]) != L:
+            raise ValueError("every group needs L queries, caches and outputs")
+        for l in range(L):
+            io.q[l] = _ptr(d["qs"][l], _bf16_types(), "q[l]", (B, 1, H, DQK))
+            io.kv[l] = _ptr(d["kvs"][l], _bf16_types(), "kv[l]", (B, N, DQK))
+            io.out[l] = _ptr(d["outs"][l], (torch.float32,), "out[l]", (B, 1, H, DV))
+    rc = lib().dsa_decode_step(ctypes.addressof(arr), G, L, B, N, H, int(k), float(scale),
+                               _ptr(ws, (torch.uint8,), "workspace"), ws.numel(), _stream(stream), _stream(side))
+    _check(rc, "dsa_decode_step")

@@ -6,6 +6,7 @@
 // steps 2.. reuse the step-1 index list, so draft-token rows are never attended; the MTP
 // layer reads the target cache -- KV Share).
 #include <cstdio>
+#include <vector>
 
 #include "dsa.h"
 #include "dsa_common.cuh"
@@ -68,6 +69,94 @@ GroupLayout group_layout(int B, int T, int N, int k, int H, int L) {
 }
 
 bool heads_supported(int H) { return H == 16 || H == 32 || H == 48 || H == 64; }
+
+// One group call, checked.
+struct GroupCall {
+  const uint16_t* iq;
+  const float* w;
+  const uint16_t* ik;
+  AttnLayers layers;
+  int L, B, T, N, H, k, compute_indices;
+  long long q_pos0;
+  float scale;
+  int32_t* idx;
+};
+
+dsa_status check_group(const uint16_t* iq, const float* w, const uint16_t* ik, const uint16_t* const* q,
+                       const uint16_t* const* kv, int L, int B, int T, int N, int H, int k, int compute_indices,
+                       int32_t* idx_shared, float* const* out, GroupCall* c) {
+  if (!q || !kv || !out || !idx_shared || !sizes_ok(B, T, N) || k <= 0 || H <= 0 || L <= 0)
+    return DSA_ERR_INVALID_ARG;
+  if (L > DSA_MAX_LAYERS || k > DSA_MAX_TOPK || !heads_supported(H)) return DSA_ERR_UNSUPPORTED;
+  if (compute_indices && (!iq || !w || !ik)) return DSA_ERR_INVALID_ARG;
+  if (compute_indices && (!aligned(iq, 16) || !aligned(ik, 16) || !aligned(w, 16))) return DSA_ERR_INVALID_ARG;
+  if (!aligned(idx_shared, 4)) return DSA_ERR_INVALID_ARG;
+  for (int l = 0; l < L; ++l) {
+    if (!q[l] || !kv[l] || !out[l]) return DSA_ERR_INVALID_ARG;
+    if (!aligned(q[l], 16) || !aligned(kv[l], 16) || !aligned(out[l], 16)) return DSA_ERR_INVALID_ARG;
+    c->layers.q[l] = q[l];
+    c->layers.kv[l] = kv[l];
+    c->layers.out[l] = out[l];
+  }
+  c->iq = iq;
+  c->w = w;
+  c->ik = ik;
+  c->L = L;
+  c->B = B;
+  c->T = T;
+  c->N = N;
+  c->H = H;
+  c->k = k;
+  c->compute_indices = compute_indices;
+  c->idx = idx_shared;
+  return DSA_OK;
+}
+
+// Enqueues one group on `stream`: the indexer (after `before`, if given; on at most idx_sms
+// SMs; `after_idx` recorded behind it, if given), then the top-k and the attention (on at
+// most tail_sms SMs).  A budget of 0 means all SMs.
+cudaError_t enqueue_group(const GroupCall& c, unsigned char* base, const GroupLayout& g, int idx_sms, int tail_sms,
+                          cudaEvent_t before, cudaEvent_t after_idx, cudaStream_t stream) {
+  const long long rows = (long long)c.B * c.T;
+  cudaError_t e;
+  if (before && (e = cudaStreamWaitEvent(stream, before, 0)) != cudaSuccess) return e;
+  if (c.compute_indices) {
+    TopkWorkspace tws = topk_workspace(base + g.topk_off, rows, c.N);
+    float* scores = reinterpret_cast<float*>(base + g.scores_off);
+    // in decode the indexer folds the first radix digit of the select into its epilogue
+    const int sms = device_sm_count();
+    if (sms <= 0) return cudaErrorInvalidDevice;
+    const int cap = idx_sms > 0 && idx_sms < sms ? idx_sms : sms;
+    const bool fused_hist = c.T == 1 && c.B <= cap;
+    if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess) return e;
+    if ((e = launch_index_score_tc(c.iq, c.w, c.ik, c.B, c.T, c.N, c.q_pos0, scores, fused_hist ? tws.hist : nullptr,
+                                   idx_sms, stream)) != cudaSuccess)
+      return e;
+    if (after_idx && (e = cudaEventRecord(after_idx, stream)) != cudaSuccess) return e;
+    if ((e = launch_topk(scores, c.B, c.T, c.N, c.q_pos0, c.k, c.idx, tws, fused_hist, tail_sms, stream)) != cudaSuccess)
+      return e;
+  }
+  return launch_sparse_attn_tc(c.layers, c.L, c.idx, c.B, c.T, c.N, c.H, c.k, c.scale, base + g.attn_off, g.attn_bytes,
+                               /*q_early=*/c.compute_indices != 0, tail_sms, stream);
+}
+
+// Events of dsa_decode_step, created once per device and host thread.
+struct DecodeEvents {
+  cudaEvent_t fork = nullptr, join = nullptr, idx[2] = {nullptr, nullptr};
+};
+
+DecodeEvents* decode_events() {
+  thread_local DecodeEvents ev[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  DecodeEvents& d = ev[dev];
+  if (!d.fork) {
+    cudaEvent_t* all[4] = {&d.fork, &d.join, &d.idx[0], &d.idx[1]};
+    for (cudaEvent_t* x : all)
+      if (cudaEventCreateWithFlags(x, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+  }
+  return &d;
+}
 
 // The error words of the indexer, the attention and the top-k, in that order.
 struct ErrorWords {
@@ -148,7 +237,7 @@ dsa_status dsa_index_score(const uint16_t* q, const float* w, const uint16_t* k,
                            long long q_pos0, float* scores, cudaStream_t stream) {
   if (!q || !w || !k || !scores || !sizes_ok(B, T, N)) return DSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 16) || !aligned(scores, 4)) return DSA_ERR_INVALID_ARG;
-  return cuda_status(launch_index_score_tc(q, w, k, B, T, N, q_pos0, scores, nullptr, stream));
+  return cuda_status(launch_index_score_tc(q, w, k, B, T, N, q_pos0, scores, nullptr, 0, stream));
 }
 
 dsa_status dsa_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx, void* workspace,
@@ -160,7 +249,7 @@ dsa_status dsa_topk(const float* scores, int B, int T, int N, long long q_pos0, 
   const size_t need = topk_workspace_bytes(rows, N);
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE;
   TopkWorkspace ws = topk_workspace(workspace, rows, N);
-  return cuda_status(launch_topk(scores, B, T, N, q_pos0, k, idx, ws, false, stream));
+  return cuda_status(launch_topk(scores, B, T, N, q_pos0, k, idx, ws, false, 0, stream));
 }
 
 dsa_status dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int N, int H,
@@ -169,55 +258,115 @@ dsa_status dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const int32_t*
   if (!q || !kv || !idx || !out || !sizes_ok(B, T, N) || k <= 0 || H <= 0) return DSA_ERR_INVALID_ARG;
   if (k > DSA_MAX_TOPK || !heads_supported(H)) return DSA_ERR_UNSUPPORTED;
   if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(idx, 4) || !aligned(out, 16)) return DSA_ERR_INVALID_ARG;
-  (void)workspace_bytes;
+  const size_t need = attn_workspace_bytes((long long)B * T, 1, H, k);
+  if (need && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return DSA_ERR_WORKSPACE;
   AttnLayers layers{};
   layers.q[0] = q;
   layers.kv[0] = kv;
   layers.out[0] = out;
-  return cuda_status(launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, workspace, false, stream));
+  return cuda_status(
+      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, workspace, workspace_bytes, false, 0, stream));
 }
 
 dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t* ik, const uint16_t* const* q,
                              const uint16_t* const* kv, int L, int B, int T, int N, long long q_pos0, int H, int k,
                              float scale, int compute_indices, int32_t* idx_shared, float* const* out, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream) {
-  if (!q || !kv || !out || !idx_shared || !sizes_ok(B, T, N) || k <= 0 || H <= 0 || L <= 0)
-    return DSA_ERR_INVALID_ARG;
-  if (L > DSA_MAX_LAYERS || k > DSA_MAX_TOPK || !heads_supported(H)) return DSA_ERR_UNSUPPORTED;
-  if (compute_indices && (!iq || !w || !ik)) return DSA_ERR_INVALID_ARG;
-  if (compute_indices && (!aligned(iq, 16) || !aligned(ik, 16) || !aligned(w, 16))) return DSA_ERR_INVALID_ARG;
-  if (!aligned(idx_shared, 4)) return DSA_ERR_INVALID_ARG;
-  AttnLayers layers{};
-  for (int l = 0; l < L; ++l) {
-    if (!q[l] || !kv[l] || !out[l]) return DSA_ERR_INVALID_ARG;
-    if (!aligned(q[l], 16) || !aligned(kv[l], 16) || !aligned(out[l], 16)) return DSA_ERR_INVALID_ARG;
-    layers.q[l] = q[l];
-    layers.kv[l] = kv[l];
-    layers.out[l] = out[l];
-  }
+  GroupCall c{};
+  const dsa_status st = check_group(iq, w, ik, q, kv, L, B, T, N, H, k, compute_indices, idx_shared, out, &c);
+  if (st != DSA_OK) return st;
+  c.q_pos0 = q_pos0;
+  c.scale = scale;
   const GroupLayout g = group_layout(B, T, N, k, H, L);
   if (!workspace || workspace_bytes < g.total || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE;
-  unsigned char* base = static_cast<unsigned char*>(workspace);
-  const long long rows = (long long)B * T;
-  cudaError_t e;
-  if (compute_indices) {
-    TopkWorkspace tws = topk_workspace(base + g.topk_off, rows, N);
-    float* scores = reinterpret_cast<float*>(base + g.scores_off);
-    // in decode the indexer folds the first radix digit of the select into its epilogue
-    const int sms = device_sm_count();
-    if (sms <= 0) return cuda_status(cudaErrorInvalidDevice);
-    const bool fused_hist = T == 1 && B <= sms;
-    if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess)
-      return cuda_status(e);
-    if ((e = launch_index_score_tc(iq, w, ik, B, T, N, q_pos0, scores, fused_hist ? tws.hist : nullptr, stream)) !=
-        cudaSuccess)
-      return cuda_status(e);
-    if ((e = launch_topk(scores, B, T, N, q_pos0, k, idx_shared, tws, fused_hist, stream)) != cudaSuccess)
-      return cuda_status(e);
+  return cuda_status(enqueue_group(c, static_cast<unsigned char*>(workspace), g, 0, 0, nullptr, nullptr, stream));
+}
+
+size_t dsa_decode_workspace_size(int B, int N, int k, int H, int L) {
+  if (!sizes_ok(B, 1, N) || k <= 0 || k > DSA_MAX_TOPK || H <= 0 || L <= 0 || L > DSA_MAX_LAYERS) return 0;
+  const int B0 = (B + 1) / 2, B1 = B - B0;
+  size_t n = round256(group_layout(B0, 1, N, k, H, L).total);
+  if (B1 > 0) n += group_layout(B1, 1, N, k, H, L).total;
+  return n;
+}
+
+dsa_status dsa_decode_step(const dsa_group_io* groups, int G, int L, int B, int N, int H, int k, float scale,
+                           void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaStream_t side) {
+  if (!groups || G <= 0 || !sizes_ok(B, 1, N)) return DSA_ERR_INVALID_ARG;
+  const int B0 = (B + 1) / 2, B1 = B - B0;
+  const GroupLayout g0 = group_layout(B0, 1, N, k, H, L);
+  const GroupLayout g1 = group_layout(B1 > 0 ? B1 : 1, 1, N, k, H, L);
+  const size_t off1 = round256(g0.total);
+  const size_t need = B1 > 0 ? off1 + g1.total : g0.total;
+  // every group's arguments are checked before anything is enqueued
+  std::vector<GroupCall> calls((size_t)G * 2);
+  for (int gi = 0; gi < G; ++gi) {
+    const dsa_group_io& io = groups[gi];
+    for (int mb = 0; mb < 2; ++mb) {
+      const int b0 = mb ? B0 : 0, bn = mb ? B1 : B0;
+      GroupCall& c = calls[(size_t)gi * 2 + mb];
+      if (bn == 0) continue;
+      const uint16_t* qs[DSA_MAX_LAYERS];
+      const uint16_t* kvs[DSA_MAX_LAYERS];
+      float* outs[DSA_MAX_LAYERS];
+      if (L <= 0 || L > DSA_MAX_LAYERS) return L <= 0 ? DSA_ERR_INVALID_ARG : DSA_ERR_UNSUPPORTED;
+      for (int l = 0; l < L; ++l) {
+        if (!io.q[l] || !io.kv[l] || !io.out[l]) return DSA_ERR_INVALID_ARG;
+        qs[l] = io.q[l] + (size_t)b0 * H * kDqk;
+        kvs[l] = io.kv[l] + (size_t)b0 * N * kDqk;
+        outs[l] = io.out[l] + (size_t)b0 * H * kDv;
+      }
+      if (!io.iq || !io.w || !io.ik || !io.idx) return DSA_ERR_INVALID_ARG;
+      const dsa_status st = check_group(io.iq + (size_t)b0 * kIndexHeads * kIndexDim, io.w + (size_t)b0 * kIndexHeads,
+                                        io.ik + (size_t)b0 * N * kIndexDim, qs, kvs, L, bn, 1, N, H, k, 1,
+                                        io.idx + (size_t)b0 * k, outs, &c);
+      if (st != DSA_OK) return st;
+      c.q_pos0 = N - 1;
+      c.scale = scale;
+    }
   }
-  e = launch_sparse_attn_tc(layers, L, idx_shared, B, T, N, H, k, scale, base + g.attn_off,
-                            /*q_early=*/compute_indices != 0, stream);
-  return cuda_status(e);
+  if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE;
+  unsigned char* base = static_cast<unsigned char*>(workspace);
+  cudaError_t e;
+  if (B1 == 0) {  // one sequence: nothing to overlap
+    for (int gi = 0; gi < G; ++gi)
+      if ((e = enqueue_group(calls[(size_t)gi * 2], base, g0, 0, 0, nullptr, nullptr, stream)) != cudaSuccess)
+        return cuda_status(e);
+    return DSA_OK;
+  }
+  const int sms = device_sm_count();
+  if (sms <= 0) return cuda_status(cudaErrorInvalidDevice);
+  // The indexer saturates HBM with about two thirds of the SMs; the other micro-batch's
+  // top-k and attention run beside it on the rest.
+  const int tail_sms = sms / 3, idx_sms = sms - tail_sms;
+  DecodeEvents* ev = decode_events();
+  if (!ev) return cuda_status(cudaErrorInvalidDevice);
+  if ((e = cudaEventRecord(ev->fork, stream)) != cudaSuccess || (e = cudaStreamWaitEvent(side, ev->fork, 0)) != cudaSuccess)
+    return cuda_status(e);
+  for (int gi = 0; gi < G; ++gi) {
+    for (int mb = 0; mb < 2; ++mb) {
+      const bool first = gi == 0 && mb == 0, last = gi == G - 1 && mb == 1;
+      // indexers alternate (each waits for the previous one); the first runs alone, and
+      // the last micro-batch's last top-k and attention run alone
+      e = enqueue_group(calls[(size_t)gi * 2 + mb], base + (mb ? off1 : 0), mb ? g1 : g0, first ? sms : idx_sms,
+                        last ? sms : tail_sms, first ? nullptr : ev->idx[1 - mb], ev->idx[mb], mb ? side : stream);
+      if (e != cudaSuccess) return cuda_status(e);
+    }
+  }
+  if ((e = cudaEventRecord(ev->join, side)) != cudaSuccess || (e = cudaStreamWaitEvent(stream, ev->join, 0)) != cudaSuccess)
+    return cuda_status(e);
+  return DSA_OK;
+}
+
+dsa_status dsa_verify(const float* p, const float* q, const int32_t* draft, const float* u, const float* u2, int B,
+                      int S, int V, float* alpha, int32_t* accept, int32_t* token, int32_t* accepted_len,
+                      cudaStream_t stream) {
+  if (!p || !q || !draft || !u || !u2 || !alpha || !accept || !token || !accepted_len) return DSA_ERR_INVALID_ARG;
+  if (B <= 0 || S <= 0 || V <= 0 || V >= (1 << 24) || (long long)B * S > 0x7FFFFFFFLL) return DSA_ERR_INVALID_ARG;
+  if (!aligned(p, 4) || !aligned(q, 4) || !aligned(alpha, 4) || !aligned(draft, 4) || !aligned(u, 4) ||
+      !aligned(u2, 4) || !aligned(accept, 4) || !aligned(token, 4) || !aligned(accepted_len, 4))
+    return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_verify(p, q, draft, u, u2, B, S, V, alpha, accept, token, accepted_len, stream));
 }
 
 }  // extern "C"

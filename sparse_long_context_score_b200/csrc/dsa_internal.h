@@ -78,6 +78,7 @@ struct TopkWorkspace {
   uint32_t* row_state;   // [rows][kRowStateWords]
   uint32_t* chunk_sel;   // [rows][nchunks]  selected threshold-bin candidates per chunk
   uint32_t* hist2;       // [rows][kHist2Bins] next 10 key bits of the threshold-bin elements
+  uint32_t* lvl;         // [rows][2][kHist2Bins] more digit histograms (one-launch select of long rows)
   uint32_t* chunk_above; // [rows][nchunks]  elements above the threshold bin per chunk
   uint32_t* chunk_off;   // [rows][nchunks]  output offset of each chunk
   uint64_t* cand;        // [rows][kCandCap] composite keys of threshold-bin elements
@@ -93,21 +94,26 @@ struct AttnLayers {
   float* out[kMaxLayers];
 };
 
-constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core attention
+constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core attention (a split's granularity)
 
 int attn_num_splits(long long rows, int L, int k, int sm_budget, const int* cluster_fit);
 int attn_split_chunk(int k, int nsplit);
-size_t attn_workspace_bytes(long long rows, int L, int H, int k);
+size_t attn_workspace_bytes(long long rows, int L, int H, int k, int sm_budget = 0);
 
 // tcgen05 indexer (T == 1: decode, one query per MMA; T > 1: 8 queries per MMA).  With a
 // histogram pointer (decode only, B <= 148) the first radix digit of the select is counted.
 cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
-                                  long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream);
+                                  long long q_pos0, float* scores, uint32_t* hist, int sm_budget, cudaStream_t stream);
 // Device addresses of the error words: the indexer's and the attention's bounded waits
 // record a code when they run out; the top-k records one when a selection invariant
 // fails (the selected count is not k).  0 = none.
 cudaError_t indexer_error_word(int** p);
 cudaError_t attn_error_word(int** p);
+
+// MTP verify step (verify.cu)
+cudaError_t launch_verify(const float* p, const float* q, const int32_t* draft, const float* u, const float* u2, int B,
+                          int S, int V, float* alpha, int32_t* accept, int32_t* token, int32_t* accepted_len,
+                          cudaStream_t stream);
 cudaError_t topk_error_word(int** p);
 
 // Whether launch_topk takes the scan kernels for this shape (and so reads and writes the
@@ -115,7 +121,7 @@ cudaError_t topk_error_word(int** p);
 bool topk_uses_workspace(long long rows, long long vmax);
 
 cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
-                        const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream);
+                        const TopkWorkspace& ws, bool hist_ready, int sm_budget, cudaStream_t stream);
 // top-k of rows short enough for one cluster of CTAs (topk_cluster.cu); launch_topk
 // chooses it when topk_cluster_plan accepts the shape.  `hist` (nullable) holds the
 // first digit's histogram per row, counted by the indexer.
@@ -126,6 +132,7 @@ cudaError_t launch_topk_cluster(const float* scores, int B, int T, int N, long l
 // q_early: the kernel before it in the stream does not write the queries (it is the
 // group's own top-k), so they are loaded before that kernel completes
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                                  int k, float scale, void* ws, bool q_early, cudaStream_t stream);
+                                  int k, float scale, void* ws, size_t ws_bytes, bool q_early, int sm_budget,
+                                  cudaStream_t stream);
 
 }  // namespace dsa

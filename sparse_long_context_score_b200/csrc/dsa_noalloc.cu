@@ -62,6 +62,6 @@ extern "C" dsa_status dsa_topk_noalloc(const float* scores, int B, int T, int N,
   const cudaError_t ea = g_scratch_address.get(&scratch);
   if (ea != cudaSuccess) return dsa::cuda_status(ea);
   dsa::TopkWorkspace ws = dsa::topk_workspace(scratch, rows, N);
-  const cudaError_t e = dsa::launch_topk(scores, B, T, N, q_pos0, k, idx, ws, false, stream);
+  const cudaError_t e = dsa::launch_topk(scores, B, T, N, q_pos0, k, idx, ws, false, 0, stream);
   return dsa::cuda_status(e);
 }

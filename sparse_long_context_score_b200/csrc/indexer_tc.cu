@@ -393,7 +393,7 @@ SymbolAddress g_err_addr;
 
 template <int QG, bool kHist>
 cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N, long long q_pos0,
-                      float* scores, uint32_t* hist, cudaStream_t stream) {
+                      float* scores, uint32_t* hist, int sm_budget, cudaStream_t stream) {
   using C = TcCfg<QG, kHist>;
   CUtensorMap kmap, qmap;
   if (!make_map(&kmap, k, N, B, kTileKeys) || !make_map(&qmap, q, (long long)T * 32, B, C::kN))
@@ -416,9 +416,11 @@ cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int 
     total += (v + kTileKeys - 1) / kTileKeys;
   }
   if (total == 0) return cudaSuccess;
+  // persistent: one CTA per SM of the budget (all SMs by default)
   const int sms = device_sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
-  const int grid = (int)(total < sms ? total : sms);
+  const int cap = sm_budget > 0 && sm_budget < sms ? sm_budget : sms;
+  const int grid = (int)(total < cap ? total : cap);
   indexer_tc_kernel<QG, kHist><<<grid, C::kThreads, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
                                                                        hist, err);
   return cudaGetLastError();
@@ -427,15 +429,19 @@ cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int 
 }  // namespace
 
 cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
-                                  long long q_pos0, float* scores, uint32_t* hist, cudaStream_t stream) {
-  // the fused histogram keeps two row slots per CTA: with contiguous item ranges over
-  // at most one CTA per SM a range spans at most two sequences when B <= the SM count
-  if (hist && (T != 1 || B > device_sm_count())) return cudaErrorNotSupported;
+                                  long long q_pos0, float* scores, uint32_t* hist, int sm_budget,
+                                  cudaStream_t stream) {
+  // the fused histogram keeps two row slots per CTA: with contiguous item ranges over at
+  // most one CTA per SM of the budget, a range spans at most two sequences when B is no
+  // more than the CTAs
+  const int sms = device_sm_count();
+  const int cap = sm_budget > 0 && sm_budget < sms ? sm_budget : sms;
+  if (hist && (T != 1 || B > cap)) return cudaErrorNotSupported;
   if (T == 1) {
-    return hist ? launch_tc<1, true>(q, w, k, B, T, N, q_pos0, scores, hist, stream)
-                : launch_tc<1, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, stream);
+    return hist ? launch_tc<1, true>(q, w, k, B, T, N, q_pos0, scores, hist, sm_budget, stream)
+                : launch_tc<1, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
   }
-  return launch_tc<8, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, stream);
+  return launch_tc<8, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
 }
 
 cudaError_t indexer_error_word(int** p) { return g_err_addr.get(g_indexer_tc_error, p); }

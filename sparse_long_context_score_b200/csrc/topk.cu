@@ -31,6 +31,7 @@
 // row is padded with -1.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
+#include "sm100.cuh"
 
 namespace dsa {
 
@@ -501,6 +502,257 @@ topk_compact_kernel(const float* __restrict__ scores, int T, int N, long long q_
   }
 }
 
+// ---------------------------------------------------------------------------- long rows
+// One launch for rows longer than a cluster holds (a 1M-token decode row), when all the
+// CTAs of the launch fit the GPU at once (a cooperative launch checks it): CTA (chunk, row)
+// keeps its 8192 order keys in shared memory, and the CTAs of a row meet at row barriers
+// (a counter in the workspace, bounded spins) to refine the threshold digit by digit -- the
+// first 12 bits from the row's histogram, then 10 bits at a time -- until the threshold
+// bin holds at most kLongCap elements.  Those are appended to the row's candidate list,
+// with every chunk's count above the bin; after one more row barrier every CTA ranks the
+// candidates itself, takes the output offset of its chunk from the counts and writes its
+// positions in order.  No CTA re-reads the scores from memory.
+constexpr int kLongCap = 4096;             // threshold-bin elements ranked in shared memory
+constexpr int kLongLevels = 6;             // digit widths after the first: 10,10,10,10,10,2
+constexpr int RS_SYNC0 = 6;                // row_state words 6.. : row barrier counters
+constexpr int kLongMaxChunks = 512;        // rows of up to 4M positions
+
+// ~50 KB, so that four CTAs share an SM (the candidates are read from L2)
+struct LongSmem {
+  uint32_t keys[kTopkChunk];
+  uint32_t radix[kHistBins];               // digit histograms (the first digit's too)
+  uint32_t chunk_ge[kLongMaxChunks];
+  uint32_t warp_tmp[32];
+  uint32_t total;
+  uint32_t digit, digit_above, digit_count, cand_base;
+};
+
+__device__ __forceinline__ uint32_t ld_acquire_gpu(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Every CTA of the row arrives, then waits (bounded) until all `n` have: writes before it
+// are visible to every CTA of the row after it.  Returns false after recording `code` when
+// the wait ran out.
+__device__ bool row_barrier(uint32_t* counter, uint32_t n, int* err, int code) {
+  __syncthreads();
+  __shared__ int ok_s;
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(counter, 1u);
+    int ok = 1;
+    const long long t0 = clock64();
+    while (ld_acquire_gpu(counter) < n) {
+      __nanosleep(64);
+      if (clock64() - t0 > sm100::kWaitLimitCycles) {
+        atomicCAS(err, 0, code);
+        ok = 0;
+        break;
+      }
+    }
+    __threadfence();
+    ok_s = ok;
+  }
+  __syncthreads();
+  return ok_s != 0;
+}
+
+// The LongSmem flavour of the block-wide digit search: sm.digit etc. (bins <= 8 x 512).
+template <class Load>
+__device__ __forceinline__ void find_digit_l(LongSmem& sm, int bins, uint32_t r, Load load) {
+  const int per = bins > kSelThreads ? bins / kSelThreads : 1;
+  const int hi = bins - (int)threadIdx.x * per;
+  uint32_t local[8];
+  uint32_t lsum = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int b = hi - 1 - i;
+    local[i] = (i < per && b >= 0) ? load(b) : 0u;
+    lsum += local[i];
+  }
+  if (threadIdx.x == 0) {
+    sm.digit = 0;
+    sm.digit_above = 0;
+    sm.digit_count = 0;
+  }
+  const uint32_t above = block_excl_scan(lsum, sm.warp_tmp, &sm.total);
+  uint32_t run = above;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i < per && hi - 1 - i >= 0 && run < r && run + local[i] >= r) {
+      sm.digit = (uint32_t)(hi - 1 - i);
+      sm.digit_above = run;
+      sm.digit_count = local[i];
+    }
+    run += local[i];
+  }
+  __syncthreads();
+}
+
+__global__ void __launch_bounds__(kSelThreads)
+topk_long_kernel(const float* __restrict__ scores, int T, int N, long long q_pos0, int k, TopkWorkspace ws,
+                 int hist_ready, int32_t* __restrict__ idx_out, int* __restrict__ err) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  LongSmem& sm = *reinterpret_cast<LongSmem*>(smem_raw);
+  const int chunk = blockIdx.x, row = blockIdx.y, nchunks = gridDim.x;
+  const long long V = visible_count(N, q_pos0, row_t(row, T));
+  const long long s0 = (long long)chunk * kTopkChunk;
+  const int n = (int)max(0LL, min((long long)kTopkChunk, V - s0));  // this chunk's visible positions
+  int32_t* out = idx_out + (size_t)row * k;
+  if (V <= k) {
+    // every visible position is kept; the rest of the row is padding (the same in every CTA
+    // of the row, so none of them waits at a row barrier)
+    for (int i = threadIdx.x; i < n; i += kSelThreads) out[s0 + i] = (int32_t)(s0 + i);
+    if (chunk == 0)
+      for (long long j = V + threadIdx.x; j < k; j += kSelThreads) out[j] = -1;
+    return;
+  }
+  uint32_t* state = ws.row_state + (size_t)row * kRowStateWords;
+  uint32_t* hist = ws.hist + (size_t)row * kHistBins;
+  const float* sr = scores + (size_t)row * N + s0;
+  for (int i = threadIdx.x; i < kTopkChunk; i += kSelThreads) sm.keys[i] = i < n ? order_key(__ldcg(sr + i)) : 0u;
+  auto comp = [&](int i) -> uint64_t { return composite(sm.keys[i], (uint32_t)(s0 + i)); };
+  int sync = 0;
+  bool ok = true;
+  if (!hist_ready) {
+    // the first digit's histogram of the row (the indexer counts it in decode)
+    for (int i = threadIdx.x; i < kHistBins; i += kSelThreads) sm.radix[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kSelThreads) atomicAdd(&sm.radix[sm.keys[i] >> kHistShift], 1u);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kHistBins; i += kSelThreads)
+      if (sm.radix[i]) atomicAdd(&hist[i], sm.radix[i]);
+    ok = row_barrier(&state[RS_SYNC0 + sync++], nchunks, err, 45);
+  }
+  // first digit: the bin where the count from the top reaches k
+  find_digit_l(sm, kHistBins, (uint32_t)k, [&](int b) { return __ldcg(&hist[b]); });
+  uint64_t prefix = (uint64_t)sm.digit << 52;
+  int pos = 52;                          // bits [pos, 64) of the threshold are fixed
+  uint32_t r = (uint32_t)k - sm.digit_above;
+  uint32_t cnt = sm.digit_count;
+  // further digits while the bin is too large to rank in shared memory
+  for (int level = 0; ok && cnt > (uint32_t)kLongCap && pos > 0 && level < kLongLevels; ++level) {
+    const int width = level < 5 ? 10 : 2;
+    const int shift = pos - width;
+    const uint32_t mask = (1u << width) - 1u;
+    uint32_t* buf = level % 3 == 0 ? ws.hist2 + (size_t)row * kHist2Bins
+                                   : ws.lvl + ((size_t)row * 2 + (level % 3 - 1)) * kHist2Bins;
+    for (int i = threadIdx.x; i < kHist2Bins; i += kSelThreads) sm.radix[i] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kSelThreads) {
+      const uint64_t c = comp(i);
+      if ((c >> pos) == (prefix >> pos)) atomicAdd(&sm.radix[(uint32_t)(c >> shift) & mask], 1u);
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i <= (int)mask; i += kSelThreads)
+      if (sm.radix[i]) atomicAdd(&buf[i], sm.radix[i]);
+    // the buffer of level + 1 (last read two levels ago, before the previous barrier):
+    // this CTA's share of it back to zero
+    if (level >= 2) {
+      uint32_t* nb = (level + 1) % 3 == 0 ? ws.hist2 + (size_t)row * kHist2Bins
+                                          : ws.lvl + ((size_t)row * 2 + ((level + 1) % 3 - 1)) * kHist2Bins;
+      const int per = (kHist2Bins + nchunks - 1) / nchunks;
+      for (int i = chunk * per + (int)threadIdx.x; i < min(kHist2Bins, (chunk + 1) * per); i += kSelThreads) nb[i] = 0u;
+    }
+    ok = row_barrier(&state[RS_SYNC0 + sync++], nchunks, err, 45);
+    find_digit_l(sm, (int)mask + 1, r, [&](int b) { return __ldcg(&buf[b]); });
+    r -= sm.digit_above;
+    prefix |= (uint64_t)sm.digit << shift;
+    pos = shift;
+    cnt = sm.digit_count;
+  }
+  // this chunk's elements above the threshold bin, and its elements in it (the candidates)
+  uint32_t n_above = 0, n_in = 0;
+  for (int i = threadIdx.x; i < n; i += kSelThreads) {
+    const uint64_t hi = comp(i) >> pos, ph = prefix >> pos;
+    n_above += hi > ph ? 1u : 0u;
+    n_in += hi == ph ? 1u : 0u;
+  }
+  (void)block_excl_scan(n_above, sm.warp_tmp, &sm.total);
+  if (threadIdx.x == 0) ws.chunk_above[(size_t)row * nchunks + chunk] = sm.total;
+  const uint32_t off = block_excl_scan(n_in, sm.warp_tmp, &sm.total);
+  if (threadIdx.x == 0) sm.cand_base = sm.total ? atomicAdd(&state[RS_CAND], sm.total) : 0u;
+  __syncthreads();
+  {
+    uint64_t* cand = ws.cand + (size_t)row * kCandCap;
+    uint32_t at = sm.cand_base + off;
+    for (int i = threadIdx.x; i < n; i += kSelThreads) {
+      const uint64_t c = comp(i);
+      if ((c >> pos) == (prefix >> pos)) {
+        if (at < (uint32_t)kCandCap) cand[at] = c;
+        ++at;
+      }
+    }
+  }
+  ok = ok && row_barrier(&state[RS_SYNC0 + kLongLevels + 1], nchunks, err, 45);
+  if (!ok) return;
+  // every CTA ranks the candidates (at most kLongCap, read from L2) on their bits below `pos`
+  const uint32_t M = min(cnt, (uint32_t)kLongCap);
+  const uint64_t* cand = ws.cand + (size_t)row * kCandCap;
+  uint64_t thr = prefix;
+  if (cnt != r) {
+    int ps = pos;
+    uint64_t p2 = prefix;
+#pragma unroll 1
+    while (ps > 0) {
+      const int width = ps >= 11 ? 11 : ps;
+      const int shift = ps - width;
+      const uint32_t mask = (1u << width) - 1u;
+      for (int i = threadIdx.x; i <= (int)mask; i += kSelThreads) sm.radix[i] = 0u;
+      __syncthreads();
+      for (uint32_t i = threadIdx.x; i < M; i += kSelThreads) {
+        const uint64_t c = __ldcg(&cand[i]);
+        if ((c >> ps) == (p2 >> ps)) atomicAdd(&sm.radix[(uint32_t)(c >> shift) & mask], 1u);
+      }
+      __syncthreads();
+      find_digit_l(sm, (int)mask + 1, r, [&](int b) { return sm.radix[b]; });
+      r -= sm.digit_above;
+      p2 |= (uint64_t)sm.digit << shift;
+      ps = shift;
+      const bool done = sm.digit_count == r;  // every element of this digit is selected
+      __syncthreads();
+      if (done) break;
+    }
+    thr = p2;
+  }
+  // selected = composite >= thr.  Output offset of this chunk: the selected elements of the
+  // chunks before it (those above the bin, counted by each chunk, and the candidates >= thr)
+  for (int i = threadIdx.x; i < nchunks; i += kSelThreads) sm.chunk_ge[i] = 0u;
+  __syncthreads();
+  for (uint32_t i = threadIdx.x; i < M; i += kSelThreads) {
+    const uint64_t c = __ldcg(&cand[i]);
+    if (c >= thr) atomicAdd(&sm.chunk_ge[(0xFFFFFFFFu - (uint32_t)c) / kTopkChunk], 1u);
+  }
+  __syncthreads();
+  uint32_t before = 0, all = 0;
+  for (int c = threadIdx.x; c < nchunks; c += kSelThreads) {
+    const uint32_t v = __ldcg(&ws.chunk_above[(size_t)row * nchunks + c]) + sm.chunk_ge[c];
+    if (c < chunk) before += v;
+    all += v;
+  }
+  (void)block_excl_scan(before, sm.warp_tmp, &sm.total);
+  const uint32_t base = sm.total;
+  (void)block_excl_scan(all, sm.warp_tmp, &sm.total);
+  if (chunk == 0 && threadIdx.x == 0 && sm.total != (uint32_t)k) atomicCAS(err, 0, 44);
+  // this chunk's selected positions in ascending order: 16 per thread, consecutive
+  constexpr int kPer = kTopkChunk / kSelThreads;
+  uint32_t bits = 0;
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) {
+    const int i = (int)threadIdx.x * kPer + j;
+    if (i < n && comp(i) >= thr) bits |= 1u << j;
+  }
+  uint32_t at = base + block_excl_scan((uint32_t)__popc(bits), sm.warp_tmp, &sm.total);
+#pragma unroll
+  for (int j = 0; j < kPer; ++j)
+    if (bits & (1u << j)) {
+      if (at < (uint32_t)k) out[at] = (int32_t)(s0 + (int)threadIdx.x * kPer + j);
+      ++at;
+    }
+}
+
 }  // namespace
 
 cudaError_t topk_error_word(int** p) { return g_topk_err_addr.get(g_topk_error, p); }
@@ -511,7 +763,7 @@ size_t topk_workspace_bytes(long long rows, int N) {
   b += (size_t)rows * kHistBins * 4;
   b += (size_t)rows * kRowStateWords * 4;
   b += (size_t)rows * nchunks * 4 * 3;
-  b += (size_t)rows * kHist2Bins * 4;
+  b += (size_t)rows * kHist2Bins * 4 * 3;
   b = (b + 255) & ~(size_t)255;
   b += (size_t)rows * kCandCap * 8;
   return (b + 255) & ~(size_t)255;
@@ -529,6 +781,8 @@ TopkWorkspace topk_workspace(void* base, long long rows, int N) {
   p += (size_t)rows * nchunks * 4;
   w.hist2 = reinterpret_cast<uint32_t*>(p);
   p += (size_t)rows * kHist2Bins * 4;
+  w.lvl = reinterpret_cast<uint32_t*>(p);
+  p += (size_t)rows * kHist2Bins * 4 * 2;
   w.zero_bytes = (size_t)(p - static_cast<unsigned char*>(base));
   w.chunk_above = reinterpret_cast<uint32_t*>(p);
   p += (size_t)rows * nchunks * 4;
@@ -540,13 +794,35 @@ TopkWorkspace topk_workspace(void* base, long long rows, int N) {
   return w;
 }
 
+namespace {
+// CTAs of topk_long_kernel that one SM holds (0 if unknown), per device
+int long_per_sm() {
+  static std::atomic<int> cap[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
+  int c = cap[dev].load(std::memory_order_relaxed);
+  if (c > 0) return c;
+  const int smem = (int)sizeof(LongSmem);
+  if (cudaFuncSetAttribute(topk_long_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return 0;
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, topk_long_kernel, kSelThreads, smem) != cudaSuccess) return 0;
+  cap[dev].store(per_sm, std::memory_order_relaxed);
+  return per_sm;
+}
+
+int budget_sms(int sm_budget) {
+  const int sms = device_sm_count();
+  return sm_budget > 0 && sm_budget < sms ? sm_budget : sms;
+}
+}  // namespace
+
 bool topk_uses_workspace(long long rows, long long vmax) {
   int C = 0, kpt = 0;
-  return !topk_cluster_plan(rows, vmax, device_sm_count(), &C, &kpt);
+  return !topk_cluster_plan(rows, vmax, budget_sms(0), &C, &kpt);
 }
 
 cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx,
-                        const TopkWorkspace& ws, bool hist_ready, cudaStream_t stream) {
+                        const TopkWorkspace& ws, bool hist_ready, int sm_budget, cudaStream_t stream) {
   const long long rows = (long long)B * T;
   const long long vmax = visible_count(N, q_pos0, T - 1);
   const long long nchunks_all = ((long long)N + kTopkChunk - 1) / kTopkChunk;
@@ -554,8 +830,24 @@ cudaError_t launch_topk(const float* scores, int B, int T, int N, long long q_po
   int C = 0, kpt = 0;
   int* err = nullptr;
   if ((e = g_topk_err_addr.get(g_topk_error, &err)) != cudaSuccess) return e;
-  if (topk_cluster_plan(rows, vmax, device_sm_count(), &C, &kpt))
+  const int sms = budget_sms(sm_budget);
+  if (topk_cluster_plan(rows, vmax, sms, &C, &kpt))
     return launch_topk_cluster(scores, B, T, N, q_pos0, k, C, kpt, hist_ready ? ws.hist : nullptr, idx, err, stream);
+  // long rows, all of whose CTAs fit the GPU at once: one cooperative launch
+  if (nchunks_all <= kLongMaxChunks && rows * nchunks_all <= (long long)long_per_sm() * sms) {
+    if (!hist_ready && (e = cudaMemsetAsync(ws.hist, 0, ws.zero_bytes, stream)) != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)nchunks_all, (unsigned)rows, 1);
+    cfg.blockDim = dim3(kSelThreads);
+    cfg.dynamicSmemBytes = sizeof(LongSmem);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, topk_long_kernel, scores, T, N, q_pos0, k, ws, hist_ready ? 1 : 0, idx, err);
+  }
   if (!hist_ready) {
     e = cudaMemsetAsync(ws.hist, 0, ws.zero_bytes, stream);
     if (e != cudaSuccess) return e;

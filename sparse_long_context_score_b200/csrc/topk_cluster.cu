@@ -16,13 +16,20 @@
 //     bin b*: the bin where the count from the top reaches k.  From then on a thread only
 //     looks at its elements with bin >= b* (a bit mask in a register): the selected
 //     elements are among them;
-//   - later digits: each CTA histograms the digit of its elements that still match the
-//     prefix and adds the non-empty bins into the bin's owner CTA (remote reductions into
-//     shared memory); one cluster barrier later every CTA reads the sums it needs;
-//   - the digits stop once every element of the bin is needed (at the latest when the
-//     64 bits are fixed: composites are distinct); the threshold is then the prefix;
-//   - every CTA sends its selected count to every peer, takes the counts of the lower
-//     ranks as its output offset and writes its positions in order (warp ballots).
+//   - merge path, when b* holds at most kMergeCap elements of the row: every CTA compacts
+//     its elements of b* (as composites) into a list in its shared memory; after one
+//     cluster barrier every CTA copies all the lists through distributed shared memory and
+//     selects the needed rank among them on its own (radix digits over the low 52 bits,
+//     shared-memory histograms, CTA barriers only), which gives the threshold and every
+//     rank's selected count without another exchange;
+//   - digit path, otherwise: each CTA histograms the next digit of its elements that still
+//     match the prefix and adds the non-empty bins into the bin's owner CTA (remote
+//     reductions into shared memory); one cluster barrier later every CTA reads the sums it
+//     needs; the digits stop once every element of the bin is needed (at the latest when
+//     the 64 bits are fixed: composites are distinct); the threshold is then the prefix,
+//     and every CTA sends its selected count to every peer;
+//   - every CTA takes the selected counts of the lower ranks as its output offset and
+//     writes its positions in order (warp ballots).
 // No global workspace, no atomics on global memory and a single launch.  Every thread
 // passes every cluster barrier: the control flow depends only on cluster-wide sums, and
 // no CTA touches another's shared memory after the last barrier.
@@ -43,16 +50,34 @@ constexpr int kMaxC = 8;
 constexpr int kLevels = 6;
 __constant__ int kDigitWidth[kLevels] = {12, 10, 10, 11, 11, 10};
 
+constexpr int kMergeCap = 4096;        // threshold-bin elements the merge path gathers
+
 struct ClusterSmem {
-  uint32_t h[kMaxBins];                   // first digit counted here: this CTA's histogram
-  uint32_t part[kMaxBins];                // ... the cluster sums of the bins this CTA owns
-  uint32_t full0[kMaxBins];               // ... the cluster sums of every bin
-  uint32_t hl[2048];                      // this CTA's histogram of a later digit
-  uint32_t fullb[3][2048];                // cluster sums of the later-digit bins this CTA owns
+  // The digit-by-digit path uses `d`; the merge path reuses the same 64 KB for its candidate
+  // lists.  The path is chosen from the cluster-wide count of the threshold bin, so every
+  // CTA of a cluster takes the same one.
+  union {
+    struct {
+      uint32_t h[kMaxBins];               // first digit counted here: this CTA's histogram
+      uint32_t full0[kMaxBins];           // ... the cluster sums of every bin
+      uint32_t hl[2048];                  // this CTA's histogram of a later digit
+      uint32_t fullb[3][2048];            // cluster sums of the later-digit bins this CTA owns
+    } d;
+    struct {
+      unsigned long long loc[kMergeCap];  // this CTA's threshold-bin composites (peers read them)
+      unsigned long long mrg[kMergeCap];  // every CTA's, in rank order
+    } m;
+  };
+  uint32_t part[kMaxBins];                // first-digit sums of the bins this CTA owns (peers read
+                                          // them); later the merge path's select histogram
   uint32_t nsel[kMaxC];                   // selected counts per sending rank
   uint32_t warp_tmp[kCWarps];
   uint32_t res[3];                        // digit search: digit, above, count
+  uint32_t n_loc, n_above;                // merge path: this CTA's candidates and elements above
+  uint32_t q_cnt[kMaxC], q_above[kMaxC], q_ge[kMaxC];  // merge path: the same per rank
 };
+static_assert(sizeof(unsigned long long) * 2 * kMergeCap <= sizeof(uint32_t) * (2 * kMaxBins + 4 * 2048),
+              "the merge lists fit the digit path's arrays");
 
 // the keys follow the struct, 16-byte aligned (they are written as uint4)
 constexpr int kKeysOff = ((int)sizeof(ClusterSmem) + 127) & ~127;
@@ -99,13 +124,38 @@ __device__ __forceinline__ void digit_search(const uint32_t (&v)[4], int per, in
   count = sm.res[2];
 }
 
+// Exclusive prefix sum of one value per thread over the CTA (kCT threads); *total gets the
+// sum.  Two barriers; warp_tmp is free again on return.
+__device__ __forceinline__ uint32_t cta_excl_scan(uint32_t v, ClusterSmem& sm, uint32_t& total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) sm.warp_tmp[warp] = x;
+  __syncthreads();
+  const uint32_t wt = sm.warp_tmp[lane];
+  uint32_t z = wt;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, z, o);
+    if (lane >= o) z += y;
+  }
+  total = __shfl_sync(0xFFFFFFFFu, z, 31);
+  const uint32_t r = __shfl_sync(0xFFFFFFFFu, z - wt, warp) + x - v;
+  __syncthreads();
+  return r;
+}
+
 // First digit counted by the CTAs: cluster-wide sum of every CTA's sm.h into sm.full0.
 // CTA r adds up its share of the bins over all peers, then every CTA reads all the sums.
 __device__ void first_digit_sum(ClusterSmem& sm, int C, int me) {
   cluster_sync();  // every CTA's histogram is complete
   const int bpc = kMaxBins / C;
   for (int b = threadIdx.x; b < bpc; b += kCT) {
-    const uint32_t a = smem_u32(&sm.h[me * bpc + b]);
+    const uint32_t a = smem_u32(&sm.d.h[me * bpc + b]);
     uint32_t s = 0;
     for (int p = 0; p < C; ++p) s += ld_cluster_u32(cluster_map(a, p));
     sm.part[b] = s;
@@ -113,7 +163,7 @@ __device__ void first_digit_sum(ClusterSmem& sm, int C, int me) {
   cluster_sync();  // every owner's sums are complete
   for (int b = threadIdx.x; b < kMaxBins; b += kCT) {
     const int owner = b / bpc;
-    sm.full0[b] = ld_cluster_u32(cluster_map(smem_u32(&sm.part[b - owner * bpc]), owner));
+    sm.d.full0[b] = ld_cluster_u32(cluster_map(smem_u32(&sm.part[b - owner * bpc]), owner));
   }
   __syncthreads();
 }
@@ -177,8 +227,8 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   // the later-digit histograms the peers add into start at zero: barrier S0 (arrive now,
   // wait before the first access to another CTA's shared memory)
   for (int i = threadIdx.x; i < 2048; i += kCT) {
-    sm.fullb[1][i] = 0u;
-    sm.hl[i] = 0u;  // the second digit is counted in the candidate pass below
+    sm.d.fullb[1][i] = 0u;
+    sm.d.hl[i] = 0u;  // the second digit is counted in the candidate pass below
   }
   cluster_arrive();
   bool s0_pending = true;
@@ -201,89 +251,201 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
   // first digit: the threshold bin b*
   uint32_t d, above, count;
   if (!hist_g) {
-    for (int b = threadIdx.x; b < kMaxBins; b += kCT) sm.h[b] = 0u;
+    for (int b = threadIdx.x; b < kMaxBins; b += kCT) sm.d.h[b] = 0u;
     __syncthreads();
 #pragma unroll 4
     for (int step = 0; step < KPT; ++step) {
       const int p = seg0 + 32 * step + lane;
-      if (c0 + p < V) atomicAdd(&sm.h[keys[p] >> kHistShift], 1u);
+      if (c0 + p < V) atomicAdd(&sm.d.h[keys[p] >> kHistShift], 1u);
     }
     wait_s0();
     first_digit_sum(sm, C, me);
 #pragma unroll
-    for (int i = 0; i < 4; ++i) hv[i] = sm.full0[kMaxBins - 1 - 4 * (int)threadIdx.x - i];
+    for (int i = 0; i < 4; ++i) hv[i] = sm.d.full0[kMaxBins - 1 - 4 * (int)threadIdx.x - i];
   }
   digit_search(hv, 4, kMaxBins, (uint32_t)k, sm, d, above, count);
   uint32_t r = (uint32_t)k - above;  // rank still needed inside the current bin (1-based)
   unsigned long long prefix = (unsigned long long)d << 52;
   int pos = 52;                      // bits [pos, 64) of the threshold are fixed in `prefix`
   const uint32_t bstar = d;
-
-  // the elements that can be selected: bin >= b*; those in b* also count their second
-  // digit (key bits 19..10) into this CTA's histogram when a second digit is needed
   static_assert(kHistShift == 20, "second digit = key bits 19..10");
-  const bool second = count != r;
-  uint32_t cand = 0;
-#pragma unroll
-  for (int step = 0; step < KPT; ++step) {
-    const int p = seg0 + 32 * step + lane;
-    if (c0 + p < V) {
-      const uint32_t key = keys[p];
-      if ((key >> kHistShift) >= bstar) cand |= 1u << step;
-      if (second && (key >> kHistShift) == bstar) atomicAdd(&sm.hl[(key >> 10) & 1023u], 1u);
-    }
-  }
 
-  // later digits, until every element of the bin is needed: then the threshold is the
-  // prefix itself.  Each CTA adds its non-empty bins into the bin's owner (CTA
-  // bin / (bins / C), triple-buffered arrays), and after one barrier every CTA reads the
-  // sums of the bins it scans from their owners.
-  for (int level = 1; level < kLevels && count != r; ++level) {
-    const int width = kDigitWidth[level];
-    const int shift = pos - width;
-    const int bins = 1 << width;
-    const int bpc = bins / C;
-    uint32_t* fb = sm.fullb[level % 3];
-    if (level > 1) {  // the second digit was counted in the candidate pass
-      for (int b = threadIdx.x; b < bins; b += kCT) sm.hl[b] = 0u;
-      __syncthreads();
-      for (uint32_t m = cand; m; m &= m - 1) {
-        const int p = seg0 + 32 * (__ffs(m) - 1) + lane;
-        const unsigned long long c = comp(p);
-        if ((c >> pos) == (prefix >> pos)) atomicAdd(&sm.hl[(uint32_t)(c >> shift) & (uint32_t)(bins - 1)], 1u);
+  // The threshold bin b* holds `count` elements of the row, r of which are selected.  When
+  // they are few, every CTA gathers all of them and selects rank r on its own (merge path:
+  // two cluster barriers); otherwise the digits are resolved one by one across the cluster.
+  const bool merge = count != r && count <= (uint32_t)kMergeCap;  // the same in every CTA
+  uint32_t sel = 0;      // this thread's selected elements (bit `step`)
+  uint32_t base = 0;     // selected elements of the lower ranks
+  uint32_t total = 0;    // selected elements of the row (k when the invariant holds)
+  if (merge) {
+    wait_s0();
+    uint32_t above_bits = 0, cand_bits = 0;
+#pragma unroll
+    for (int step = 0; step < KPT; ++step) {
+      const int p = seg0 + 32 * step + lane;
+      if (c0 + p < V) {
+        const uint32_t bin = keys[p] >> kHistShift;
+        above_bits |= (bin > bstar ? 1u : 0u) << step;
+        cand_bits |= (bin == bstar ? 1u : 0u) << step;
       }
     }
+    // this CTA's b* elements, compacted into its list (at most `count` <= kMergeCap)
+    uint32_t n_loc = 0, n_above = 0;
+    uint32_t j = cta_excl_scan((uint32_t)__popc(cand_bits), sm, n_loc);
+    (void)cta_excl_scan((uint32_t)__popc(above_bits), sm, n_above);
+    for (uint32_t m = cand_bits; m; m &= m - 1) {
+      const int step = __ffs(m) - 1;
+      if (j < (uint32_t)kMergeCap) sm.m.loc[j] = comp(seg0 + 32 * step + lane);
+      ++j;
+    }
+    if (threadIdx.x == 0) {
+      sm.n_loc = n_loc;
+      sm.n_above = n_above;
+    }
+    cluster_sync();  // #A: every CTA's list and counts are complete
+    if ((int)threadIdx.x < C) {
+      sm.q_cnt[threadIdx.x] = ld_cluster_u32(cluster_map(smem_u32(&sm.n_loc), threadIdx.x));
+      sm.q_above[threadIdx.x] = ld_cluster_u32(cluster_map(smem_u32(&sm.n_above), threadIdx.x));
+      sm.q_ge[threadIdx.x] = 0u;
+    }
     __syncthreads();
-    wait_s0();
-    for (int b = threadIdx.x; b < bins; b += kCT) {
-      const uint32_t x = sm.hl[b];
-      if (x) red_cluster_add(cluster_map(smem_u32(&fb[b % bpc]), b / bpc), x);
+    // every CTA's list, in rank order
+    uint32_t M = 0;
+    for (int q = 0; q < C; ++q) {
+      const uint32_t n = min(sm.q_cnt[q], (uint32_t)kMergeCap - M);
+      for (uint32_t i = threadIdx.x; i < n; i += kCT)
+        sm.m.mrg[M + i] = ld_cluster_u64(cluster_map(smem_u32(&sm.m.loc[i]), q));
+      M += n;
     }
-    // the owned part of the next level's array: its last readers were done two barriers ago
-    for (int i = threadIdx.x; i < bpc; i += kCT) sm.fullb[(level + 1) % 3][i] = 0u;
-    cluster_sync();  // every addition is in its owner
-    const int per = bins / kCT;
-    uint32_t lv[4] = {0u, 0u, 0u, 0u};
+    cluster_arrive();  // done with the peers' memory (#B; its wait is at the very end)
+    __syncthreads();
+    // rank r among the gathered elements, on their low 52 bits (the top 12 are b*), by
+    // radix digits of 11, 11, 10, 10, 10 bits until every element of the digit is needed
+    constexpr unsigned long long kLow52 = (1ull << 52) - 1;
+    unsigned long long p52 = 0;
+    int ps = 52;
+    uint32_t rr = r;
+#pragma unroll 1
+    for (int pass = 0; pass < 5; ++pass) {
+      const int width = pass < 2 ? 11 : 10;
+      const int shift = ps - width;
+      const int bins = 1 << width;
+      for (int b2 = threadIdx.x; b2 < bins; b2 += kCT) sm.part[b2] = 0u;
+      __syncthreads();
+      for (uint32_t i = threadIdx.x; i < M; i += kCT) {
+        const unsigned long long c = sm.m.mrg[i] & kLow52;
+        if (ps == 52 || (c >> ps) == (p52 >> ps)) atomicAdd(&sm.part[(uint32_t)(c >> shift) & (uint32_t)(bins - 1)], 1u);
+      }
+      __syncthreads();
+      const int per = bins / kCT;
+      uint32_t lv[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int b = bins - 1 - per * (int)threadIdx.x - i;
-      if (i < per) lv[i] = ld_cluster_u32(cluster_map(smem_u32(&fb[b % bpc]), b / bpc));
+      for (int i = 0; i < 4; ++i)
+        if (i < per) lv[i] = sm.part[bins - 1 - per * (int)threadIdx.x - i];
+      uint32_t dd, ab, cn;
+      digit_search(lv, per, bins, rr, sm, dd, ab, cn);
+      rr -= ab;
+      p52 |= (unsigned long long)dd << shift;
+      ps = shift;
+      if (cn == rr) break;  // every element of this digit is selected
     }
-    digit_search(lv, per, bins, r, sm, d, above, count);
-    r -= above;
-    prefix |= (unsigned long long)d << shift;
-    pos = shift;
-  }
-  wait_s0();
-  const unsigned long long thr = prefix;  // every element of the final bin is selected
+    const unsigned long long thr = ((unsigned long long)bstar << 52) | p52;
+    // selected elements per rank: those above b* and the gathered ones >= thr
+    uint32_t start[kMaxC + 1];
+    start[0] = 0;
+    for (int q = 0; q < C; ++q) start[q + 1] = start[q] + min(sm.q_cnt[q], (uint32_t)kMergeCap - start[q]);
+    for (uint32_t i = threadIdx.x; i < M; i += kCT)
+      if (sm.m.mrg[i] >= thr) {
+        int q = 0;
+        while (q + 1 < C && i >= start[q + 1]) ++q;
+        atomicAdd(&sm.q_ge[q], 1u);
+      }
+    __syncthreads();
+    for (int q = 0; q < C; ++q) {
+      const uint32_t n = sm.q_above[q] + sm.q_ge[q];
+      if (q < me) base += n;
+      total += n;
+    }
+    sel = above_bits;
+    for (uint32_t m = cand_bits; m; m &= m - 1) {
+      const int step = __ffs(m) - 1;
+      if (comp(seg0 + 32 * step + lane) >= thr) sel |= 1u << step;
+    }
+  } else {
+    // the elements that can be selected: bin >= b*; those in b* also count their second
+    // digit (key bits 19..10) into this CTA's histogram when a second digit is needed
+    const bool second = count != r;
+    uint32_t cand = 0;
+#pragma unroll
+    for (int step = 0; step < KPT; ++step) {
+      const int p = seg0 + 32 * step + lane;
+      if (c0 + p < V) {
+        const uint32_t key = keys[p];
+        if ((key >> kHistShift) >= bstar) cand |= 1u << step;
+        if (second && (key >> kHistShift) == bstar) atomicAdd(&sm.d.hl[(key >> 10) & 1023u], 1u);
+      }
+    }
 
-  // selected = composite >= thr (all have bin >= b*); output offset = the selected count
-  // of the lower ranks, then of the lower warps
-  uint32_t sel = 0;
-  for (uint32_t m = cand; m; m &= m - 1) {
-    const int step = __ffs(m) - 1;
-    if (comp(seg0 + 32 * step + lane) >= thr) sel |= 1u << step;
+    // later digits, until every element of the bin is needed: then the threshold is the
+    // prefix itself.  Each CTA adds its non-empty bins into the bin's owner (CTA
+    // bin / (bins / C), triple-buffered arrays), and after one barrier every CTA reads the
+    // sums of the bins it scans from their owners.
+    for (int level = 1; level < kLevels && count != r; ++level) {
+      const int width = kDigitWidth[level];
+      const int shift = pos - width;
+      const int bins = 1 << width;
+      const int bpc = bins / C;
+      uint32_t* fb = sm.d.fullb[level % 3];
+      if (level > 1) {  // the second digit was counted in the candidate pass
+        for (int b = threadIdx.x; b < bins; b += kCT) sm.d.hl[b] = 0u;
+        __syncthreads();
+        for (uint32_t m = cand; m; m &= m - 1) {
+          const int p = seg0 + 32 * (__ffs(m) - 1) + lane;
+          const unsigned long long c = comp(p);
+          if ((c >> pos) == (prefix >> pos)) atomicAdd(&sm.d.hl[(uint32_t)(c >> shift) & (uint32_t)(bins - 1)], 1u);
+        }
+      }
+      __syncthreads();
+      wait_s0();
+      for (int b = threadIdx.x; b < bins; b += kCT) {
+        const uint32_t x = sm.d.hl[b];
+        if (x) red_cluster_add(cluster_map(smem_u32(&fb[b % bpc]), b / bpc), x);
+      }
+      // the owned part of the next level's array: its last readers were done two barriers ago
+      for (int i = threadIdx.x; i < bpc; i += kCT) sm.d.fullb[(level + 1) % 3][i] = 0u;
+      cluster_sync();  // every addition is in its owner
+      const int per = bins / kCT;
+      uint32_t lv[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int b = bins - 1 - per * (int)threadIdx.x - i;
+        if (i < per) lv[i] = ld_cluster_u32(cluster_map(smem_u32(&fb[b % bpc]), b / bpc));
+      }
+      digit_search(lv, per, bins, r, sm, d, above, count);
+      r -= above;
+      prefix |= (unsigned long long)d << shift;
+      pos = shift;
+    }
+    wait_s0();
+    const unsigned long long thr = prefix;  // every element of the final bin is selected
+    for (uint32_t m = cand; m; m &= m - 1) {
+      const int step = __ffs(m) - 1;
+      if (comp(seg0 + 32 * step + lane) >= thr) sel |= 1u << step;
+    }
+    // the selected counts of every rank, exchanged
+    uint32_t cta_total = 0;
+    (void)cta_excl_scan((uint32_t)__popc(sel), sm, cta_total);
+    if ((int)threadIdx.x < C) st_cluster_u32(cluster_map(smem_u32(&sm.nsel[me]), threadIdx.x), cta_total);
+    cluster_sync();  // every CTA's count is in every CTA; no shared-memory access across CTAs after this
+    for (int q = 0; q < C; ++q) {
+      if (q < me) base += sm.nsel[q];
+      total += sm.nsel[q];
+    }
   }
+  // every row selects exactly k elements (k < V here); anything else is a broken invariant
+  if (me == 0 && threadIdx.x == 0 && total != (uint32_t)k) atomicCAS(err, 0, 41);
+
+  // output offset: the selected count of the lower ranks, then of the lower warps
   uint32_t wcnt = __popc(sel);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) wcnt += __shfl_xor_sync(0xFFFFFFFFu, wcnt, o);
@@ -296,18 +458,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
     const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, z, o);
     if (lane >= o) z += y;
   }
-  const uint32_t wbase = __shfl_sync(0xFFFFFFFFu, z - wt, warp);
-  const uint32_t cta_total = __shfl_sync(0xFFFFFFFFu, z, 31);
-  if (threadIdx.x < C) st_cluster_u32(cluster_map(smem_u32(&sm.nsel[me]), threadIdx.x), cta_total);
-  cluster_sync();  // every CTA's count is in every CTA; no shared-memory access across CTAs after this
-  uint32_t o = wbase;
-  for (int q = 0; q < me; ++q) o += sm.nsel[q];
-  if (me == 0 && threadIdx.x == 0) {
-    // every row selects exactly k elements (k < V here); anything else is a broken invariant
-    uint32_t total = 0;
-    for (int q = 0; q < C; ++q) total += sm.nsel[q];
-    if (total != (uint32_t)k) atomicCAS(err, 0, 41);
-  }
+  uint32_t o = base + __shfl_sync(0xFFFFFFFFu, z - wt, warp);
 #pragma unroll 4
   for (int step = 0; step < KPT; ++step) {
     const bool b = (sel >> step) & 1u;
@@ -318,6 +469,7 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
     }
     o += __popc(m);
   }
+  if (merge) cluster_wait();  // #B: no CTA leaves while a peer may still read its list
 }
 template <int KPT>
 cudaError_t launch_kpt(const float* scores, long long rows, int T, int N, long long q_pos0, int k, int C,

@@ -87,3 +87,27 @@ def test_mtp_draft_steps_reuse_step1_indices(dsa, orc):
             assert torch.equal(didx, saved)
         assert np.all(idx < 4000)
         assert_close(host(outs[0]), routs[0], f"mtp step {step + 1}")
+
+
+@pytest.mark.parametrize("B,G", [(3, 2), (2, 3), (1, 2), (8, 1)])
+def test_decode_step_matches_oracle(dsa, orc, B, G):
+    """dsa_decode_step (two micro-batches on two streams, indexers taking turns) gives every
+    group the oracle's index list bit for bit and its attention within the tolerance."""
+    import torch
+    w = C.scaled(C.WORKLOADS["decode1m"], B=B, N=9000, q_pos0=8999, groups=G)
+    groups, ref = [], []
+    for g in range(G):
+        iq, wt, ik, qs, kvs = C.host_group_inputs(w, g)
+        ref.append(orc.group_forward(iq, wt, ik, qs, kvs, w.q_pos0, w.k, C.SCALE))
+        groups.append(dict(iq=dev_bf16(iq), w=dev(wt), ik=dev_bf16(ik), qs=[dev_bf16(x) for x in qs],
+                           kvs=[dev_bf16(x) for x in kvs],
+                           idx=torch.empty(B, 1, w.k, dtype=torch.int32, device="cuda"),
+                           outs=[torch.empty(B, 1, w.H, 512, dtype=torch.float32, device="cuda") for _ in range(w.L)]))
+    dsa.dsa_decode_step(groups, w.k, C.SCALE)
+    torch.cuda.synchronize()
+    assert dsa.dsa_check_device_status() == 0
+    for g in range(G):
+        ridx, routs = ref[g]
+        assert np.array_equal(host(groups[g]["idx"]), ridx), f"group {g}"
+        for l in range(w.L):
+            assert_close(host(groups[g]["outs"][l]), routs[l], f"group {g} layer {l}")
