@@ -17,7 +17,8 @@ import subprocess
 import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_SRCS = [os.path.join(_HERE, "dsa_oracle.c"), os.path.join(_HERE, "verify_oracle.c")]
+_SRCS = [os.path.join(_HERE, "dsa_oracle.c"), os.path.join(_HERE, "verify_oracle.c"),
+         os.path.join(_HERE, "fp8_oracle.c")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 OR_OK = 0
@@ -58,8 +59,11 @@ class Oracle:
         L.oracle_dense_masked_attn.argtypes = [P, P, P, I, I, I, I, I, I, I, D, P]
         L.oracle_group_forward.argtypes = [P, P, P, P, P, I, I, I, I, I, I, Lg, I, I, I, I, D, I, P, P]
         L.oracle_verify.argtypes = [P, P, P, P, P, I, I, I, P, P, P, P]
+        L.oracle_index_score_e4m3.argtypes = [P, P, P, I, I, I, I, I, Lg, P]
+        L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
+        L.oracle_e4m3_to_double.restype = D
         for f in ("oracle_index_score", "oracle_topk", "oracle_sparse_attn",
-                  "oracle_dense_masked_attn", "oracle_group_forward", "oracle_verify"):
+                  "oracle_dense_masked_attn", "oracle_group_forward", "oracle_verify", "oracle_index_score_e4m3"):
             getattr(L, f).restype = I
         self.L = L
 
@@ -129,6 +133,23 @@ class Oracle:
                "oracle_group_forward")
         return idx_shared, outs
 
+
+    def e4m3_to_double(self, b: int) -> float:
+        """One E4M3 byte decoded (fp8_oracle.c)."""
+        return float(self.L.oracle_e4m3_to_double(int(b)))
+
+    def index_score_e4m3(self, q: np.ndarray, w: np.ndarray, k: np.ndarray, q_pos0: int) -> np.ndarray:
+        """q [B,T,nh,hd] E4M3 bytes, w [B,T,nh] f32, k [B,N,hd] E4M3 bytes -> scores [B,T,N]
+        f64 (-inf where the position is not visible to the query)."""
+        q = np.ascontiguousarray(q, dtype=np.uint8)
+        k = np.ascontiguousarray(k, dtype=np.uint8)
+        w = np.ascontiguousarray(w, dtype=np.float32)
+        B, T, nh, hd = q.shape
+        N = k.shape[1]
+        out = np.empty((B, T, N), dtype=np.float64)
+        _check(self.L.oracle_index_score_e4m3(_ptr(q), _ptr(w), _ptr(k), B, T, N, nh, hd, q_pos0, _ptr(out)),
+               "oracle_index_score_e4m3")
+        return out
 
     def verify(self, p: np.ndarray, q: np.ndarray, draft: np.ndarray, u: np.ndarray, u2: np.ndarray):
         """MTP verify step (rejection sampling), verify_oracle.c.  p, q [B, S, V] float32

@@ -12,6 +12,7 @@ Generator (counter based, SplitMix64 of Steele, Lea and Flood, OOPSLA 2014):
     draw(key, j)  = mix64(key + GAMMA*(j+1))          GAMMA = 0x9E3779B97F4A7C15
 Distributions, for the element with flat index i:
     int17   (integer-valued bf16, uniform on -8..8):  ((draw(key,i) >> 32) mod 17) - 8
+            (int17_e4m3: the same integers as E4M3 bytes)
     pow2    (float32 head weight, 2^-1 .. 2^-6):      2^-(1 + ((draw(key,i) >> 32) mod 6))
     normal  (bf16, approximately N(0,1)): the sum S of the twelve 16-bit fields of
             draw(key,3i), draw(key,3i+1), draw(key,3i+2) (Irwin-Hall with 12 terms),
@@ -90,6 +91,19 @@ def int17_bf16(key: int, shape=None, index: np.ndarray = None) -> np.ndarray:
     i = _flat(index if index is not None else shape)
     v = ((draws(key, i) >> np.uint64(32)) % np.uint64(17)).astype(np.int64) - 8
     out = f32_to_bf16_bits(v.astype(np.float32))
+    return out.reshape(shape) if index is None else out
+
+
+# E4M3 bytes of the integers 0..8 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits)
+E4M3_OF_INT = np.array([0x00, 0x38, 0x40, 0x44, 0x48, 0x4A, 0x4C, 0x4E, 0x50], dtype=np.uint8)
+
+
+def int17_e4m3(key: int, shape=None, index: np.ndarray = None) -> np.ndarray:
+    """The same integers as int17_bf16 (same key, same draws), as E4M3 bytes."""
+    i = _flat(index if index is not None else shape)
+    v = ((draws(key, i) >> np.uint64(32)) % np.uint64(17)).astype(np.int64) - 8
+    out = E4M3_OF_INT[np.abs(v)] | np.where(v < 0, np.uint8(0x80), np.uint8(0))
+    out = out.astype(np.uint8)
     return out.reshape(shape) if index is None else out
 
 

@@ -460,4 +460,50 @@ def pin_verify_accepted_length_is_leading_run(o):
     del V
 
 
+# ------------------------------------------------------------------ FP8 index keys
+# "Le contexte d'un million de tokens", Entraînement par renforcement: an FP8 KV cache.
+# Read as E4M3; its values are fixed by the format's definition.
+
+def pin_e4m3_decode_reference_values(o):
+    """E4M3 reference values: 1.0, 2.0, 3.0, the largest finite 448, the smallest normal
+    2^-6, the smallest subnormal 2^-9, signed zero, NaN only at S.1111.111, and the
+    positive codes ordered as their values."""
+    ref = {0x00: 0.0, 0x38: 1.0, 0x40: 2.0, 0x44: 3.0, 0x7E: 448.0, 0x08: 2.0 ** -6, 0x01: 2.0 ** -9,
+           0x07: 7 * 2.0 ** -9, 0x3F: 1.875, 0xB8: -1.0, 0xFE: -448.0}
+    for b, v in ref.items():
+        assert o.e4m3_to_double(b) == v, hex(b)
+    assert math.copysign(1.0, o.e4m3_to_double(0x80)) == -1.0 and o.e4m3_to_double(0x80) == 0.0
+    assert math.isnan(o.e4m3_to_double(0x7F)) and math.isnan(o.e4m3_to_double(0xFF))
+    pos = [o.e4m3_to_double(b) for b in range(0x7F)]
+    assert all(a < b for a, b in zip(pos, pos[1:]))
+
+
+def pin_index_score_e4m3_equals_bf16_on_integers(o):
+    """The workload's integer-valued keys and queries encoded as E4M3 and as bf16 give
+    the same scores (the values are exact in both formats)."""
+    key = lambda kind: synth.stream_key(91, synth.tensor_id(kind))
+    q8 = synth.int17_e4m3(key(synth.KIND_IQ), (2, 3, 32, 128))
+    k8 = synth.int17_e4m3(key(synth.KIND_IK), (2, 300, 128))
+    qb = synth.int17_bf16(key(synth.KIND_IQ), (2, 3, 32, 128))
+    kb = synth.int17_bf16(key(synth.KIND_IK), (2, 300, 128))
+    w = synth.pow2_f32(key(synth.KIND_W), (2, 3, 32))
+    a = o.index_score_e4m3(q8, w, k8, 200)
+    b = o.index_score(qb, w, kb, 200)
+    assert np.array_equal(a, b)
+    assert np.isinf(a[:, 0, 201:]).all() and np.isfinite(a[:, 2, :203]).all()
+
+
+def pin_index_score_e4m3_one_hot(o):
+    """q[t,h] = e_h and k[s] = e_h for all heads: I = sum_h w[t,h] (E4M3 1.0 = 0x38)."""
+    q = np.zeros((1, 1, 4, 8), np.uint8)
+    for h in range(4):
+        q[0, 0, h, h] = 0x38
+    k = np.zeros((1, 2, 8), np.uint8)
+    k[0, 0, :4] = 0x38   # dot 1 with every head
+    k[0, 1, :4] = 0xB8   # dot -1: ReLU gives 0
+    w = np.array([[[0.5, 0.25, 0.125, 0.0625]]], np.float32)
+    s = o.index_score_e4m3(q, w, k, 1)
+    assert s[0, 0, 0] == 0.9375 and s[0, 0, 1] == 0.0
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

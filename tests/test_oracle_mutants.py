@@ -12,7 +12,8 @@ import pins
 HERE = os.path.dirname(oracle.__file__)
 SRC = os.path.join(HERE, "dsa_oracle.c")
 VERIFY_SRC = os.path.join(HERE, "verify_oracle.c")
-SOURCES = [SRC, VERIFY_SRC]
+FP8_SRC = os.path.join(HERE, "fp8_oracle.c")
+SOURCES = [SRC, VERIFY_SRC, FP8_SRC]
 
 MUTANTS = {
     "relu_dropped": ("double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
@@ -42,6 +43,11 @@ MUTANTS = {
                                VERIFY_SRC),
     "verify_len_counts_all": ("while (n < S && accept[(long)b * S + n]) ++n;",
                               "for (int j = 0; j < S; ++j) n += accept[(long)b * S + j];", VERIFY_SRC),
+    # FP8 index keys (fp8_oracle.c)
+    "e4m3_bias": ("ldexp(1.0 + (double)m / 8.0, e - 7)", "ldexp(1.0 + (double)m / 8.0, e - 8)", FP8_SRC),
+    "e4m3_subnormal_scale": ("ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)", FP8_SRC),
+    "e4m3_relu_dropped": ("total += (double)wt[h] * (dot > 0.0 ? dot : 0.0);", "total += (double)wt[h] * dot;", FP8_SRC),
+    "e4m3_key_index": ("oracle_e4m3_to_double(ks[d])", "oracle_e4m3_to_double(ks[0])", FP8_SRC),
 }
 
 
