@@ -58,7 +58,9 @@ def algorithmic(w):
     queries and writes the outputs; the index list is written once.  The score write
     (4 B per visible key, L2-resident) is not algorithmic: it is returned separately."""
     vis = min(w.N, w.q_pos0 + w.T)
-    idx_launch = w.B * w.T * INDEXER_BYTES_PER_QUERY + w.B * vis * INDEXER_BYTES_PER_KEY
+    esz = 1 if w.index_fp8 else 2  # E4M3 or bf16 index keys and indexer queries
+    per_query = INDEXER_BYTES_PER_QUERY - 32 * 128 * (2 - esz)
+    idx_launch = w.B * w.T * per_query + w.B * vis * INDEXER_BYTES_PER_KEY * esz // 2
     attn = w.B * w.T * w.L * w.steps * (w.k * ROW_BYTES + w.H * 576 * 2 + w.H * 512 * 4)
     scores = w.B * w.T * vis * SCORE_BYTES_PER_KEY
     return w.groups * (idx_launch + attn + w.B * w.T * w.k * 4), idx_launch, scores
@@ -203,23 +205,25 @@ def make_inputs(w, device, rank):
     bf = torch.bfloat16
     f32 = torch.float32
     ins, outs_spec = [], []
+    ixt = torch.uint8 if w.index_fp8 else bf
+    fill_index = sd.int17_e4m3 if w.index_fp8 else sd.int17_bf16
     for g in range(w.groups):
-        ins += [((w.B, w.T, 32, 128), bf), ((w.B, w.T, 32), f32)]
+        ins += [((w.B, w.T, 32, 128), ixt), ((w.B, w.T, 32), f32)]
         ins += [((w.B, w.T, w.H, 576), bf)] * (w.L + max(0, w.steps - 1))
         outs_spec += [((w.B, w.T, w.k), torch.int32)] + [((w.B, w.T, w.H, 512), f32)] * w.L
     in_buf, in_views = _packed(ins, device)
     out_buf, out_views = _packed(outs_spec, device)
     groups = []
     for g in range(w.groups):
-        ik = torch.empty(w.B, w.N, 128, dtype=bf, device=device)
-        sd.int17_bf16(ik, rank_key(w.key(synth.KIND_IK, g), rank))
+        ik = torch.empty(w.B, w.N, 128, dtype=ixt, device=device)
+        fill_index(ik, rank_key(w.key(synth.KIND_IK, g), rank))
         kvs = []
         for l in range(w.L):
             kv = torch.empty(w.B, w.N, 576, dtype=bf, device=device)
             sd.normal_bf16(kv, rank_key(w.key(synth.KIND_KV, g, l), rank))
             kvs.append(kv)
         iq, wt = in_views.pop(0), in_views.pop(0)
-        sd.int17_bf16(iq, rank_key(w.key(synth.KIND_IQ, g), rank))
+        fill_index(iq, rank_key(w.key(synth.KIND_IQ, g), rank))
         sd.pow2_f32(wt, rank_key(w.key(synth.KIND_W, g), rank))
         qs = []
         for l in range(w.L):
@@ -251,6 +255,8 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     dsa.lib()
     groups = make_inputs(w, device, rank)
     micro = args.schedule == "micro" and w.T == 1 and w.steps == 1 and w.B >= 2
+    if w.index_fp8 and not micro:
+        raise ValueError("the E4M3 index format runs through the micro-batched decode step only")
     ws = dsa.decode_workspace(w.B, w.N, w.k, w.H, w.L, device) if micro else \
         dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, device)
     stream = torch.cuda.Stream(device)
@@ -325,12 +331,13 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     scores = torch.empty(w.B, w.T, w.N, dtype=torch.float32, device=device)
     # captured in a graph like the step, so the host-side set-up of a launch (tensor-map
     # encoding) is not inside the timed region
+    index_score = dsa.dsa_index_score_e4m3 if w.index_fp8 else dsa.dsa_index_score
     with torch.cuda.stream(stream):
-        dsa.dsa_index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores, stream=stream)
+        index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores, stream=stream)
     torch.cuda.synchronize()
     igraph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(igraph, stream=stream):
-        dsa.dsa_index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores, stream=stream)
+        index_score(g0["iq"], g0["wt"], g0["ik"], w.q_pos0, scores=scores, stream=stream)
     torch.cuda.synchronize()
     idx_times = timed(igraph.replay, args.steps, args.warmup)
     res["idx_ms"] = sum(idx_times) / len(idx_times)
@@ -495,7 +502,7 @@ def workload_config(w, world: int) -> dict:
     """The `config` object of the bench line: the workload and how it is run (the same in
     both arms)."""
     return {"workload": w.name, "B": w.B, "T": w.T, "N": w.N, "k": w.k, "H": w.H, "L": w.L, "groups": w.groups,
-            "draft_steps": w.steps, "parallelism": f"dp{world}" if world > 1 else "single GPU",
+            "draft_steps": w.steps, "index_keys": "e4m3" if w.index_fp8 else "bf16", "parallelism": f"dp{world}" if world > 1 else "single GPU",
             "l2": "flushed before every timed step (512 MiB write, then a 512 MiB read so the write-back is not timed)"}
 
 
@@ -673,7 +680,7 @@ def main():
     }
     if not args.no_extra and args.workload == "decode128k":
         extra = {"mtp_verify": run_verify(args, device, peak)}
-        for name in ("decode1m", "mtp", "prefill"):
+        for name in ("decode1m", "mtp", "prefill", "decode128k_fp8"):
             we, r2 = run_ours(args, rank, world, device, w=C.WORKLOADS[name], e2e=False)
             b2, ib2, _ = algorithmic(we)
             ms, ims = r2["step_ms"], r2["idx_ms"]

@@ -117,6 +117,23 @@ dsa_status dsa_index_score(const uint16_t *q, const float *w, const uint16_t *k,
                            cudaStream_t stream);
 
 /*
+ * Step 1 over an FP8 index-key cache ("Le contexte d'un million de tokens", reinforcement
+ * learning of the agent: an FP8 KV cache keeps memory within budget; the format is not
+ * named there and E4M3 is taken: 1 sign bit, 4 exponent bits with bias 7, 3 mantissa
+ * bits, subnormals, S.1111.111 = NaN).  Same layouts and output as dsa_index_score with
+ * one byte per element of q and k, which halves the bytes of the key stream:
+ *   q      [B, T, 32, 128]  E4M3   indexer queries
+ *   w      [B, T, 32]       f32    per-query head weights
+ *   k      [B, N, 128]      E4M3   index-key cache
+ *   scores [B, T, N]        f32    out, as dsa_index_score
+ * Products of E4M3 values are exact in f32; they are accumulated in f32 on the tensor
+ * cores.
+ */
+dsa_status dsa_index_score_e4m3(const uint8_t *q, const float *w, const uint8_t *k,
+                                int B, int T, int N, long long q_pos0, float *scores,
+                                cudaStream_t stream);
+
+/*
  * Step 2 -- top-k select.
  *   scores [B, T, N] f32 (only s <= q_pos0 + t is read)
  *   idx    [B, T, k] i32 out: the selected token positions in ascending order; when
@@ -207,13 +224,16 @@ dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t 
  *   workspace   dsa_decode_workspace_size(B, N, k, H, L) bytes, 256-byte aligned
  * Uses events created once per device and host thread.
  */
+#define DSA_INDEX_BF16 0 /* index_format: iq and ik hold bf16                          */
+#define DSA_INDEX_E4M3 1 /* index_format: iq and ik hold E4M3 bytes (dsa_index_score_e4m3) */
 typedef struct {
-    const uint16_t *iq, *ik; /* [B, 1, 32, 128] and [B, N, 128] bf16                        */
+    const void *iq, *ik;     /* [B, 1, 32, 128] and [B, N, 128], element type index_format    */
     const float *w;          /* [B, 1, 32] f32                                                */
     const uint16_t *q[DSA_MAX_LAYERS];  /* [B, 1, H, 576] bf16 per layer                     */
     const uint16_t *kv[DSA_MAX_LAYERS]; /* [B, N, 576] bf16 per layer                        */
     int32_t *idx;                       /* [B, 1, k] out: the group's index list            */
     float *out[DSA_MAX_LAYERS];         /* [B, 1, H, 512] f32 per layer                     */
+    int index_format;                   /* DSA_INDEX_BF16 or DSA_INDEX_E4M3                  */
 } dsa_group_io;
 
 size_t dsa_decode_workspace_size(int B, int N, int k, int H, int L);

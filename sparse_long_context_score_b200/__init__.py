@@ -28,7 +28,8 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
           -4: "DSA_ERR_CUDA", -5: "DSA_ERR_TIMEOUT", -6: "DSA_ERR_DEVICE"}
 
 # every symbol include/dsa.h declares
-EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_topk",
+EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_index_score_e4m3",
+           "dsa_topk",
            "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error",
            "dsa_check_device_status", "dsa_last_cuda_error", "dsa_cuda_error_string", "dsa_verify",
            "dsa_decode_workspace_size", "dsa_decode_step")
@@ -38,7 +39,7 @@ class GroupIO(ctypes.Structure):
     """dsa_group_io: one IndexShare group's tensors for dsa_decode_step."""
     _fields_ = [("iq", ctypes.c_void_p), ("ik", ctypes.c_void_p), ("w", ctypes.c_void_p),
                 ("q", ctypes.c_void_p * MAX_LAYERS), ("kv", ctypes.c_void_p * MAX_LAYERS), ("idx", ctypes.c_void_p),
-                ("out", ctypes.c_void_p * MAX_LAYERS)]
+                ("out", ctypes.c_void_p * MAX_LAYERS), ("index_format", ctypes.c_int)]
 
 
 class DsaError(RuntimeError):
@@ -65,6 +66,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_workspace_size.argtypes = [I, I, I, I, I, I]
         L.dsa_workspace_size.restype = S
         L.dsa_index_score.argtypes = [P, P, P, I, I, I, LL, P, P]
+        L.dsa_index_score_e4m3.argtypes = [P, P, P, I, I, I, LL, P, P]
         L.dsa_topk.argtypes = [P, I, I, I, LL, I, P, P, S, P]
         L.dsa_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, F, P, P, S, P]
         L.dsa_group_forward.argtypes = [P, P, P, P, P, I, I, I, I, LL, I, I, F, I, P, P, P, S, P]
@@ -82,7 +84,7 @@ def lib() -> ctypes.CDLL:
         L.dsa_decode_workspace_size.restype = S
         L.dsa_decode_step.argtypes = [P, I, I, I, I, I, I, F, P, S, P, P]
         L.dsa_decode_step.restype = I
-        for f in ("dsa_index_score", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc",
+        for f in ("dsa_index_score", "dsa_index_score_e4m3", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc",
                   "dsa_verify"):
             getattr(L, f).restype = I
         _lib = L
@@ -171,6 +173,22 @@ def dsa_index_score(q, w, k, q_pos0: int, scores=None, stream=None):
                                _ptr(k, _bf16_types(), "k", (B, N, INDEX_DIM)), B, T, N, int(q_pos0),
                                _ptr(scores, (torch.float32,), "scores", (B, T, N)), _stream(stream))
     _check(rc, "dsa_index_score")
+    return scores
+
+
+def dsa_index_score_e4m3(q, w, k, q_pos0: int, scores=None, stream=None):
+    """q [B,T,32,128] E4M3 bytes (uint8), w [B,T,32] f32, k [B,N,128] E4M3 bytes -> scores
+    [B,T,N] f32."""
+    torch = _torch()
+    B, T = q.shape[0], q.shape[1]
+    N = k.shape[1]
+    if scores is None:
+        scores = torch.empty((B, T, N), dtype=torch.float32, device=q.device)
+    rc = lib().dsa_index_score_e4m3(_ptr(q, (torch.uint8,), "q", (B, T, INDEX_HEADS, INDEX_DIM)),
+                                    _ptr(w, (torch.float32,), "w", (B, T, INDEX_HEADS)),
+                                    _ptr(k, (torch.uint8,), "k", (B, N, INDEX_DIM)), B, T, N, int(q_pos0),
+                                    _ptr(scores, (torch.float32,), "scores", (B, T, N)), _stream(stream))
+    _check(rc, "dsa_index_score_e4m3")
     return scores
 
 
@@ -288,7 +306,8 @@ def decode_workspace(B: int, N: int, k: int, H: int, L: int, device=None):
 def dsa_decode_step(groups, k: int, scale: float, ws=None, stream=None, side=None):
     """A micro-batched decode step over IndexShare groups (see include/dsa.h).  `groups` is
     a list of dicts with iq, w, ik, qs (L tensors), kvs (L tensors), idx, outs (L tensors);
-    `side` a second CUDA stream (created when None)."""
+    iq and ik are bf16, or uint8 holding E4M3 bytes (the index format is taken from their
+    dtype); `side` a second CUDA stream (created when None)."""
     torch = _torch()
     G = len(groups)
     L = len(groups[0]["qs"])
@@ -301,9 +320,12 @@ def dsa_decode_step(groups, k: int, scale: float, ws=None, stream=None, side=Non
     arr = (GroupIO * G)()
     for g, d in enumerate(groups):
         io = arr[g]
-        io.iq = _ptr(d["iq"], _bf16_types(), "iq", (B, 1, INDEX_HEADS, INDEX_DIM))
+        f8 = d["ik"].dtype == torch.uint8
+        itypes = (torch.uint8,) if f8 else _bf16_types()
+        io.index_format = 1 if f8 else 0
+        io.iq = _ptr(d["iq"], itypes, "iq", (B, 1, INDEX_HEADS, INDEX_DIM))
         io.w = _ptr(d["w"], (torch.float32,), "w", (B, 1, INDEX_HEADS))
-        io.ik = _ptr(d["ik"], _bf16_types(), "ik", (B, N, INDEX_DIM))
+        io.ik = _ptr(d["ik"], itypes, "ik", (B, N, INDEX_DIM))
         io.idx = _ptr(d["idx"], (torch.int32,), "idx", (B, 1, k))
         if len(d["qs"]) != L or len(d["kvs"]) != L or len(d["outs"]) != L:
             raise ValueError("every group needs L queries, caches and outputs")

@@ -12,29 +12,32 @@
 // M = 64 reaches ~600 MAC/cycle at N = 32, ~1200 at N = 64, ~2000 at N >= 128), so the
 // S product is issued with the widest N the shared memory allows: two stages of 64 rows
 // (73.7 KB each) beside the 73.7 KB of Q.
-// Because S has one head per TMEM lane, each softmax thread owns one head: its running
-// max and sum stay in registers and need no cross-thread reduction.  The running max is
+// S has one head per TMEM lane, so a head's logits stay within one warp: its running max
+// and sum live in registers (four threads per head, two shuffles per reduction).  The running max is
 // only moved (and O rescaled in TMEM) when a tile's max exceeds it by more than 2^8, so
 // rescaling is rare; exponentials may then exceed 1 by at most 2^8, which f32 and bf16
 // carry without loss of relative precision.
 //
-// Warp roles (416 threads):
+// Warp roles (448 threads):
 //   warps 0..7  gather: warps 4s..4s+3 own stage s and its tiles s, s+2, s+4, ...; each
 //               brings 16 of the 64 selected rows as 16-byte cp.async chunks written
-//               straight into the 128-byte-swizzled tensor-core layout, waits for its own
-//               copies, fences them to the async proxy and arrives on the stage barrier,
-//               so both stages gather at once; a lane's row index for the warp's next tile
-//               is loaded while the current one is copied.  (Random 1152-byte rows are too
-//               small for TMA: measured on B200 with the same bytes in flight, a 128-byte
-//               box per row reached 0.57 TB/s, 4-row gather boxes 1.6 TB/s, one bulk copy
-//               per row 2.8 TB/s, 16-byte cp.async 4.9 TB/s.)
+//               straight into the 128-byte-swizzled tensor-core layout (a lane holds its
+//               own rows' indices, and one instruction moves four whole 128-byte lines),
+//               waits for its own copies, fences them to the async proxy and arrives on the
+//               stage barrier, so both stages gather at once; the row indices of the warp's
+//               next tile are loaded while the current one is copied.  (Random 1152-byte
+//               rows are too small for TMA: measured on B200 with the same bytes in flight,
+//               a 128-byte box per row reached 0.57 TB/s, 4-row gather boxes 1.6 TB/s, one
+//               bulk copy per row 2.8 TB/s, 16-byte cp.async 4.9 TB/s.)
 //   warp 8      TMEM allocation and the query load (one TMA load of the 64 query rows);
-//               one elected lane issues S(i) once tile i has landed and O += P(i) V(i)
-//               once P(i) is published, whichever is ready (PV first), so the softmax of
-//               one tile overlaps the next tile's logits and a stage is released as soon
-//               as its PV completes;
-//   warps 9..12 softmax (threads on lanes 0..15 of each warp own a head), P as bf16 in
-//               shared memory.
+//               one elected lane issues S(i) once tile i has landed and its S buffer is
+//               free, so the softmax of one tile overlaps the next tile's logits;
+//   warps 9..12 softmax (warp q reads TMEM lanes 0..15 of quarter q, heads 16q..16q+15;
+//               four threads per head), P as bf16 in shared memory;
+//   warp 13     one elected lane issues O += P(i) V(i) once P(i) is published; as a warp
+//               of its own it does not wait behind the next S, whose MMAs its own
+//               interleave with in the tensor pipe, and a stage is released as soon as its
+//               PV completes.
 // The key splits of one (row, layer) run as one thread-block cluster.  After the main
 // loop the splits exchange their running max and sum per head through distributed shared
 // memory; each split scales its unnormalised O by its share of the normaliser and writes it
@@ -72,13 +75,12 @@ static_assert(64 * kKeys * 2 == kBlockBytes, "P fills one column block");
 constexpr int kProducerWarps = 8;                // four warps per stage, 16 rows each
 constexpr int kWarpsPerStage = kProducerWarps / kStages;
 constexpr int kRowsPerWarp = kKeys / kWarpsPerStage;           // 16
-constexpr int kChunksPerRow = kDqk / 8;                         // 72 chunks of 16 bytes
-constexpr int kChunksPerLane = kRowsPerWarp * kChunksPerRow / 32;  // 36
-constexpr int kMmaWarp = kProducerWarps;
+constexpr int kMmaWarp = kProducerWarps;           // Q load, TMEM allocation, S = Q K^T
 constexpr int kSoftmaxWarp0 = kProducerWarps + 1;
-constexpr int kThreadsA = (kProducerWarps + 5) * 32;  // 416
-static_assert(kSoftmaxWarp0 + 4 == kThreadsA / 32, "four softmax warps, one per TMEM lane quarter");
-static_assert(kRowsPerWarp * kChunksPerRow % 32 == 0, "whole chunks per lane");
+constexpr int kPvWarp = kSoftmaxWarp0 + 4;         // O^T += V^T P^T
+constexpr int kThreadsA = (kPvWarp + 1) * 32;      // 448
+static_assert(kThreadsA == 448, "8 gather, 1 S, 4 softmax and 1 PV warp");
+static_assert(kRowsPerWarp == 16, "a gather warp copies 4 x 4 rows");
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kMaxSplits = 8;                    // key splits of one (row, layer): one portable cluster
 
@@ -90,7 +92,7 @@ constexpr int kOffM = kOffL + 64 * 4;            // [64] f32
 constexpr int kOffCoef = kOffM + 64 * 4;         // [64] f32: this split's share of the normaliser
 constexpr int kOffMask = kOffCoef + 64 * 4;      // [kStages] u64: valid rows of the tile in the stage
 constexpr int kOffVote = kOffMask + kStages * 8;  // [2] u32 (tile parity): one byte per softmax warp
-constexpr int kNumBars = 2 * kStages + 10;
+constexpr int kNumBars = 2 * kStages + 11;
 constexpr int kOffBar = kOffVote + 8;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmemA = kOffTmem + 16 + 1024;     // + alignment slack
@@ -134,6 +136,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   const uint32_t ofinal_bar = bar0 + 8u * (2 * kStages + 7);
   const uint32_t qfull_bar = bar0 + 8u * (2 * kStages + 8);
   const uint32_t grp_bar = bar0 + 8u * (2 * kStages + 9);
+  const uint32_t sdone_bar = bar0 + 8u * (2 * kStages + 10);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
 
   const int split = blockIdx.x, row = blockIdx.y, layer = blockIdx.z;
@@ -158,6 +161,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     mbar_init(ofinal_bar, 1);
     mbar_init(qfull_bar, 1);
     mbar_init(grp_bar, 128);
+    mbar_init(sdone_bar, 1);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -183,41 +187,53 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     const int32_t* sel = idx + (size_t)row * k + j0;
     const uint16_t* kvb = layers.kv[layer] + (size_t)b * N * kDqk;
     const uint32_t st = sStage + ps * kStageBytes;
-    auto load_index = [&](int tile) {
-      const int key = tile * kKeys + r0 + (lane & 15);
-      return (tile < ntiles && key < nkeys) ? __ldg(&sel[key]) : -1;
+    // lane l copies, for g < 4, row r0 + 4g + l/8 of the tile: its 16-byte chunks l%8 + 8m
+    // (m < 9), i.e. 16 bytes of each of the row's nine 128-byte column blocks.  One
+    // instruction thus moves four whole 128-byte lines (four rows, one column block), and
+    // every lane holds its own rows' indices (no shuffles in the copy loop).
+    const int rsub = lane >> 3, c8 = lane & 7;
+    auto load_index = [&](int tile, int (&out)[4]) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int key = tile * kKeys + r0 + 4 * g + rsub;
+        out[g] = (tile < ntiles && key < nkeys) ? __ldg(&sel[key]) : -1;
+      }
     };
-    int cur = load_index(ps);
+    int cur[4], nxt[4];
+    load_index(ps, cur);
     for (int i = ps; i < ntiles; i += kStages) {
-      const int nxt = load_index(i + kStages);  // in flight while this tile is copied
+      load_index(i + kStages, nxt);  // in flight while this tile is copied
       bool ok = true;
       if (lane == 0) ok = mbar_wait(empty_bar(ps), ((i / kStages) & 1) ^ 1, err, 21);
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
-      const bool valid = cur >= 0 && cur < N;
-      const uint32_t vm = __ballot_sync(0xFFFFFFFFu, valid) & 0xFFFFu;
+      uint32_t vm = 0;  // bit 4g + t: row r0 + 4g + t of the tile is a valid selection
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const uint32_t bal = __ballot_sync(0xFFFFFFFFu, cur[g] >= 0 && cur[g] < N);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) vm |= ((bal >> (8 * t)) & 1u) << (4 * g + t);
+      }
       if (lane == 0) reinterpret_cast<uint16_t*>(s_mask + ps)[wq] = (uint16_t)vm;
-      const int my_row = valid ? cur : 0;
-#pragma unroll 6
-      for (int j = 0; j < kChunksPerLane; ++j) {
-        const int q = lane + 32 * j;
-        const int rl = q / kChunksPerRow;            // row of the warp, 0..15
-        const int c = q - rl * kChunksPerRow;        // 16-byte chunk of the row, 0..71
-        const int srow = __shfl_sync(0xFFFFFFFFu, my_row, rl);
-        const bool v = (vm >> rl) & 1u;
-        const int r = r0 + rl;
-        const uint32_t dst = st + (c >> 3) * kBlockBytes + r * 128 + (((c & 7) ^ (r & 7)) << 4);
-        cp_async_16(dst, kvb + (size_t)srow * kDqk + c * 8, v ? 16 : 0);
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const bool v = cur[g] >= 0 && cur[g] < N;
+        const uint16_t* src = kvb + (size_t)(v ? cur[g] : 0) * kDqk + c8 * 8;
+        const int r = r0 + 4 * g + rsub;
+        const uint32_t dst = st + r * 128 + ((c8 ^ (r & 7)) << 4);
+#pragma unroll
+        for (int m = 0; m < kBlocks; ++m) cp_async_16(dst + m * kBlockBytes, src + m * 64, v ? 16 : 0);
       }
       cp_async_commit();
       cp_async_wait<0>();
       fence_proxy_async();  // the copies are visible to the tensor core (async proxy)
       __syncwarp();
       if (lane == 0) mbar_arrive(full_bar(ps));
-      cur = nxt;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) cur[g] = nxt[g];
     }
   } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------------ S issuer
     // the whole warp runs the loop (descriptor arithmetic stays warp-uniform); one
     // elected lane issues the tensor-core instructions
     const bool leader = elect_one();
@@ -232,88 +248,79 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     }
     __syncwarp();
     constexpr uint32_t idS = idesc_bf16_f32(64, kKeys);              // Q (K-major) x K (K-major)
-    constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true, false);  // V^T (M-major) x P (K-major)
     bool ok = mbar_wait(qfull_bar, 0, err, 22);
     const uint64_t dq = sdesc_kmajor_sw128(sQ);
-    const int leader_lane = __ffs(__ballot_sync(0xFFFFFFFFu, leader)) - 1;
-    // S(i) needs tile i in its stage and a free S buffer; PV(j) needs P(j).  Each is issued
-    // as soon as it can be, PV first: a stage is released by its PV.  The leader polls; the
-    // warp follows its decisions.
-    int is = 0, ipv = 0;
-    long long idle_since = clock64();
-    int spins = 0;
-    while (ok && ipv < ntiles) {
-      bool pv_ready = false, s_ready = false;
+    // S(i) needs tile i in its stage and a free S buffer.  PV is issued by its own warp, so
+    // a PV that becomes ready enters the tensor pipe between the MMAs of the next S
+    // instead of behind all of them.
+    for (int i = 0; i < ntiles && ok; ++i) {
+      const int st = i % kStages, sb = i & 1;
+      ok = mbar_wait(full_bar(st), (i / kStages) & 1, err, 24) &&
+           mbar_wait(sfree_bar(sb), ((i >> 1) & 1) ^ 1, err, 25);
+      if (!ok) break;
+      tc_fence_after();
+      const uint32_t dS = tmem + kTmemS + kKeys * sb;
+      // descriptors differ only in their start address: compile-time offsets from a base
+      const uint64_t dk = sdesc_kmajor_sw128(sStage + st * kStageBytes);
       if (leader) {
-        pv_ready = ipv < is && mbar_test_wait(pfull_bar(ipv % kStages), (ipv / kStages) & 1);
-        s_ready = is < ntiles && mbar_test_wait(full_bar(is % kStages), (is / kStages) & 1) &&
-                  mbar_test_wait(sfree_bar(is & 1), ((is >> 1) & 1) ^ 1);
-      }
-      pv_ready = __shfl_sync(0xFFFFFFFFu, pv_ready, leader_lane);
-      s_ready = __shfl_sync(0xFFFFFFFFu, s_ready, leader_lane);
-      if (pv_ready) {
-        const int jt = ipv, sj = jt % kStages;
-        tc_fence_after();
-        const uint64_t da = sdesc_mnmajor_sw128(sStage + sj * kStageBytes, kBlockBytes, 1024);
-        const uint64_t dp = sdesc_kmajor_sw128(sStage + sj * kStageBytes + kPBlock * kBlockBytes);
-        if (leader) {
 #pragma unroll
-          for (int mb = 0; mb < 4; ++mb)
-#pragma unroll
-            for (int ks = 0; ks < kKeys / 16; ++ks)
-              mma_bf16(tmem + kTmemO + 64 * mb, da + (uint64_t)(((2 * mb) * kBlockBytes + ks * 16 * 128) >> 4),
-                       dp + (uint64_t)((ks * 32) >> 4), idPV, (jt > 0 || ks > 0) ? 1u : 0u);
-          mma_commit(pfree_bar);
-          mma_commit(empty_bar(sj));
-        }
-        __syncwarp();
-        ++ipv;
+        for (int kk = 0; kk < 4 * kBlocks; ++kk)
+          mma_bf16(dS, dq + (uint64_t)((((kk >> 2) * kQBlockBytes) + (kk & 3) * 32) >> 4),
+                   dk + (uint64_t)((((kk >> 2) * kBlockBytes) + (kk & 3) * 32) >> 4), idS, kk > 0);
+        mma_commit(sfull_bar(sb));
       }
-      if (s_ready) {
-        const int i = is, st = i % kStages, sb = i & 1;
-        tc_fence_after();
-        const uint32_t dS = tmem + kTmemS + kKeys * sb;
-        // descriptors differ only in their start address: compile-time offsets from a base
-        const uint64_t dk = sdesc_kmajor_sw128(sStage + st * kStageBytes);
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < 4 * kBlocks; ++kk)
-            mma_bf16(dS, dq + (uint64_t)((((kk >> 2) * kQBlockBytes) + (kk & 3) * 32) >> 4),
-                     dk + (uint64_t)((((kk >> 2) * kBlockBytes) + (kk & 3) * 32) >> 4), idS, kk > 0);
-          mma_commit(sfull_bar(sb));
-        }
-        __syncwarp();
-        ++is;
-      }
-      if (pv_ready || s_ready) {
-        idle_since = clock64();
-        spins = 0;
-      } else if (++spins == 64) {
-        // bounded like every other wait: give up after kWaitLimitCycles without progress,
-        // or when another thread has already failed
-        spins = 0;
-        const bool late = __any_sync(0xFFFFFFFFu, clock64() - idle_since > kWaitLimitCycles);
-        const bool failed = __any_sync(0xFFFFFFFFu, *reinterpret_cast<volatile int*>(err) != 0);
-        if (late && leader) atomicCAS(err, 0, 23);
-        ok = !(late || failed);
-      }
+      __syncwarp();
     }
     if (leader) {
-      mma_commit(ofinal_bar);
-      if (!mbar_wait_drain(ofinal_bar, 0)) atomicCAS(err, 0, 26);
+      mma_commit(sdone_bar);
+      if (!mbar_wait_drain(sdone_bar, 0)) atomicCAS(err, 0, 26);
       // the query load has landed even when the loop gave up early
       mbar_wait_drain(qfull_bar, 0);
     }
     __syncwarp();
+  } else if (warp == kPvWarp) {
+    // ------------------------------------------------------------------ PV issuer
+    const bool leader = elect_one();
+    constexpr uint32_t idPV = idesc_bf16_f32(128, 64, true, false);  // V^T (M-major) x P (K-major)
+    bool ok = true;
+    for (int j = 0; j < ntiles && ok; ++j) {
+      const int sj = j % kStages;
+      ok = mbar_wait(pfull_bar(sj), (j / kStages) & 1, err, 23);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t da = sdesc_mnmajor_sw128(sStage + sj * kStageBytes, kBlockBytes, 1024);
+      const uint64_t dp = sdesc_kmajor_sw128(sStage + sj * kStageBytes + kPBlock * kBlockBytes);
+      if (leader) {
+#pragma unroll
+        for (int mb = 0; mb < 4; ++mb)
+#pragma unroll
+          for (int ks = 0; ks < kKeys / 16; ++ks)
+            mma_bf16(tmem + kTmemO + 64 * mb, da + (uint64_t)(((2 * mb) * kBlockBytes + ks * 16 * 128) >> 4),
+                     dp + (uint64_t)((ks * 32) >> 4), idPV, (j > 0 || ks > 0) ? 1u : 0u);
+        mma_commit(pfree_bar);
+        mma_commit(empty_bar(sj));  // the stage's rows and P are consumed
+      }
+      __syncwarp();
+    }
+    if (leader) {
+      mma_commit(ofinal_bar);
+      if (!mbar_wait_drain(ofinal_bar, 0)) atomicCAS(err, 0, 26);
+    }
+    __syncwarp();
   } else {
     // ------------------------------------------------------------------ softmax
+    // One 16-lane x 64-column TMEM load per tile gives every thread of the warp 32 logits:
+    // heads hA = 16 quarter + t/4 and hB = hA + 8, keys 8j + 2(t % 4) + {0, 1} (j < 8).  The
+    // four threads of a head hold identical copies of its running max (reduced over them
+    // with two shuffles) and partial sums of its normaliser.
     const int quarter = warp & 3;
-    const bool owner = lane < 16;                 // this thread's TMEM lane holds a head of S
-    const int head = 16 * quarter + (lane & 15);
+    const int c4 = lane & 3;
+    const int hA = 16 * quarter + (lane >> 2), hB = hA + 8;
     const uint32_t lane_addr = (uint32_t)(32 * quarter) << 16;
-    float m_used = -INFINITY, l_run = 0.f;
+    float mA = -INFINITY, mB = -INFINITY, lA = 0.f, lB = 0.f;
     uint32_t grp_phase = 0;
     bool ok = true;
+    unsigned char* pbase = smem + kOffStage + kPBlock * kBlockBytes;
     for (int i = 0; i < ntiles && ok; ++i) {
       const int sb = i & 1, s = i % kStages;
       ok = mbar_wait(sfull_bar(sb), (i >> 1) & 1, err, 27);
@@ -321,76 +328,64 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
       tc_fence_after();
       ok = mbar_wait(full_bar(s), (i / kStages) & 1, err, 28);  // orders the gather's mask write
       if (!ok) break;
-      const unsigned long long mask = s_mask[s];
+      // this thread's keys: 8j + 2 c4 + e; shifted so that bit 2j + e is key 8j + 2 c4 + e
+      const unsigned long long mask = s_mask[s] >> (2 * c4);
       float* alpha = s_alpha + 64 * (i & 1);
-      const uint32_t s_addr = tmem + lane_addr + kTmemS + kKeys * sb;
-      unsigned char* prow = smem + kOffStage + s * kStageBytes + kPBlock * kBlockBytes + head * 128;
-      // One pass over the tile's logits (TMEM loads slow the row gather down, so they are
-      // kept few): P is written with the running max, and the tile is redone with a new one
-      // only in the rare case that its max exceeds the running max by more than 2^8.  A
-      // head's first tile with a valid key takes its max first.  tcgen05.ld is warp-wide:
-      // every lane loads, the lanes that own a head use the values, and the decisions to
-      // take another pass are taken per warp.
-      auto tile_max = [&]() {
-        float mt = -INFINITY;
+      uint32_t r[32];
+      tmem_ld16x256b_x8(tmem + lane_addr + kTmemS + kKeys * sb, r);
+      tmem_ld_wait();
+      float tA = -INFINITY, tB = -INFINITY;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[32];
-          tmem_ld32(s_addr + 32 * hf, r);
-          tmem_ld_wait();
+      for (int j = 0; j < 8; ++j)
 #pragma unroll
-          for (int j = 0; j < 32; ++j)
-            if ((mask >> (32 * hf + j)) & 1ull) mt = fmaxf(mt, __uint_as_float(r[j]) * scale_log2);
+        for (int e = 0; e < 2; ++e) {
+          const bool v = (mask >> (8 * j + e)) & 1ull;
+          const float zA = v ? __uint_as_float(r[4 * j + e]) * scale_log2 : -INFINITY;
+          const float zB = v ? __uint_as_float(r[4 * j + 2 + e]) * scale_log2 : -INFINITY;
+          r[4 * j + e] = __float_as_uint(zA);
+          r[4 * j + 2 + e] = __float_as_uint(zB);
+          tA = fmaxf(tA, zA);
+          tB = fmaxf(tB, zB);
         }
-        return mt;
-      };
-      // writes this head's P row with reference mu; returns the row sum and the tile max
-      auto write_p = [&](float mu, float& mt) {
-        float ls = 0.f;
-        mt = -INFINITY;
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          uint32_t r[32];
-          tmem_ld32(s_addr + 32 * hf, r);
-          tmem_ld_wait();
-          if (owner) {
-            uint32_t packed[16];
-#pragma unroll
-            for (int j = 0; j < 32; j += 2) {
-              const bool v0 = (mask >> (32 * hf + j)) & 1ull, v1 = (mask >> (32 * hf + j + 1)) & 1ull;
-              const float z0 = __uint_as_float(r[j]) * scale_log2, z1 = __uint_as_float(r[j + 1]) * scale_log2;
-              mt = fmaxf(mt, v0 ? z0 : -INFINITY);
-              mt = fmaxf(mt, v1 ? z1 : -INFINITY);
-              const float p0 = v0 ? exp2f(z0 - mu) : 0.f;
-              const float p1 = v1 ? exp2f(z1 - mu) : 0.f;
-              ls += p0 + p1;
-              packed[j / 2] = pack_bf16x2(p0, p1);
-            }
-#pragma unroll
-            for (int c = 0; c < 4; ++c)
-              *reinterpret_cast<uint4*>(prow + (((4 * hf + c) ^ (head & 7)) << 4)) =
-                  make_uint4(packed[4 * c], packed[4 * c + 1], packed[4 * c + 2], packed[4 * c + 3]);
-          }
-        }
-        return ls;
-      };
-      if (__any_sync(0xFFFFFFFFu, owner && m_used == -INFINITY)) {
-        const float mt = tile_max();
-        if (m_used == -INFINITY) m_used = mt;  // O and l of this head are still zero
+      for (int o = 1; o < 4; o <<= 1) {
+        tA = fmaxf(tA, __shfl_xor_sync(0xFFFFFFFFu, tA, o));
+        tB = fmaxf(tB, __shfl_xor_sync(0xFFFFFFFFu, tB, o));
       }
-      float mt, ls = write_p(m_used == -INFINITY ? 0.f : m_used, mt);
-      float a = 1.f;
-      if (__any_sync(0xFFFFFFFFu, owner && mt > m_used + kRescaleLog2)) {
-        if (mt > m_used + kRescaleLog2) {
-          a = exp2f(m_used - mt);
-          m_used = mt;
-          l_run *= a;
+      // The running max moves only on a head's first tile with a valid key (O and l are
+      // still zero) or when the tile's max exceeds it by more than 2^8 (O is rescaled).
+      auto update = [&](float& m, float& l, float t) {
+        float a = 1.f;
+        if (m == -INFINITY) {
+          m = t;
+        } else if (t > m + kRescaleLog2) {
+          a = exp2f(m - t);
+          m = t;
+          l *= a;
         }
-        ls = write_p(m_used, mt);
+        return a;
+      };
+      const float aA = update(mA, lA, tA), aB = update(mB, lB, tB);
+      const float muA = mA == -INFINITY ? 0.f : mA, muB = mB == -INFINITY ? 0.f : mB;
+      unsigned char* prowA = pbase + s * kStageBytes + hA * 128 + 4 * c4;
+      unsigned char* prowB = pbase + s * kStageBytes + hB * 128 + 4 * c4;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float pA0 = exp2f(__uint_as_float(r[4 * j]) - muA), pA1 = exp2f(__uint_as_float(r[4 * j + 1]) - muA);
+        const float pB0 = exp2f(__uint_as_float(r[4 * j + 2]) - muB), pB1 = exp2f(__uint_as_float(r[4 * j + 3]) - muB);
+        lA += pA0 + pA1;
+        lB += pB0 + pB1;
+        // P rows are K-major with the 128-byte swizzle: 16-byte chunk j of row h sits at
+        // chunk j ^ (h % 8)
+        *reinterpret_cast<uint32_t*>(prowA + ((j ^ (hA & 7)) << 4)) = pack_bf16x2(pA0, pA1);
+        *reinterpret_cast<uint32_t*>(prowB + ((j ^ (hB & 7)) << 4)) = pack_bf16x2(pB0, pB1);
       }
-      if (owner) alpha[head] = a;
+      if (c4 == 0) {
+        alpha[hA] = aA;
+        alpha[hB] = aB;
+      }
       // one vote per warp: does any of its heads need O rescaled?
-      const uint32_t vote = __ballot_sync(0xFFFFFFFFu, owner && head < H && a != 1.f);
+      const uint32_t vote = __ballot_sync(0xFFFFFFFFu, (hA < H && aA != 1.f) || (hB < H && aB != 1.f));
       if (lane == 0) reinterpret_cast<volatile unsigned char*>(s_vote + (i & 1))[quarter] = vote != 0u ? 1 : 0;
       // every head's factor is known before O is touched
       mbar_arrive(grp_bar);
@@ -418,57 +413,50 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
           }
         tmem_st_wait();
       }
-      if (owner) {
-        l_run += ls;
-        fence_proxy_async();
-      }
+      fence_proxy_async();  // the P stores are visible to the tensor core (async proxy)
       // S of this tile has been read: its TMEM buffer is free for the next-but-one tile
       tc_fence_before();
       mbar_arrive(sfree_bar(sb));
       tc_fence_before();
       mbar_arrive(pfull_bar(s));
     }
-    if (owner) {
-      s_l[head] = l_run;
-      s_m[head] = m_used;
+    // the normaliser of each head: the sum of its four threads' partial sums
+#pragma unroll
+    for (int o = 1; o < 4; o <<= 1) {
+      lA += __shfl_xor_sync(0xFFFFFFFFu, lA, o);
+      lB += __shfl_xor_sync(0xFFFFFFFFu, lB, o);
+    }
+    if (c4 == 0) {
+      s_l[hA] = lA;
+      s_m[hA] = mA;
+      s_l[hB] = lB;
+      s_m[hB] = mB;
     }
   }
 
   // ------------------------------------------------------------------ split reduction
   //   out[h] = sum_s c_s[h] O_s[h],  c_s[h] = 2^(m_s[h] - M[h]) / sum_r 2^(m_r[h] - M[h]) l_r[h],
-  // M[h] = max_r m_r[h].  Each split publishes its (m, l) per head; after a cluster barrier
-  // it computes its own c_s from all of them.  Every thread passes the cluster barriers on
-  // every path (a failed wait above only skips work), so none of them can be left waiting.
+  // M[h] = max_r m_r[h].  Each split writes its unnormalised O straight from TMEM to its
+  // partial block (L2-resident) while its (m, l) stay in shared memory; after one cluster
+  // barrier split r reads every split's (m, l) through distributed shared memory, forms the
+  // c_s of all heads, and sums slice r of the [H][512] output over the partials.  A single
+  // split writes O / l directly.  Every thread passes the cluster barriers on every path (a
+  // failed wait above only skips work), so none of them can be left waiting.
   tc_fence_before();
-  cluster_sync();  // #1: (m, l) of every split published; this CTA's MMAs have completed
+  __syncthreads();  // (m, l) of this split published; its MMAs have completed
   tc_fence_after();
   if (threadIdx.x < 64) {
     const int h = threadIdx.x;
-    float mr[kMaxSplits], lr[kMaxSplits];
-    float M = -INFINITY;
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp) {
-      mr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_m + h), sp)) : -INFINITY;
-      lr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_l + h), sp)) : 0.f;
-      M = fmaxf(M, mr[sp]);
-    }
-    float den = 0.f, mine = 0.f;
-#pragma unroll
-    for (int sp = 0; sp < kMaxSplits; ++sp) {
-      const float e = mr[sp] == -INFINITY ? 0.f : exp2f(mr[sp] - M);
-      den += e * lr[sp];
-      if (sp == split) mine = e;
-    }
-    s_coef[h] = den > 0.f ? mine / den : 0.f;
+    s_coef[h] = nsplit > 1 ? 1.f : (s_l[h] > 0.f ? 1.f / s_l[h] : 0.f);
   }
   __syncthreads();  // s_coef
-  // O^T (TMEM lane = value dim, column = head), scaled by this split's coefficients, goes to
-  // global memory: the output itself for a single split, else this split's partial.  Twelve
-  // warps, three per TMEM lane quarter, take the eight 32-column chunks (value block mb,
-  // head half); for each head a warp writes 32 consecutive value dims (128 bytes).
+  // O^T (TMEM lane = value dim, column = head) goes to global memory: the output itself for
+  // a single split, else this split's partial.  Twelve warps, three per TMEM lane quarter,
+  // take the eight 32-column chunks (value block mb, head half); for each head a warp
+  // writes 32 consecutive value dims (128 bytes).
   float* dst = nsplit == 1 ? layers.out[layer] + (size_t)row * H * kDv
                            : partials + (((size_t)layer * gridDim.y + row) * nsplit + split) * kPartialFloats;
-  if (warp != kMmaWarp) {
+  if (warp != kMmaWarp && warp != kPvWarp) {
     const int quarter = warp & 3;
     const int jw = warp < kProducerWarps ? warp >> 2 : 2;
     const uint32_t lane_base = tmem + ((uint32_t)(32 * quarter) << 16) + kTmemO;
@@ -500,7 +488,30 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     }
   }
   if (nsplit > 1) {
-    cluster_sync();  // #2: every split's partial is in global memory
+    cluster_sync();  // every split's partial is in global memory and its (m, l) in shared memory
+    // c_s[h] of every split, from the (m, l) of all splits; s_cs[s][h] reuses the first
+    // stage's space (its tiles are consumed)
+    float* s_cs = reinterpret_cast<float*>(smem + kOffStage);
+    if (threadIdx.x < 64) {
+      const int h = threadIdx.x;
+      float mr[kMaxSplits], lr[kMaxSplits];
+      float M = -INFINITY;
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplits; ++sp) {
+        mr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_m + h), sp)) : -INFINITY;
+        lr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_l + h), sp)) : 0.f;
+        M = fmaxf(M, mr[sp]);
+      }
+      float den = 0.f;
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplits; ++sp) den += (mr[sp] == -INFINITY ? 0.f : exp2f(mr[sp] - M)) * lr[sp];
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplits; ++sp)
+        if (sp < nsplit) s_cs[sp * 64 + h] = (den > 0.f && mr[sp] != -INFINITY) ? exp2f(mr[sp] - M) / den : 0.f;
+    }
+    // this CTA has read the other splits' shared memory: they may exit once all have
+    cluster_arrive();
+    __syncthreads();  // s_cs
     // this split's slice of the output: float4 e = h * 128 + d / 4 of the [H][512] block
     const int total = H * (kDv / 4);
     const int e0 = (int)((long long)split * total / nsplit), e1 = (int)((long long)(split + 1) * total / nsplit);
@@ -510,27 +521,38 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     // two elements per thread at a time: all their partial loads are in flight together
     for (int e = e0 + (int)threadIdx.x; e < e1; e += 2 * kThreadsA) {
       const int e2 = e + kThreadsA;
+      const bool has2 = e2 < e1;
+      const int h = e >> 7, h2 = has2 ? e2 >> 7 : h;
+      float4 v[kMaxSplits], v2[kMaxSplits];
+#pragma unroll
+      for (int sp = 0; sp < kMaxSplits; ++sp) {
+        if (sp < nsplit) {
+          v[sp] = __ldcg(part + (size_t)sp * (kPartialFloats / 4) + e);
+          if (has2) v2[sp] = __ldcg(part + (size_t)sp * (kPartialFloats / 4) + e2);
+        }
+      }
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
 #pragma unroll
       for (int sp = 0; sp < kMaxSplits; ++sp) {
         if (sp < nsplit) {
-          const float4 v = __ldcg(part + (size_t)sp * (kPartialFloats / 4) + e);
-          const float4 v2 = e2 < e1 ? __ldcg(part + (size_t)sp * (kPartialFloats / 4) + e2) : acc2;
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
-          if (e2 < e1) {
-            acc2.x += v2.x;
-            acc2.y += v2.y;
-            acc2.z += v2.z;
-            acc2.w += v2.w;
+          const float c = s_cs[sp * 64 + h];
+          acc.x += c * v[sp].x;
+          acc.y += c * v[sp].y;
+          acc.z += c * v[sp].z;
+          acc.w += c * v[sp].w;
+          if (has2) {
+            const float c2 = s_cs[sp * 64 + h2];
+            acc2.x += c2 * v2[sp].x;
+            acc2.y += c2 * v2[sp].y;
+            acc2.z += c2 * v2[sp].z;
+            acc2.w += c2 * v2[sp].w;
           }
         }
       }
       out4[e] = acc;
-      if (e2 < e1) out4[e2] = acc2;
+      if (has2) out4[e2] = acc2;
     }
+    cluster_wait();
   }
   tc_fence_before();
   __syncthreads();

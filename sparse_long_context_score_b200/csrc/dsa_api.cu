@@ -72,9 +72,10 @@ bool heads_supported(int H) { return H == 16 || H == 32 || H == 48 || H == 64; }
 
 // One group call, checked.
 struct GroupCall {
-  const uint16_t* iq;
+  const void* iq;  // bf16 or (f8) E4M3 elements
   const float* w;
-  const uint16_t* ik;
+  const void* ik;
+  bool f8;
   AttnLayers layers;
   int L, B, T, N, H, k, compute_indices;
   long long q_pos0;
@@ -82,7 +83,7 @@ struct GroupCall {
   int32_t* idx;
 };
 
-dsa_status check_group(const uint16_t* iq, const float* w, const uint16_t* ik, const uint16_t* const* q,
+dsa_status check_group(const void* iq, const float* w, const void* ik, bool f8, const uint16_t* const* q,
                        const uint16_t* const* kv, int L, int B, int T, int N, int H, int k, int compute_indices,
                        int32_t* idx_shared, float* const* out, GroupCall* c) {
   if (!q || !kv || !out || !idx_shared || !sizes_ok(B, T, N) || k <= 0 || H <= 0 || L <= 0)
@@ -101,6 +102,7 @@ dsa_status check_group(const uint16_t* iq, const float* w, const uint16_t* ik, c
   c->iq = iq;
   c->w = w;
   c->ik = ik;
+  c->f8 = f8;
   c->L = L;
   c->B = B;
   c->T = T;
@@ -130,7 +132,7 @@ cudaError_t enqueue_group(const GroupCall& c, unsigned char* base, const GroupLa
     const bool fused_hist = c.T == 1 && c.B <= cap;
     if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess) return e;
     if ((e = launch_index_score_tc(c.iq, c.w, c.ik, c.B, c.T, c.N, c.q_pos0, scores, fused_hist ? tws.hist : nullptr,
-                                   idx_sms, stream)) != cudaSuccess)
+                                   idx_sms, c.f8, stream)) != cudaSuccess)
       return e;
     if (after_idx && (e = cudaEventRecord(after_idx, stream)) != cudaSuccess) return e;
     if ((e = launch_topk(scores, c.B, c.T, c.N, c.q_pos0, c.k, c.idx, tws, fused_hist, tail_sms, stream)) != cudaSuccess)
@@ -237,7 +239,14 @@ dsa_status dsa_index_score(const uint16_t* q, const float* w, const uint16_t* k,
                            long long q_pos0, float* scores, cudaStream_t stream) {
   if (!q || !w || !k || !scores || !sizes_ok(B, T, N)) return DSA_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 16) || !aligned(scores, 4)) return DSA_ERR_INVALID_ARG;
-  return cuda_status(launch_index_score_tc(q, w, k, B, T, N, q_pos0, scores, nullptr, 0, stream));
+  return cuda_status(launch_index_score_tc(q, w, k, B, T, N, q_pos0, scores, nullptr, 0, false, stream));
+}
+
+dsa_status dsa_index_score_e4m3(const uint8_t* q, const float* w, const uint8_t* k, int B, int T, int N,
+                                long long q_pos0, float* scores, cudaStream_t stream) {
+  if (!q || !w || !k || !scores || !sizes_ok(B, T, N)) return DSA_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(w, 16) || !aligned(scores, 4)) return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_index_score_tc(q, w, k, B, T, N, q_pos0, scores, nullptr, 0, true, stream));
 }
 
 dsa_status dsa_topk(const float* scores, int B, int T, int N, long long q_pos0, int k, int32_t* idx, void* workspace,
@@ -273,7 +282,7 @@ dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t*
                              float scale, int compute_indices, int32_t* idx_shared, float* const* out, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream) {
   GroupCall c{};
-  const dsa_status st = check_group(iq, w, ik, q, kv, L, B, T, N, H, k, compute_indices, idx_shared, out, &c);
+  const dsa_status st = check_group(iq, w, ik, false, q, kv, L, B, T, N, H, k, compute_indices, idx_shared, out, &c);
   if (st != DSA_OK) return st;
   c.q_pos0 = q_pos0;
   c.scale = scale;
@@ -317,9 +326,14 @@ dsa_status dsa_decode_step(const dsa_group_io* groups, int G, int L, int B, int 
         outs[l] = io.out[l] + (size_t)b0 * H * kDv;
       }
       if (!io.iq || !io.w || !io.ik || !io.idx) return DSA_ERR_INVALID_ARG;
-      const dsa_status st = check_group(io.iq + (size_t)b0 * kIndexHeads * kIndexDim, io.w + (size_t)b0 * kIndexHeads,
-                                        io.ik + (size_t)b0 * N * kIndexDim, qs, kvs, L, bn, 1, N, H, k, 1,
-                                        io.idx + (size_t)b0 * k, outs, &c);
+      if (io.index_format != DSA_INDEX_BF16 && io.index_format != DSA_INDEX_E4M3) return DSA_ERR_UNSUPPORTED;
+      const bool f8 = io.index_format == DSA_INDEX_E4M3;
+      const size_t esz = f8 ? 1 : 2;
+      const dsa_status st =
+          check_group(static_cast<const unsigned char*>(io.iq) + (size_t)b0 * kIndexHeads * kIndexDim * esz,
+                      io.w + (size_t)b0 * kIndexHeads,
+                      static_cast<const unsigned char*>(io.ik) + (size_t)b0 * N * kIndexDim * esz, f8, qs, kvs, L, bn,
+                      1, N, H, k, 1, io.idx + (size_t)b0 * k, outs, &c);
       if (st != DSA_OK) return st;
       c.q_pos0 = N - 1;
       c.scale = scale;

@@ -102,8 +102,9 @@ size_t attn_workspace_bytes(long long rows, int L, int H, int k, int sm_budget =
 
 // tcgen05 indexer (T == 1: decode, one query per MMA; T > 1: 8 queries per MMA).  With a
 // histogram pointer (decode only, B <= 148) the first radix digit of the select is counted.
-cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
-                                  long long q_pos0, float* scores, uint32_t* hist, int sm_budget, cudaStream_t stream);
+// f8: q and k hold E4M3 bytes instead of bf16 (the same layouts, one byte per element).
+cudaError_t launch_index_score_tc(const void* q, const float* w, const void* k, int B, int T, int N, long long q_pos0,
+                                  float* scores, uint32_t* hist, int sm_budget, bool f8, cudaStream_t stream);
 // Device addresses of the error words: the indexer's and the attention's bounded waits
 // record a code when they run out; the top-k records one when a selection invariant
 // fails (the selected count is not k).  0 = none.

@@ -10,19 +10,19 @@
 //
 // Warp roles (one CTA per SM, persistent over a contiguous range of (query group, key
 // tile) items):
-//   warp 0      TMA producer: 128x128 bf16 key tiles (two 64-column boxes, 128-byte
-//               swizzle) into a ring of shared-memory stages; the query group once per
-//               group change;
-//   warp 1      allocates TMEM; one thread issues tcgen05.mma into one of two TMEM
-//               accumulators (2 x 32*QG columns) and commits to the stage / accumulator
-//               barriers;
-//   warps 2..   epilogue (4 warps in decode, 8 in prefill: two per TMEM lane quarter, each
-//               scoring 4 of the 8 queries): each thread owns one key row of the
-//               accumulator (its warp's TMEM lane quarter), loads the 32 head columns of a
-//               query, applies ReLU and the head weights, sums, and stores the score
-//               (coalesced: a warp writes 32 consecutive keys).  In decode it can also
-//               count the first radix digit of each score into a per-row histogram for the
-//               top-k select.
+//   warp 0      TMA producer: 128x128 key tiles (bf16: two 64-column boxes; E4M3: one
+//               128-column box; 128-byte swizzle) into a ring of shared-memory stages; the
+//               query group once per group change;
+//   warp 1      allocates TMEM; one thread issues tcgen05.mma into a ring of TMEM
+//               accumulators (decode: 4 x 32 columns; prefill: 2 x 256) and commits to the
+//               stage / accumulator barriers;
+//   warps 2..9  epilogue, two warps per TMEM lane quarter (decode: the two take alternate
+//               tiles, so two tiles are scored at once; prefill: each scores 4 of the 8
+//               queries): each thread owns one key row of the accumulator (its warp's TMEM
+//               lane quarter), loads the 32 head columns of a query, applies ReLU and the
+//               head weights, sums, and stores the score (coalesced: a warp writes 32
+//               consecutive keys).  In decode it can also count the first radix digit of
+//               each score into a per-row histogram for the top-k select.
 // Every mbarrier wait is bounded (see sm100.cuh); a timeout sets the device error word.
 #include <cudaTypedefs.h>
 
@@ -39,23 +39,30 @@ using namespace sm100;
 static __device__ int g_indexer_tc_error;
 
 constexpr int kTileKeys = 128;
-constexpr int kHalfBytesA = kTileKeys * 128;  // 128 rows x 64 bf16 = 16 KB
-constexpr int kStageBytesA = 2 * kHalfBytesA;
+constexpr int kHalfBytesA = kTileKeys * 128;  // 128 rows x 128 bytes (64 bf16 or 128 E4M3) = 16 KB
 
-template <int QG, bool kHist>
+// kF8: keys and queries in E4M3 (one 128-byte box per row, kind::f8f6f4 MMAs of K = 32);
+// otherwise bf16 (two 64-column boxes per row, kind::f16 MMAs of K = 16)
+template <int QG, bool kHist, bool kF8 = false>
 struct TcCfg {
-  static constexpr int kEpiWarps = QG == 1 ? 4 : 8;   // prefill: two warps per TMEM lane quarter
+  // 8 epilogue warps, two per TMEM lane quarter: in decode the two take alternate tiles
+  // (four accumulators, so the MMA runs up to four tiles ahead of the epilogue); in
+  // prefill the two split the tile's 8 queries (two accumulators of 256 columns)
+  static constexpr int kEpiWarps = 8;
+  static constexpr int kAccBufs = QG == 1 ? 4 : 2;
   static constexpr int kThreads = 64 + 32 * kEpiWarps;
   static constexpr int kN = 32 * QG;                  // MMA N
-  static constexpr int kStages = QG == 1 ? 5 : 4;
+  static constexpr int kHalves = kF8 ? 1 : 2;         // 128-byte column boxes per 128-wide row
+  static constexpr int kStageBytesA = kHalves * kHalfBytesA;
+  static constexpr int kStages = kF8 ? (QG == 1 ? 10 : 8) : (QG == 1 ? 5 : 4);  // same bytes in flight
   static constexpr int kHalfBytesB = kN * 128;
-  static constexpr int kBytesB = 2 * kHalfBytesB;
-  static constexpr int kTmemCols = (2 * kN) < 32 ? 32 : 2 * kN;  // power of two for QG in {1, 8}
+  static constexpr int kBytesB = kHalves * kHalfBytesB;
+  static constexpr int kTmemCols = kAccBufs * kN;  // 128 or 512: a power of two >= 32
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kStageBytesA;
   static constexpr int kOffHist = kOffB + kBytesB;     // two row histograms (a CTA spans <= 2 rows)
   static constexpr int kOffBar = kOffHist + (kHist ? 2 * kHistBins * 4 : 0);
-  static constexpr int kNumBars = 2 * kStages + 4 + 3;
+  static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 3;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffTmem + 16 + 1024;  // + alignment slack
   static_assert(kSmem <= 232448, "shared memory budget");
@@ -105,12 +112,12 @@ struct Cursor {
   }
 };
 
-template <int QG, bool kHist>
-__global__ void __launch_bounds__(TcCfg<QG, kHist>::kThreads, 1)
+template <int QG, bool kHist, bool kF8>
+__global__ void __launch_bounds__(TcCfg<QG, kHist, kF8>::kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                   const float* __restrict__ w, int B, int T, int N, long long q_pos0, long long total_items,
                   float* __restrict__ scores, uint32_t* __restrict__ hist, int* __restrict__ err) {
-  using C = TcCfg<QG, kHist>;
+  using C = TcCfg<QG, kHist, kF8>;
   grid_dep_launch();  // the top-k may be scheduled as SMs free up; it waits for these scores
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -122,10 +129,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   auto full_bar = [&](int s) { return bar0 + 8u * s; };
   auto empty_bar = [&](int s) { return bar0 + 8u * (C::kStages + s); };
   auto tfull_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + b); };
-  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + 2 + b); };
-  const uint32_t qfull_bar = bar0 + 8u * (2 * C::kStages + 4);
-  const uint32_t qfree_bar = bar0 + 8u * (2 * C::kStages + 5);
-  const uint32_t done_bar = bar0 + 8u * (2 * C::kStages + 6);
+  auto tempty_bar = [&](int b) { return bar0 + 8u * (2 * C::kStages + C::kAccBufs + b); };
+  const uint32_t qfull_bar = bar0 + 8u * (2 * C::kStages + 2 * C::kAccBufs);
+  const uint32_t qfree_bar = bar0 + 8u * (2 * C::kStages + 2 * C::kAccBufs + 1);
+  const uint32_t done_bar = bar0 + 8u * (2 * C::kStages + 2 * C::kAccBufs + 2);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffTmem);
 
   const int warp = threadIdx.x >> 5;
@@ -141,9 +148,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       mbar_init(full_bar(s), 1);
       mbar_init(empty_bar(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(tfull_bar(b), 1);
-      mbar_init(tempty_bar(b), 32 * C::kEpiWarps);
+      mbar_init(tempty_bar(b), QG == 1 ? 32 * C::kEpiWarps / 2 : 32 * C::kEpiWarps);  // decode: one warp group per tile
     }
     mbar_init(qfull_bar, 1);
     mbar_init(qfree_bar, 1);
@@ -183,8 +190,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
           }
           const int b = cur.qg / it.G, t0 = (cur.qg % it.G) * QG;
           mbar_arrive_expect_tx(qfull_bar, C::kBytesB);
-          tma_load_3d(sB, &qmap, qfull_bar, 0, t0 * 32, b);
-          tma_load_3d(sB + C::kHalfBytesB, &qmap, qfull_bar, 64, t0 * 32, b);
+          for (int hh = 0; hh < C::kHalves; ++hh) tma_load_3d(sB + hh * C::kHalfBytesB, &qmap, qfull_bar, 64 * hh, t0 * 32, b);
           q_pending = true;
           q_parity = (cur_qg >= 0) ? (q_parity ^ 1) : 0;
           cur_qg = cur.qg;
@@ -192,10 +198,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         ok = mbar_wait(empty_bar(stage), phase ^ 1, err, 2);
         if (!ok) break;
         const int b = cur.qg / it.G;
-        const uint32_t dst = sA + stage * kStageBytesA;
-        mbar_arrive_expect_tx(full_bar(stage), kStageBytesA);
-        tma_load_3d(dst, &kmap, full_bar(stage), 0, cur.tile * kTileKeys, b);
-        tma_load_3d(dst + kHalfBytesA, &kmap, full_bar(stage), 64, cur.tile * kTileKeys, b);
+        const uint32_t dst = sA + stage * C::kStageBytesA;
+        mbar_arrive_expect_tx(full_bar(stage), C::kStageBytesA);
+        for (int hh = 0; hh < C::kHalves; ++hh)
+          tma_load_3d(dst + hh * kHalfBytesA, &kmap, full_bar(stage), 64 * hh, cur.tile * kTileKeys, b);
         ++issued;
         if (++stage == C::kStages) {
           stage = 0;
@@ -215,7 +221,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     // the whole warp runs the loop (descriptor arithmetic stays warp-uniform); one
     // elected lane issues the tensor-core instructions
     const bool leader = elect_one();
-    constexpr uint32_t idesc = idesc_bf16_f32(kTileKeys, C::kN);
+    constexpr uint32_t idesc = kF8 ? idesc_e4m3_f32(kTileKeys, C::kN) : idesc_bf16_f32(kTileKeys, C::kN);
     Cursor cur;
     cur.start(it, begin, end);
     int stage = 0;
@@ -233,8 +239,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         if (!ok) break;
         cur_qg = cur.qg;
       }
-      const int buf = (int)(acc & 1);
-      const uint32_t use = (uint32_t)(acc >> 1);
+      const int buf = (int)(acc % C::kAccBufs);
+      const uint32_t use = (uint32_t)(acc / C::kAccBufs);
       ok = mbar_wait(tempty_bar(buf), (use & 1) ^ 1, err, 5);
       if (!ok) break;
       tc_fence_after();
@@ -242,14 +248,20 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
       if (!ok) break;
       tc_fence_after();
       const uint32_t d = tmem_base + buf * C::kN;
-      const uint64_t ad0 = sdesc_kmajor_sw128(sA + stage * kStageBytesA);
+      const uint64_t ad0 = sdesc_kmajor_sw128(sA + stage * C::kStageBytesA);
       if (leader) {
+        // each MMA takes 32 bytes of K: 16 bf16 or 32 E4M3 values
 #pragma unroll
-        for (int kh = 0; kh < 2; ++kh)
+        for (int kh = 0; kh < C::kHalves; ++kh)
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(d, ad0 + (uint64_t)((kh * kHalfBytesA + ks * 32) >> 4),
-                     bd0 + (uint64_t)((kh * C::kHalfBytesB + ks * 32) >> 4), idesc, (kh | ks) != 0);
+          for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t a = ad0 + (uint64_t)((kh * kHalfBytesA + ks * 32) >> 4);
+            const uint64_t bb = bd0 + (uint64_t)((kh * C::kHalfBytesB + ks * 32) >> 4);
+            if (kF8)
+              mma_e4m3(d, a, bb, idesc, (kh | ks) != 0);
+            else
+              mma_bf16(d, a, bb, idesc, (kh | ks) != 0);
+          }
         mma_commit(empty_bar(stage));
         mma_commit(tfull_bar(buf));
       }
@@ -270,7 +282,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
   } else {
     // ------------------------------------------------------------------ epilogue
     const int quarter = warp & 3;  // TMEM lanes [32*quarter, 32*quarter + 32)
-    const int qhalf = (warp - 2) >> 2;  // prefill: which half of the 8 queries this warp scores
+    const int qhalf = (warp - 2) >> 2;  // prefill: which half of the 8 queries this warp scores;
+                                        // decode: which of two alternate tiles it scores
     const int row_in_tile = 32 * quarter + lane;
     Cursor cur;
     cur.start(it, begin, end);
@@ -280,6 +293,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     float wr[32];  // head weights of the current query (decode)
     bool ok = true;
     while (cur.valid() && ok) {
+      if (QG == 1 && (int)(acc & 1) != qhalf) {  // the other warp group's tile
+        ++acc;
+        cur.next(it);
+        continue;
+      }
       const int b = cur.qg / it.G, t0 = (cur.qg % it.G) * QG;
       if (QG == 1 && cur.qg != cur_qg) {
         const float* wq = w + ((size_t)b * T + t0) * 32;
@@ -287,8 +305,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         for (int h = 0; h < 32; ++h) wr[h] = __ldg(&wq[h]);
         cur_qg = cur.qg;
       }
-      const int buf = (int)(acc & 1);
-      const uint32_t use = (uint32_t)(acc >> 1);
+      const int buf = (int)(acc % C::kAccBufs);
+      const uint32_t use = (uint32_t)(acc / C::kAccBufs);
       ok = mbar_wait(tfull_bar(buf), use & 1, err, 8);
       if (!ok) break;
       tc_fence_after();
@@ -375,35 +393,38 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map over [d2][d1][128] with a box of 64 x rows x 1 and 128-byte swizzle
-bool make_map(CUtensorMap* map, const void* base, long long d1, long long d2, int rows) {
+// 3-D map over [d2][d1][128 values] with a box of one 128-byte column block x rows x 1 and
+// the 128-byte swizzle: bf16 (64-value blocks) or E4M3 bytes (128-value blocks)
+bool make_map(CUtensorMap* map, const void* base, long long d1, long long d2, int rows, bool f8) {
   auto fn = encode_fn();
   if (!fn) return false;
+  const int esz = f8 ? 1 : 2;
   cuuint64_t dims[3] = {128, (cuuint64_t)d1, (cuuint64_t)d2};
-  cuuint64_t strides[2] = {256, (cuuint64_t)d1 * 256};
-  cuuint32_t box[3] = {64, (cuuint32_t)rows, 1};
+  cuuint64_t strides[2] = {(cuuint64_t)128 * esz, (cuuint64_t)d1 * 128 * esz};
+  cuuint32_t box[3] = {(cuuint32_t)(128 / esz), (cuuint32_t)rows, 1};
   cuuint32_t estr[3] = {1, 1, 1};
-  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  const CUresult r = fn(map, f8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
 SymbolAddress g_err_addr;
 
-template <int QG, bool kHist>
-cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N, long long q_pos0,
+template <int QG, bool kHist, bool kF8>
+cudaError_t launch_tc(const void* q, const float* w, const void* k, int B, int T, int N, long long q_pos0,
                       float* scores, uint32_t* hist, int sm_budget, cudaStream_t stream) {
-  using C = TcCfg<QG, kHist>;
+  using C = TcCfg<QG, kHist, kF8>;
   CUtensorMap kmap, qmap;
-  if (!make_map(&kmap, k, N, B, kTileKeys) || !make_map(&qmap, q, (long long)T * 32, B, C::kN))
+  if (!make_map(&kmap, k, N, B, kTileKeys, kF8) || !make_map(&qmap, q, (long long)T * 32, B, C::kN, kF8))
     return cudaErrorInvalidValue;
   int* err = nullptr;
   cudaError_t e = g_err_addr.get(g_indexer_tc_error, &err);
   if (e != cudaSuccess) return e;
   static DeviceOnce once;
   if ((e = once.run([] {
-         return cudaFuncSetAttribute(indexer_tc_kernel<QG, kHist>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+         return cudaFuncSetAttribute(indexer_tc_kernel<QG, kHist, kF8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::kSmem);
        })) != cudaSuccess)
     return e;
   // items = sum over query groups of the key tiles they see
@@ -421,27 +442,31 @@ cudaError_t launch_tc(const uint16_t* q, const float* w, const uint16_t* k, int 
   if (sms <= 0) return cudaErrorInvalidDevice;
   const int cap = sm_budget > 0 && sm_budget < sms ? sm_budget : sms;
   const int grid = (int)(total < cap ? total : cap);
-  indexer_tc_kernel<QG, kHist><<<grid, C::kThreads, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
+  indexer_tc_kernel<QG, kHist, kF8><<<grid, C::kThreads, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
                                                                        hist, err);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_index_score_tc(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
-                                  long long q_pos0, float* scores, uint32_t* hist, int sm_budget,
-                                  cudaStream_t stream) {
+cudaError_t launch_index_score_tc(const void* q, const float* w, const void* k, int B, int T, int N, long long q_pos0,
+                                  float* scores, uint32_t* hist, int sm_budget, bool f8, cudaStream_t stream) {
   // the fused histogram keeps two row slots per CTA: with contiguous item ranges over at
   // most one CTA per SM of the budget, a range spans at most two sequences when B is no
   // more than the CTAs
   const int sms = device_sm_count();
   const int cap = sm_budget > 0 && sm_budget < sms ? sm_budget : sms;
   if (hist && (T != 1 || B > cap)) return cudaErrorNotSupported;
-  if (T == 1) {
-    return hist ? launch_tc<1, true>(q, w, k, B, T, N, q_pos0, scores, hist, sm_budget, stream)
-                : launch_tc<1, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
+  if (f8) {
+    if (T == 1)
+      return hist ? launch_tc<1, true, true>(q, w, k, B, T, N, q_pos0, scores, hist, sm_budget, stream)
+                  : launch_tc<1, false, true>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
+    return launch_tc<8, false, true>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
   }
-  return launch_tc<8, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
+  if (T == 1)
+    return hist ? launch_tc<1, true, false>(q, w, k, B, T, N, q_pos0, scores, hist, sm_budget, stream)
+                : launch_tc<1, false, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
+  return launch_tc<8, false, false>(q, w, k, B, T, N, q_pos0, scores, nullptr, sm_budget, stream);
 }
 
 cudaError_t indexer_error_word(int** p) { return g_err_addr.get(g_indexer_tc_error, p); }

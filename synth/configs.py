@@ -36,6 +36,7 @@ class Workload:
     L: int               # layers per IndexShare group (attention calls per index list)
     groups: int = 1      # IndexShare groups run in sequence
     steps: int = 1       # MTP draft steps (steps 2.. reuse the step-1 indices)
+    index_fp8: bool = False  # index keys and indexer queries as E4M3 bytes instead of bf16
     note: str = ""
 
     @property
@@ -63,6 +64,9 @@ WORKLOADS = {
     # the step-1 query sits at the last target position, so the draft rows are never visible.
     "mtp": Workload("mtp", 5, B=16, T=1, N=262144 + 7, q_pos0=262143, k=2048, H=64, L=1,
                     steps=7, note="MTP drafting, 1 layer, 7 draft steps reusing step-1 indices"),
+    # decode at 128K over an FP8 (E4M3) index-key cache: the same integers as decode128k
+    "decode128k_fp8": Workload("decode128k_fp8", 2, B=8, T=1, N=131072, q_pos0=131071, k=2048, H=64, L=4,
+                               index_fp8=True, note="decode at 128K, E4M3 index keys and queries"),
 }
 
 

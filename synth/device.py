@@ -31,7 +31,7 @@ def lib():
     global _lib
     if _lib is None:
         _lib = ctypes.CDLL(build())
-        for name in ("synth_fill_int17_bf16", "synth_fill_pow2_f32", "synth_fill_normal_bf16",
+        for name in ("synth_fill_int17_bf16", "synth_fill_int17_e4m3", "synth_fill_pow2_f32", "synth_fill_normal_bf16",
                      "synth_fill_unit_f32"):
             fn = getattr(_lib, name)
             fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.c_uint64, ctypes.c_int64,
@@ -53,6 +53,12 @@ def _fill(name, tensor, key, offset=0):
 def int17_bf16(tensor, key, offset=0):
     """tensor: contiguous torch.bfloat16 (or int16) CUDA tensor, filled in place."""
     return _fill("synth_fill_int17_bf16", tensor, key, offset)
+
+
+def int17_e4m3(tensor, key, offset=0):
+    """tensor: contiguous torch.uint8 CUDA tensor, filled in place with the integers of
+    int17_bf16 (same key, same draws) as E4M3 bytes."""
+    return _fill("synth_fill_int17_e4m3", tensor, key, offset)
 
 
 def pow2_f32(tensor, key, offset=0):

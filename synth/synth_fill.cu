@@ -34,6 +34,17 @@ __global__ void fill_int17_bf16(uint16_t* out, int64_t n, uint64_t key, int64_t 
   }
 }
 
+// E4M3 bytes of the integers 0..8 (1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits)
+__constant__ uint8_t kE4M3OfInt[9] = {0x00, 0x38, 0x40, 0x44, 0x48, 0x4A, 0x4C, 0x4E, 0x50};
+
+__global__ void fill_int17_e4m3(uint8_t* out, int64_t n, uint64_t key, int64_t offset) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    uint64_t h = draw(key, (uint64_t)(offset + i));
+    int v = (int)((h >> 32) % 17u) - 8;
+    out[i] = (uint8_t)(kE4M3OfInt[v < 0 ? -v : v] | (v < 0 ? 0x80 : 0));
+  }
+}
+
 __global__ void fill_pow2_f32(float* out, int64_t n, uint64_t key, int64_t offset) {
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
     uint64_t h = draw(key, (uint64_t)(offset + i));
@@ -78,6 +89,11 @@ extern "C" {
 int synth_fill_int17_bf16(void* out, int64_t n, uint64_t key, int64_t offset, cudaStream_t s) {
   if (n <= 0) return 0;
   fill_int17_bf16<<<grid_for(n), 256, 0, s>>>((uint16_t*)out, n, key, offset);
+  return (int)cudaGetLastError();
+}
+int synth_fill_int17_e4m3(void* out, int64_t n, uint64_t key, int64_t offset, cudaStream_t s) {
+  if (n <= 0) return 0;
+  fill_int17_e4m3<<<grid_for(n), 256, 0, s>>>((uint8_t*)out, n, key, offset);
   return (int)cudaGetLastError();
 }
 int synth_fill_pow2_f32(void* out, int64_t n, uint64_t key, int64_t offset, cudaStream_t s) {
