@@ -42,10 +42,11 @@ def parse():
     p.add_argument("--cpu-sample", type=int, default=2, help="sequences in the CPU-oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra", action="store_true", help="skip the 1M / MTP / prefill workloads")
-    p.add_argument("--schedule", default="micro", choices=["micro", "sequential"],
-                   help="decode workloads: dsa_decode_step (two micro-batches on two streams) or one "
-                        "dsa_group_forward per group in order on one stream")
-    p.add_argument("--ncu-case", choices=["indexer", "topk", "attn", "indexer_prefill", "attn_mtp", "topk_1m"],
+    p.add_argument("--schedule", default="sequential", choices=["micro", "sequential"],
+                   help="decode workloads: one dsa_group_forward per group in order on one stream (the "
+                        "faster on B200), or dsa_decode_step (two micro-batches on two streams)")
+    p.add_argument("--ncu-case", choices=["indexer", "topk", "attn", "indexer_prefill", "attn_mtp", "topk_1m",
+                                          "indexer_fp8"],
                    help="run one kernel of the decode step a few times on a profiler-sized case and exit "
                         "(for ncu captures; prints no benchmark line)")
     return p.parse_args()
@@ -255,9 +256,11 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     dsa.lib()
     groups = make_inputs(w, device, rank)
     micro = args.schedule == "micro" and w.T == 1 and w.steps == 1 and w.B >= 2
-    if w.index_fp8 and not micro:
-        raise ValueError("the E4M3 index format runs through the micro-batched decode step only")
-    ws = dsa.decode_workspace(w.B, w.N, w.k, w.H, w.L, device) if micro else \
+    # the E4M3 index format runs through dsa_decode_step (in order: side = stream)
+    use_step = micro or (w.index_fp8 and w.T == 1 and w.steps == 1)
+    if w.index_fp8 and not use_step:
+        raise ValueError("the E4M3 index format runs through the decode step only")
+    ws = dsa.decode_workspace(w.B, w.N, w.k, w.H, w.L, device) if use_step else \
         dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, device)
     stream = torch.cuda.Stream(device)
     side = torch.cuda.Stream(device)
@@ -273,8 +276,8 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         flush_rd.view(torch.int64).sum()
 
     def step():
-        if micro:
-            dsa.dsa_decode_step(dgroups, w.k, C.SCALE, ws=ws, stream=stream, side=side)
+        if use_step:
+            dsa.dsa_decode_step(dgroups, w.k, C.SCALE, ws=ws, stream=stream, side=side if micro else stream)
             return
         for g in groups:
             dsa.dsa_group_forward(g["iq"], g["wt"], g["ik"], g["qs"], g["kvs"], w.q_pos0, w.k, C.SCALE,
@@ -324,7 +327,8 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     res = {"step_ms": sum(times) / len(times), "clocks": clk.summary(),
-           "schedule": "two micro-batches (dsa_decode_step)" if micro else "groups in order (dsa_group_forward)"}
+           "schedule": "two micro-batches (dsa_decode_step)" if micro else
+           "groups in order (dsa_decode_step, side = stream)" if use_step else "groups in order (dsa_group_forward)"}
 
     # the dominant kernel alone: the indexer over the first group's cache, same launch shape
     g0 = groups[0]
@@ -545,6 +549,7 @@ def step_launches(w, micro: bool) -> int:
 def ncu_case(kind: str) -> None:
     """A few launches of one kernel, sized for an ncu capture (a few GB on the device):
       indexer, topk   the decode128k shapes (268 MB of keys, 4 MB of scores);
+      indexer_fp8     the decode128k indexer over E4M3 keys and queries (134 MB of keys);
       attn            32 (row, layer) units as in the decode128k step (4 key splits each)
                       over caches of 65536 rows (2.4 GB, larger than L2);
       attn_mtp        16 units as in an MTP draft step, run once first so that the 37.7 MB
@@ -574,6 +579,13 @@ def ncu_case(kind: str) -> None:
                 dsa.dsa_index_score(iq, wt, ik, w.q_pos0, scores=sc)
             else:
                 dsa.dsa_topk(sc, w.q_pos0, w.k, idx=idx, ws=ws)
+    elif kind == "indexer_fp8":
+        iq = sd.int17_e4m3(torch.empty(w.B, 1, 32, 128, dtype=torch.uint8, device="cuda"), w.key(synth.KIND_IQ))
+        wt = sd.pow2_f32(torch.empty(w.B, 1, 32, dtype=torch.float32, device="cuda"), w.key(synth.KIND_W))
+        ik = sd.int17_e4m3(torch.empty(w.B, w.N, 128, dtype=torch.uint8, device="cuda"), w.key(synth.KIND_IK))
+        sc = torch.empty(w.B, 1, w.N, dtype=torch.float32, device="cuda")
+        for _ in range(launches + 1):
+            dsa.dsa_index_score_e4m3(iq, wt, ik, w.q_pos0, scores=sc)
     elif kind == "indexer_prefill":
         wp = C.WORKLOADS["prefill"]
         T = 512

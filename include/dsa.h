@@ -217,8 +217,11 @@ dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t 
  * groups in order (group g+1's indexer after group g's attention, as in a model).  The
  * HBM-bound indexers of the two micro-batches take turns (each waits for the other's
  * previous one) on about two thirds of the SMs, and each micro-batch's top-k and
- * attention run beside the other's indexer on the remaining third.  With B = 1 the groups
- * run in order on `stream`.
+ * attention run beside the other's indexer on the remaining third.  With B = 1, or with
+ * side == stream, the groups run in order over the whole batch on `stream`, exactly like
+ * one dsa_group_forward per group (on B200 this in-order step is the faster of the two at
+ * the decode shapes measured: the top-k and attention are latency-bound and take nearly
+ * as long for half a batch as for all of it).
  *   groups[g]   the group's tensors for all B sequences, in the layouts of
  *               dsa_group_forward with T = 1 (q, kv, out: L entries each)
  *   workspace   dsa_decode_workspace_size(B, N, k, H, L) bytes, 256-byte aligned

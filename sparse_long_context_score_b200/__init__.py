@@ -307,7 +307,8 @@ def dsa_decode_step(groups, k: int, scale: float, ws=None, stream=None, side=Non
     """A micro-batched decode step over IndexShare groups (see include/dsa.h).  `groups` is
     a list of dicts with iq, w, ik, qs (L tensors), kvs (L tensors), idx, outs (L tensors);
     iq and ik are bf16, or uint8 holding E4M3 bytes (the index format is taken from their
-    dtype); `side` a second CUDA stream (created when None)."""
+    dtype); `side` a second CUDA stream (created when None), or `stream` itself to run the
+    whole batch's groups in order on one stream."""
     torch = _torch()
     G = len(groups)
     L = len(groups[0]["qs"])

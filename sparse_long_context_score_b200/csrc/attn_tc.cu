@@ -92,7 +92,7 @@ constexpr int kOffM = kOffL + 64 * 4;            // [64] f32
 constexpr int kOffCoef = kOffM + 64 * 4;         // [64] f32: this split's share of the normaliser
 constexpr int kOffMask = kOffCoef + 64 * 4;      // [kStages] u64: valid rows of the tile in the stage
 constexpr int kOffVote = kOffMask + kStages * 8;  // [2] u32 (tile parity): one byte per softmax warp
-constexpr int kNumBars = 2 * kStages + 11;
+constexpr int kNumBars = 2 * kStages + 12;
 constexpr int kOffBar = kOffVote + 8;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmemA = kOffTmem + 16 + 1024;     // + alignment slack
@@ -104,6 +104,8 @@ constexpr int kTmemS = 256;    // S: 2 buffers x 64 columns, lanes 0..15 of each
 constexpr int kTmemCols = 512;
 
 constexpr int kPartialFloats = 64 * kDv;         // one split's [64][512] partial output
+constexpr int kCsOffset = kPartialFloats + 4 * kMaxSplits;  // floats from the staging buffer to c_s
+static_assert((kCsOffset + kMaxSplits * 64) * 4 <= kStages * kStageBytes, "staged O, received slices and c_s fit");
 
 struct AttnMaps {
   CUtensorMap q[kMaxLayers];
@@ -137,6 +139,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   const uint32_t qfull_bar = bar0 + 8u * (2 * kStages + 8);
   const uint32_t grp_bar = bar0 + 8u * (2 * kStages + 9);
   const uint32_t sdone_bar = bar0 + 8u * (2 * kStages + 10);
+  const uint32_t rbar = bar0 + 8u * (2 * kStages + 11);  // split reduction: the slices landed
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
 
   const int split = blockIdx.x, row = blockIdx.y, layer = blockIdx.z;
@@ -162,6 +165,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     mbar_init(qfull_bar, 1);
     mbar_init(grp_bar, 128);
     mbar_init(sdone_bar, 1);
+    mbar_init(rbar, 1);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -436,26 +440,26 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
 
   // ------------------------------------------------------------------ split reduction
   //   out[h] = sum_s c_s[h] O_s[h],  c_s[h] = 2^(m_s[h] - M[h]) / sum_r 2^(m_r[h] - M[h]) l_r[h],
-  // M[h] = max_r m_r[h].  Each split writes its unnormalised O straight from TMEM to its
-  // partial block (L2-resident) while its (m, l) stay in shared memory; after one cluster
-  // barrier split r reads every split's (m, l) through distributed shared memory, forms the
-  // c_s of all heads, and sums slice r of the [H][512] output over the partials.  A single
-  // split writes O / l directly.  Every thread passes the cluster barriers on every path (a
-  // failed wait above only skips work), so none of them can be left waiting.
+  // M[h] = max_r m_r[h].  Every split stages its O (unnormalised; a single split: O / l) from
+  // TMEM as [H][512] f32 in its consumed stages and writes it with one bulk copy: to its
+  // partial block (L2-resident), or, for a single split, to the output.  After one cluster
+  // barrier split r reads every split's (m, l) through distributed shared memory, bulk-loads
+  // slice r of every split's partial, and writes slice r of the output.  Every thread passes
+  // the cluster barriers on every path (a failed wait above only skips work), so none of
+  // them can be left waiting.
   tc_fence_before();
   __syncthreads();  // (m, l) of this split published; its MMAs have completed
   tc_fence_after();
+  const bool split_mode = nsplit > 1;
   if (threadIdx.x < 64) {
     const int h = threadIdx.x;
-    s_coef[h] = nsplit > 1 ? 1.f : (s_l[h] > 0.f ? 1.f / s_l[h] : 0.f);
+    s_coef[h] = split_mode ? 1.f : (s_l[h] > 0.f ? 1.f / s_l[h] : 0.f);
   }
   __syncthreads();  // s_coef
-  // O^T (TMEM lane = value dim, column = head) goes to global memory: the output itself for
-  // a single split, else this split's partial.  Twelve warps, three per TMEM lane quarter,
-  // take the eight 32-column chunks (value block mb, head half); for each head a warp
-  // writes 32 consecutive value dims (128 bytes).
-  float* dst = nsplit == 1 ? layers.out[layer] + (size_t)row * H * kDv
-                           : partials + (((size_t)layer * gridDim.y + row) * nsplit + split) * kPartialFloats;
+  // Twelve warps, three per TMEM lane quarter, take the eight 32-column chunks of O^T (TMEM
+  // lane = value dim, column = head); for each head a warp stores 32 consecutive value dims
+  // (128 bytes, conflict-free) of the staging buffer.
+  float* obuf = reinterpret_cast<float*>(smem + kOffStage);
   if (warp != kMmaWarp && warp != kPvWarp) {
     const int quarter = warp & 3;
     const int jw = warp < kProducerWarps ? warp >> 2 : 2;
@@ -476,22 +480,44 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
       {
         const int hh = 32 * (c0 & 1), dim = 128 * (c0 >> 1) + 32 * quarter + lane;
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2)
-          if (hh + c2 < H) dst[(size_t)(hh + c2) * kDv + dim] = __uint_as_float(o0[c2]) * s_coef[hh + c2];
+        for (int c2 = 0; c2 < 32; ++c2) obuf[(hh + c2) * kDv + dim] = __uint_as_float(o0[c2]) * s_coef[hh + c2];
       }
       if (two) {
         const int hh = 32 * (c1 & 1), dim = 128 * (c1 >> 1) + 32 * quarter + lane;
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2)
-          if (hh + c2 < H) dst[(size_t)(hh + c2) * kDv + dim] = __uint_as_float(o1[c2]) * s_coef[hh + c2];
+        for (int c2 = 0; c2 < 32; ++c2) obuf[(hh + c2) * kDv + dim] = __uint_as_float(o1[c2]) * s_coef[hh + c2];
       }
     }
+    fence_proxy_async();  // the staged O is visible to the bulk copy (async proxy)
   }
-  if (nsplit > 1) {
+  __syncthreads();
+  float* dst = split_mode ? partials + (((size_t)layer * gridDim.y + row) * nsplit + split) * kPartialFloats
+                          : layers.out[layer] + (size_t)row * H * kDv;
+  if (threadIdx.x == 0) {
+    bulk_store(dst, smem_u32(obuf), (uint32_t)(H * kDv * 4));
+    bulk_commit();
+    bulk_wait_all();  // written (and the staging buffer read)
+    fence_proxy_async_global();
+  }
+  if (split_mode) {
     cluster_sync();  // every split's partial is in global memory and its (m, l) in shared memory
-    // c_s[h] of every split, from the (m, l) of all splits; s_cs[s][h] reuses the first
-    // stage's space (its tiles are consumed)
-    float* s_cs = reinterpret_cast<float*>(smem + kOffStage);
+    // this split's slice of the output: float4 e = h * 128 + d / 4 of the [H][512] block,
+    // a contiguous range of every split's partial, bulk-loaded into the staging buffer
+    const int total = H * (kDv / 4);
+    const int e0 = (int)((long long)split * total / nsplit), e1 = (int)((long long)(split + 1) * total / nsplit);
+    const uint32_t slice_bytes = (uint32_t)(e1 - e0) * 16u;
+    const float* part = partials + ((size_t)layer * gridDim.y + row) * nsplit * kPartialFloats;
+    if (threadIdx.x == 0 && slice_bytes > 0) {
+      fence_proxy_async_global();
+      mbar_arrive_expect_tx(rbar, slice_bytes * (uint32_t)nsplit);
+      for (int sp = 0; sp < nsplit; ++sp)
+        bulk_load(smem_u32(obuf) + (uint32_t)sp * slice_bytes, part + (size_t)sp * kPartialFloats + 4 * (size_t)e0,
+                  slice_bytes, rbar);
+    }
+    // c_s[h] of every split while the slices land; s_cs[s][h] sits past the received
+    // slices (nsplit slices of at most ceil(H * 128 / nsplit) float4: up to kMaxSplits - 1
+    // float4 more than the [H][512] block)
+    float* s_cs = obuf + kCsOffset;
     if (threadIdx.x < 64) {
       const int h = threadIdx.x;
       float mr[kMaxSplits], lr[kMaxSplits];
@@ -512,45 +538,28 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     // this CTA has read the other splits' shared memory: they may exit once all have
     cluster_arrive();
     __syncthreads();  // s_cs
-    // this split's slice of the output: float4 e = h * 128 + d / 4 of the [H][512] block
-    const int total = H * (kDv / 4);
-    const int e0 = (int)((long long)split * total / nsplit), e1 = (int)((long long)(split + 1) * total / nsplit);
-    const float4* part = reinterpret_cast<const float4*>(partials + ((size_t)layer * gridDim.y + row) * nsplit *
-                                                                        kPartialFloats);
-    float4* out4 = reinterpret_cast<float4*>(layers.out[layer] + (size_t)row * H * kDv);
-    // two elements per thread at a time: all their partial loads are in flight together
-    for (int e = e0 + (int)threadIdx.x; e < e1; e += 2 * kThreadsA) {
-      const int e2 = e + kThreadsA;
-      const bool has2 = e2 < e1;
-      const int h = e >> 7, h2 = has2 ? e2 >> 7 : h;
-      float4 v[kMaxSplits], v2[kMaxSplits];
+    bool landed = slice_bytes == 0 || mbar_wait(rbar, 0, err, 31);
+    if (!landed && slice_bytes > 0) landed = mbar_wait_drain(rbar, 0);  // the copies end before the CTA does
+    if (landed) {
+      const float4* recv = reinterpret_cast<const float4*>(obuf);
+      const int n4 = e1 - e0;
+      float4* out4 = reinterpret_cast<float4*>(layers.out[layer] + (size_t)row * H * kDv) + e0;
+      for (int e = (int)threadIdx.x; e < n4; e += kThreadsA) {
+        const int h = (e0 + e) >> 7;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-      for (int sp = 0; sp < kMaxSplits; ++sp) {
-        if (sp < nsplit) {
-          v[sp] = __ldcg(part + (size_t)sp * (kPartialFloats / 4) + e);
-          if (has2) v2[sp] = __ldcg(part + (size_t)sp * (kPartialFloats / 4) + e2);
-        }
-      }
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f), acc2 = acc;
-#pragma unroll
-      for (int sp = 0; sp < kMaxSplits; ++sp) {
-        if (sp < nsplit) {
-          const float c = s_cs[sp * 64 + h];
-          acc.x += c * v[sp].x;
-          acc.y += c * v[sp].y;
-          acc.z += c * v[sp].z;
-          acc.w += c * v[sp].w;
-          if (has2) {
-            const float c2 = s_cs[sp * 64 + h2];
-            acc2.x += c2 * v2[sp].x;
-            acc2.y += c2 * v2[sp].y;
-            acc2.z += c2 * v2[sp].z;
-            acc2.w += c2 * v2[sp].w;
+        for (int sp = 0; sp < kMaxSplits; ++sp) {
+          if (sp < nsplit) {
+            const float c = s_cs[sp * 64 + h];
+            const float4 v = recv[sp * n4 + e];
+            acc.x += c * v.x;
+            acc.y += c * v.y;
+            acc.z += c * v.z;
+            acc.w += c * v.w;
           }
         }
+        out4[e] = acc;
       }
-      out4[e] = acc;
-      if (has2) out4[e2] = acc2;
     }
     cluster_wait();
   }

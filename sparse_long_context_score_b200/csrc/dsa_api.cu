@@ -296,13 +296,15 @@ size_t dsa_decode_workspace_size(int B, int N, int k, int H, int L) {
   const int B0 = (B + 1) / 2, B1 = B - B0;
   size_t n = round256(group_layout(B0, 1, N, k, H, L).total);
   if (B1 > 0) n += group_layout(B1, 1, N, k, H, L).total;
-  return n;
+  const size_t whole = group_layout(B, 1, N, k, H, L).total;  // the in-order step (side == stream)
+  return n > whole ? n : whole;
 }
 
 dsa_status dsa_decode_step(const dsa_group_io* groups, int G, int L, int B, int N, int H, int k, float scale,
                            void* workspace, size_t workspace_bytes, cudaStream_t stream, cudaStream_t side) {
   if (!groups || G <= 0 || !sizes_ok(B, 1, N)) return DSA_ERR_INVALID_ARG;
-  const int B0 = (B + 1) / 2, B1 = B - B0;
+  // side == stream: the whole batch runs its groups in order on `stream`
+  const int B0 = side == stream ? B : (B + 1) / 2, B1 = B - B0;
   const GroupLayout g0 = group_layout(B0, 1, N, k, H, L);
   const GroupLayout g1 = group_layout(B1 > 0 ? B1 : 1, 1, N, k, H, L);
   const size_t off1 = round256(g0.total);
@@ -350,8 +352,9 @@ dsa_status dsa_decode_step(const dsa_group_io* groups, int G, int L, int B, int 
   }
   const int sms = device_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorInvalidDevice);
-  // The indexer saturates HBM with about two thirds of the SMs; the other micro-batch's
-  // top-k and attention run beside it on the rest.
+  // The indexer keeps HBM near its peak on about two thirds of the SMs; the other
+  // micro-batch's top-k and attention run beside it on the rest (measured on B200: a
+  // 7/16 share for them was slower).
   const int tail_sms = sms / 3, idx_sms = sms - tail_sms;
   DecodeEvents* ev = decode_events();
   if (!ev) return cuda_status(cudaErrorInvalidDevice);

@@ -54,14 +54,18 @@ struct TcCfg {
   static constexpr int kN = 32 * QG;                  // MMA N
   static constexpr int kHalves = kF8 ? 1 : 2;         // 128-byte column boxes per 128-wide row
   static constexpr int kStageBytesA = kHalves * kHalfBytesA;
-  static constexpr int kStages = kF8 ? (QG == 1 ? 10 : 8) : (QG == 1 ? 5 : 4);  // same bytes in flight
+  // 160 KB of keys in flight per SM in decode (measured on B200: a deeper ring is no
+  // faster); prefill: a shallower ring beside the larger B
+  static constexpr int kStages = kF8 ? (QG == 1 ? 10 : 8) : (QG == 1 ? 5 : 4);
   static constexpr int kHalfBytesB = kN * 128;
   static constexpr int kBytesB = kHalves * kHalfBytesB;
   static constexpr int kTmemCols = kAccBufs * kN;  // 128 or 512: a power of two >= 32
   static constexpr int kOffA = 0;
   static constexpr int kOffB = kOffA + kStages * kStageBytesA;
-  static constexpr int kOffHist = kOffB + kBytesB;     // two row histograms (a CTA spans <= 2 rows)
-  static constexpr int kOffBar = kOffHist + (kHist ? 2 * kHistBins * 4 : 0);
+  // two row histograms (a CTA spans <= 2 rows) of 16-bit counts, two bins per 32-bit word
+  // (a CTA counts at most its item range: fewer than 2^16 keys at one CTA per SM)
+  static constexpr int kOffHist = kOffB + kBytesB;
+  static constexpr int kOffBar = kOffHist + (kHist ? 2 * kHistBins * 2 : 0);
   static constexpr int kNumBars = 2 * kStages + 2 * kAccBufs + 3;
   static constexpr int kOffTmem = kOffBar + kNumBars * 8;
   static constexpr int kSmem = kOffTmem + 16 + 1024;  // + alignment slack
@@ -164,7 +168,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     tmem_relinquish();
   }
   if (kHist)
-    for (int i = threadIdx.x; i < 2 * kHistBins; i += C::kThreads) s_hist[i] = 0;
+    for (int i = threadIdx.x; i < kHistBins; i += C::kThreads) s_hist[i] = 0;
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -316,7 +320,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         atomicCAS(err, 0, 9);
         slot = 1;
       }
-      uint32_t* hslot = s_hist + slot * kHistBins;
+      uint32_t* hslot = s_hist + slot * (kHistBins / 2);
       (void)hslot;
       if (QG == 1) {
         uint32_t r[32];
@@ -327,7 +331,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         for (int h = 0; h < 32; ++h) sc = fmaf(wr[h], fmaxf(__uint_as_float(r[h]), 0.f), sc);
         if (t0 < T && key < visible_count(N, q_pos0, t0)) {
           scores[((size_t)b * T + t0) * N + key] = sc;
-          if (kHist) atomicAdd(&hslot[order_key(sc) >> kHistShift], 1u);
+          if (kHist) {
+            const uint32_t bin = order_key(sc) >> kHistShift;
+            atomicAdd(&hslot[bin >> 1], 1u << (16 * (bin & 1)));
+          }
         }
       } else {
         // two queries (64 columns) per TMEM round trip; head weights as 16-byte loads
@@ -373,10 +380,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     Cursor cur;
     cur.start(it, begin, end);
     const int b_first = cur.qg / it.G;
-    for (int i = threadIdx.x; i < 2 * kHistBins; i += C::kThreads) {
+    for (int i = threadIdx.x; i < kHistBins; i += C::kThreads) {  // word i: bins 2i, 2i + 1 of a slot
       const uint32_t c = s_hist[i];
-      const int row = b_first + i / kHistBins;
-      if (c && row < B) atomicAdd(&hist[(size_t)row * kHistBins + (i % kHistBins)], c);
+      const int row = b_first + i / (kHistBins / 2);
+      const int bin = 2 * (i % (kHistBins / 2));
+      if (c && row < B) {
+        if (c & 0xFFFFu) atomicAdd(&hist[(size_t)row * kHistBins + bin], c & 0xFFFFu);
+        if (c >> 16) atomicAdd(&hist[(size_t)row * kHistBins + bin + 1], c >> 16);
+      }
     }
   }
 }

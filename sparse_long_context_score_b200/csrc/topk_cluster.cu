@@ -309,13 +309,25 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
       sm.q_ge[threadIdx.x] = 0u;
     }
     __syncthreads();
-    // every CTA's list, in rank order
-    uint32_t M = 0;
-    for (int q = 0; q < C; ++q) {
-      const uint32_t n = min(sm.q_cnt[q], (uint32_t)kMergeCap - M);
-      for (uint32_t i = threadIdx.x; i < n; i += kCT)
-        sm.m.mrg[M + i] = ld_cluster_u64(cluster_map(smem_u32(&sm.m.loc[i]), q));
-      M += n;
+    // every CTA's list, in rank order: per round, each thread's element of every list is
+    // loaded first (up to kMaxC remote loads in flight), then stored
+    uint32_t off[kMaxC], cnt[kMaxC];
+    uint32_t M = 0, nmax = 0;
+#pragma unroll
+    for (int q = 0; q < kMaxC; ++q) {
+      cnt[q] = q < C ? min(sm.q_cnt[q], (uint32_t)kMergeCap - M) : 0u;
+      off[q] = M;
+      M += cnt[q];
+      nmax = max(nmax, cnt[q]);
+    }
+    for (uint32_t i = threadIdx.x; i < nmax; i += kCT) {
+      unsigned long long vq[kMaxC];
+#pragma unroll
+      for (int q = 0; q < kMaxC; ++q)
+        if (i < cnt[q]) vq[q] = ld_cluster_u64(cluster_map(smem_u32(&sm.m.loc[i]), q));
+#pragma unroll
+      for (int q = 0; q < kMaxC; ++q)
+        if (i < cnt[q]) sm.m.mrg[off[q] + i] = vq[q];
     }
     cluster_arrive();  // done with the peers' memory (#B; its wait is at the very end)
     __syncthreads();

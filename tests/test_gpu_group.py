@@ -89,8 +89,9 @@ def test_mtp_draft_steps_reuse_step1_indices(dsa, orc):
         assert_close(host(outs[0]), routs[0], f"mtp step {step + 1}")
 
 
-@pytest.mark.parametrize("B,G", [(3, 2), (2, 3), (1, 2), (8, 1)])
-def test_decode_step_matches_oracle(dsa, orc, B, G):
+@pytest.mark.parametrize("B,G,in_order", [(3, 2, False), (2, 3, False), (1, 2, False), (8, 1, False),
+                                          (3, 2, True)])
+def test_decode_step_matches_oracle(dsa, orc, B, G, in_order):
     """dsa_decode_step (two micro-batches on two streams, indexers taking turns) gives every
     group the oracle's index list bit for bit and its attention within the tolerance."""
     import torch
@@ -103,7 +104,9 @@ def test_decode_step_matches_oracle(dsa, orc, B, G):
                            kvs=[dev_bf16(x) for x in kvs],
                            idx=torch.empty(B, 1, w.k, dtype=torch.int32, device="cuda"),
                            outs=[torch.empty(B, 1, w.H, 512, dtype=torch.float32, device="cuda") for _ in range(w.L)]))
-    dsa.dsa_decode_step(groups, w.k, C.SCALE)
+    stream = torch.cuda.current_stream()
+    # in order: side == stream runs the whole batch's groups on one stream
+    dsa.dsa_decode_step(groups, w.k, C.SCALE, stream=stream, side=stream if in_order else None)
     torch.cuda.synchronize()
     assert dsa.dsa_check_device_status() == 0
     for g in range(G):

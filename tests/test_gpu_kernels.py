@@ -122,6 +122,18 @@ def test_sparse_attn(dsa, orc, B, T, N, H, k, inv):
     assert_close(got, ref, "sparse attention")
 
 
+@pytest.mark.parametrize("rows", [21, 24, 29, 37])
+def test_sparse_attn_uneven_splits(dsa, orc, rows):
+    """Row counts whose key splits (148 SMs: 7, 6, 5 or 4 CTAs per row) cut the [H][512]
+    output into slices of unequal length, so the split reduction's received slices do not
+    tile the block exactly."""
+    N, H, k = 3000, 64, 2048
+    q, kv, idx = _attn_case(9000 + rows, rows, 1, N, H, k, 0.01)
+    got = host(dsa.dsa_sparse_attn(dev_bf16(q), dev_bf16(kv), dev(idx), C.SCALE))
+    ref = orc.sparse_attn(q, kv, idx, C.SCALE)
+    assert_close(got, ref, f"sparse attention, {rows} rows")
+
+
 def test_sparse_attn_empty_rows_are_zero(dsa):
     q, kv, idx = _attn_case(3, 1, 2, 100, 16, 40)
     idx[0, 1, :] = -1
