@@ -18,7 +18,7 @@ import numpy as np
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRCS = [os.path.join(_HERE, "dsa_oracle.c"), os.path.join(_HERE, "verify_oracle.c"),
-         os.path.join(_HERE, "fp8_oracle.c")]
+         os.path.join(_HERE, "fp8_oracle.c"), os.path.join(_HERE, "shard_oracle.c")]
 _LIB = os.path.join(_HERE, "liboracle.so")
 
 OR_OK = 0
@@ -62,8 +62,12 @@ class Oracle:
         L.oracle_index_score_e4m3.argtypes = [P, P, P, I, I, I, I, I, Lg, P]
         L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_to_double.restype = D
+        L.oracle_sparse_attn_partial.argtypes = [P, P, P, I, I, I, Lg, I, I, I, I, D, P, P]
+        L.oracle_merge_partials.argtypes = [P, P, I, Lg, I, P]
+        L.oracle_merge_candidates.argtypes = [P, P, Lg, I, I, P]
         for f in ("oracle_index_score", "oracle_topk", "oracle_sparse_attn",
-                  "oracle_dense_masked_attn", "oracle_group_forward", "oracle_verify", "oracle_index_score_e4m3"):
+                  "oracle_dense_masked_attn", "oracle_group_forward", "oracle_verify", "oracle_index_score_e4m3",
+                  "oracle_sparse_attn_partial", "oracle_merge_partials", "oracle_merge_candidates"):
             getattr(L, f).restype = I
         self.L = L
 
@@ -151,6 +155,42 @@ class Oracle:
                "oracle_index_score_e4m3")
         return out
 
+    def sparse_attn_partial(self, q, kv, idx, offset: int, scale: float, dv: int = 512):
+        """Attention over the selected rows of one context shard (shard_oracle.c): kv holds
+        global positions [offset, offset + Ns).  Returns (out [B,T,H,dv] f64, lse [B,T,H] f64)."""
+        q = _bf16(q)
+        kv = _bf16(kv)
+        idx = np.ascontiguousarray(idx, dtype=np.int32)
+        B, T, H, dqk = q.shape
+        Ns = kv.shape[1]
+        k = idx.shape[2]
+        out = np.empty((B, T, H, dv), np.float64)
+        lse = np.empty((B, T, H), np.float64)
+        _check(self.L.oracle_sparse_attn_partial(_ptr(q), _ptr(kv), _ptr(idx), B, T, Ns, int(offset), H, k, dqk, dv,
+                                                 float(scale), _ptr(out), _ptr(lse)), "oracle_sparse_attn_partial")
+        return out, lse
+
+    def merge_partials(self, outs, lses):
+        """outs [W, ..., dv], lses [W, ...] -> out [..., dv] (shard_oracle.c)."""
+        outs = np.ascontiguousarray(outs, dtype=np.float64)
+        lses = np.ascontiguousarray(lses, dtype=np.float64)
+        W, dv = outs.shape[0], outs.shape[-1]
+        R = lses[0].size
+        out = np.empty(outs.shape[1:], np.float64)
+        _check(self.L.oracle_merge_partials(_ptr(outs), _ptr(lses), W, R, dv, _ptr(out)), "oracle_merge_partials")
+        return out
+
+    def merge_candidates(self, score, pos, k: int):
+        """score [..., M] f32, pos [..., M] i32 (< 0: none) -> idx [..., k] (shard_oracle.c)."""
+        score = np.ascontiguousarray(score, dtype=np.float32)
+        pos = np.ascontiguousarray(pos, dtype=np.int32)
+        M = score.shape[-1]
+        R = score.size // M if M else 0
+        idx = np.empty(score.shape[:-1] + (k,), np.int32)
+        _check(self.L.oracle_merge_candidates(_ptr(score), _ptr(pos), R, M, int(k), _ptr(idx)),
+               "oracle_merge_candidates")
+        return idx
+
     def verify(self, p: np.ndarray, q: np.ndarray, draft: np.ndarray, u: np.ndarray, u2: np.ndarray):
         """MTP verify step (rejection sampling), verify_oracle.c.  p, q [B, S, V] float32
         target / draft probabilities; draft, u, u2 [B, S].  Returns (alpha [B,S] f64,
@@ -215,3 +255,15 @@ def group_forward(*a, **kw):
 
 def verify(*a, **kw):
     return default().verify(*a, **kw)
+
+
+def sparse_attn_partial(*a, **kw):
+    return default().sparse_attn_partial(*a, **kw)
+
+
+def merge_partials(*a, **kw):
+    return default().merge_partials(*a, **kw)
+
+
+def merge_candidates(*a, **kw):
+    return default().merge_candidates(*a, **kw)

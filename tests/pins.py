@@ -506,4 +506,111 @@ def pin_index_score_e4m3_one_hot(o):
     assert s[0, 0, 0] == 0.9375 and s[0, 0, 1] == 0.0
 
 
+# ---------------------------------------------------------------- context-sharded decode
+
+def pin_partial_single_row_lse_is_logit(o):
+    """One selected row in the shard: its value part is the output and the log-sum-exp is
+    its logit scale * q . kv (computed here with numpy, in float64)."""
+    q, kv, _ = _attn_inputs(30, N=60)
+    offset = 1000                      # the shard holds global positions 1000..1059
+    idx = np.full((1, 2, 4), -1, np.int32)
+    idx[0, 0, 1] = offset + 17
+    idx[0, 1, 3] = offset + 59
+    idx[0, 1, 0] = 5                   # outside the shard: skipped
+    out, lse = o.sparse_attn_partial(q, kv, idx, offset, C.SCALE)
+    for t, row in ((0, 17), (1, 59)):
+        for h in range(3):
+            assert np.array_equal(out[0, t, h], f(kv[0, row, :512]))
+            want = C.SCALE * float(np.dot(f(q[0, t, h]), f(kv[0, row])))
+            assert abs(lse[0, t, h] - want) <= 1e-12 * max(1.0, abs(want))
+
+
+def pin_partial_uniform_logits_lse_is_log_count(o):
+    """q = 0: every logit is 0, so the log-sum-exp is ln(number of rows in the shard)."""
+    q, kv, idx = _attn_inputs(31, N=60, k=20)
+    q[:] = 0
+    offset = 300
+    gidx = idx + offset
+    gidx[0, 1, :7] = -1                # 13 rows left in query 1
+    _, lse = o.sparse_attn_partial(q, kv, gidx, offset, C.SCALE)
+    assert np.allclose(lse[0, 0], math.log(20), rtol=0, atol=1e-13)
+    assert np.allclose(lse[0, 1], math.log(13), rtol=0, atol=1e-13)
+
+
+def pin_partial_whole_cache_equals_sparse_attn(o):
+    """A shard holding the whole cache (offset 0) is the unsharded attention."""
+    q, kv, idx = _attn_inputs(32, B=2, T=2, H=2, N=50, k=12)
+    out, _ = o.sparse_attn_partial(q, kv, idx, 0, C.SCALE)
+    assert np.array_equal(out, o.sparse_attn(q, kv, idx, C.SCALE))
+
+
+def pin_merged_partials_equal_unsharded_attention(o):
+    """Three contiguous shards of the cache: their partials combined by log-sum-exp equal
+    the attention over the whole selection (float64, to rounding)."""
+    q, kv, idx = _attn_inputs(33, B=2, T=2, H=3, N=90, k=30)
+    full = o.sparse_attn(q, kv, idx, C.SCALE)
+    outs, lses = [], []
+    for lo, hi in ((0, 25), (25, 61), (61, 90)):
+        out, lse = o.sparse_attn_partial(q, kv[:, lo:hi].copy(), idx, lo, C.SCALE)
+        outs.append(out)
+        lses.append(lse)
+    merged = o.merge_partials(np.stack(outs), np.stack(lses))
+    assert np.allclose(merged, full, rtol=0, atol=1e-12)
+
+
+def pin_merge_partials_one_shard_empty(o):
+    """A shard without selected rows (lse = -inf) contributes nothing; all empty gives 0."""
+    outs = np.zeros((2, 1, 4), np.float64)
+    outs[0, 0] = [1.0, -2.0, 3.0, 0.5]
+    lses = np.array([[0.7], [-np.inf]])
+    assert np.array_equal(o.merge_partials(outs, lses)[0], outs[0, 0])
+    assert np.array_equal(o.merge_partials(outs, np.full((2, 1), -np.inf))[0], np.zeros(4))
+
+
+def pin_merge_partials_weights(o):
+    """Two shards with log-sum-exps ln 1 and ln 3: weights 1/4 and 3/4 (closed form)."""
+    outs = np.zeros((2, 1, 2), np.float64)
+    outs[0, 0] = [4.0, 0.0]
+    outs[1, 0] = [0.0, 8.0]
+    got = o.merge_partials(outs, np.array([[0.0], [math.log(3.0)]]))[0]
+    assert np.allclose(got, [1.0, 6.0], rtol=0, atol=1e-14)
+
+
+def _shard_candidates(o, row_scores, bounds, k):
+    """Per shard: the oracle's top-k of the shard's scores (positions local), mapped to
+    global positions, with their scores; -1 / -inf padding."""
+    T = row_scores.shape[0]
+    score, pos = [], []
+    for lo, hi in bounds:
+        loc = o.topk(row_scores[None, :, lo:hi].copy(), hi - lo - 1, k)[0]
+        g = np.where(loc >= 0, loc + lo, -1).astype(np.int32)
+        sc = np.where(loc >= 0, np.take_along_axis(row_scores[:, lo:hi], np.maximum(loc, 0), axis=1),
+                      -np.inf).astype(np.float32)
+        score.append(sc)
+        pos.append(g)
+    return np.concatenate(score, axis=1), np.concatenate(pos, axis=1)
+
+
+def pin_sharded_topk_equals_full_topk(o):
+    """Top-k per contiguous shard, then the k best candidates, equals the top-k of the
+    whole row (numpy lexsort of the full row) -- with many ties across shard borders."""
+    r = _rng(34)
+    T, N, k = 3, 997, 40
+    scores = r.integers(-20, 21, size=(T, N)).astype(np.float32) / 4   # heavy ties
+    bounds = ((0, 250), (250, 251), (251, 700), (700, N))
+    cs, cp = _shard_candidates(o, scores, bounds, k)
+    got = o.merge_candidates(cs, cp, k)
+    for t in range(T):
+        assert got[t].tolist() == _lexsort_topk(scores[t], N, k)
+
+
+def pin_merge_candidates_ties_and_padding(o):
+    """Equal scores go to the lower position whatever the candidate order; fewer than k
+    candidates are all kept, ascending, then -1."""
+    score = np.array([[5.0, 7.0, 5.0, 5.0, 1.0, 0.0]], np.float32)
+    pos = np.array([[90, 40, 10, 60, -1, 3]], np.int32)
+    assert o.merge_candidates(score, pos, 3)[0].tolist() == [10, 40, 60]
+    assert o.merge_candidates(score, pos, 8)[0].tolist() == [3, 10, 40, 60, 90, -1, -1, -1]
+
+
 ALL_PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -13,7 +13,8 @@ HERE = os.path.dirname(oracle.__file__)
 SRC = os.path.join(HERE, "dsa_oracle.c")
 VERIFY_SRC = os.path.join(HERE, "verify_oracle.c")
 FP8_SRC = os.path.join(HERE, "fp8_oracle.c")
-SOURCES = [SRC, VERIFY_SRC, FP8_SRC]
+SHARD_SRC = os.path.join(HERE, "shard_oracle.c")
+SOURCES = [SRC, VERIFY_SRC, FP8_SRC, SHARD_SRC]
 
 MUTANTS = {
     "relu_dropped": ("double relu = dot > 0.0 ? dot : 0.0;", "double relu = dot;"),
@@ -48,6 +49,20 @@ MUTANTS = {
     "e4m3_subnormal_scale": ("ldexp((double)m / 8.0, -6)", "ldexp((double)m / 8.0, -7)", FP8_SRC),
     "e4m3_relu_dropped": ("total += (double)wt[h] * (dot > 0.0 ? dot : 0.0);", "total += (double)wt[h] * dot;", FP8_SRC),
     "e4m3_key_index": ("oracle_e4m3_to_double(ks[d])", "oracle_e4m3_to_double(ks[0])", FP8_SRC),
+    # context-sharded decode (shard_oracle.c)
+    "shard_lse_base2": ("lse[(b * T + t) * (long)H + h] = zmax + log(denom);",
+                        "lse[(b * T + t) * (long)H + h] = zmax + log2(denom);", SHARD_SRC),
+    "shard_lse_drops_max": ("lse[(b * T + t) * (long)H + h] = zmax + log(denom);",
+                            "lse[(b * T + t) * (long)H + h] = log(denom);", SHARD_SRC),
+    "shard_range_exclusive_low": ("if (g < offset || g >= offset + Ns) continue;\n                    const uint16_t *c",
+                                  "if (g <= offset || g >= offset + Ns) continue;\n                    const uint16_t *c",
+                                  SHARD_SRC),
+    "merge_weight_sign": ("const double c = exp(lses[(long)w * R + r] - m) / s;",
+                          "const double c = exp(m - lses[(long)w * R + r]) / s;", SHARD_SRC),
+    "merge_unnormalised": ("const double c = exp(lses[(long)w * R + r] - m) / s;",
+                           "const double c = exp(lses[(long)w * R + r] - m);", SHARD_SRC),
+    "cand_tie_to_higher": ("return a->pos < b->pos;", "return a->pos > b->pos;", SHARD_SRC),
+    "cand_not_sorted": ("qsort(o, (size_t)take, sizeof(int32_t), sh_cmp_i32);", "", SHARD_SRC),
 }
 
 
