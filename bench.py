@@ -42,6 +42,9 @@ def parse():
     p.add_argument("--cpu-sample", type=int, default=2, help="sequences in the CPU-oracle sample")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-extra", action="store_true", help="skip the 1M / MTP / prefill workloads")
+    p.add_argument("--shard", default="batch", choices=["batch", "context"],
+                   help="multi-GPU: each rank its own batch (weak scaling), or every sequence's context "
+                        "spread over the ranks (strong scaling; sparse_long_context_score_b200.sharded)")
     p.add_argument("--schedule", default="sequential", choices=["micro", "sequential"],
                    help="decode workloads: one dsa_group_forward per group in order on one stream (the "
                         "faster on B200), or dsa_decode_step (two micro-batches on two streams)")
@@ -623,6 +626,72 @@ def ncu_case(kind: str) -> None:
         sys.exit(1)
 
 
+def run_context_sharded(args, rank, world, device, w):
+    """The decode step of `w` with every sequence's cached tokens spread over the ranks
+    (contiguous shards): per group, the sharded group of sparse_long_context_score_b200.sharded
+    (local indexer and top-k, candidate all-gather and merge, local attention, partial
+    all-gather and merge).  Eager calls (NCCL collectives between the kernels), L2 flushed
+    before every step, CUDA events on the stream, the max over ranks.  Returns (ms per
+    step, clock record)."""
+    import torch
+    import synth
+    import synth.device as sd
+    from sparse_long_context_score_b200 import sharded
+    from synth import configs as C
+    torch.cuda.set_device(device)
+    offset, n = sharded.shard_bounds(w.N, world)[rank]
+    bf = torch.bfloat16
+    groups = []
+    for g in range(w.groups):
+        # the shard of each cache: positions [offset, offset + n) of the same seeded tensors
+        ik = torch.empty(w.B, n, 128, dtype=bf, device=device)
+        kvs = [torch.empty(w.B, n, 576, dtype=bf, device=device) for _ in range(w.L)]
+        for b in range(w.B):
+            sd.int17_bf16(ik[b], w.key(synth.KIND_IK, g), offset=(b * w.N + offset) * 128)
+            for l in range(w.L):
+                sd.normal_bf16(kvs[l][b], w.key(synth.KIND_KV, g, l), offset=(b * w.N + offset) * 576)
+        iq = sd.int17_bf16(torch.empty(w.B, 1, 32, 128, dtype=bf, device=device), w.key(synth.KIND_IQ, g))
+        wt = sd.pow2_f32(torch.empty(w.B, 1, 32, dtype=torch.float32, device=device), w.key(synth.KIND_W, g))
+        qs = [sd.normal_bf16(torch.empty(w.B, 1, w.H, 576, dtype=bf, device=device), w.key(synth.KIND_Q, g, l))
+              for l in range(w.L)]
+        groups.append((iq, wt, ik, qs, kvs))
+    comm = sharded.TorchComm() if world > 1 else None
+    ops = sharded.cuda_ops()
+
+    class _Self:  # one rank: the all-gather of a tensor is that tensor with a leading axis
+        @staticmethod
+        def all_gather(t):
+            return t.unsqueeze(0)
+    comm = comm or _Self()
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    flush_rd = torch.zeros(512 << 20, dtype=torch.uint8, device=device)
+
+    def step():
+        for iq, wt, ik, qs, kvs in groups:
+            sharded.sharded_group_forward(comm, ops, iq, wt, ik, qs, kvs, w.q_pos0, offset, w.k, C.SCALE)
+
+    times = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for i in range(args.warmup + args.steps):
+            flush.zero_()
+            flush_rd.view(torch.int64).sum()
+            if world > 1:
+                torch.distributed.barrier()
+            torch.cuda.synchronize()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            step()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= args.warmup:
+                times.append(a.elapsed_time(b))
+    import sparse_long_context_score_b200 as dsa
+    if dsa.dsa_check_device_status() != 0:
+        raise RuntimeError("device status after the context-sharded steps")
+    ms = max_over_ranks([sum(times) / len(times)], world, device)[0]
+    return ms, clk.summary()
+
+
 def main():
     args = parse()
     if args.ncu_case:
@@ -666,6 +735,22 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
     device = torch.device("cuda", local)
+    if args.shard == "context":
+        wc = C.WORKLOADS[args.workload if args.workload != "decode128k" else "decode1m"]
+        ms, clocks = run_context_sharded(args, rank, world, device, wc)
+        if rank == 0:
+            tokens = wc.B * wc.T
+            cfg = workload_config(wc, world)
+            cfg["parallelism"] = f"context shards x{world}" if world > 1 else "single GPU (one context shard)"
+            print(json.dumps({"metric": metric, "value": tokens / (ms * 1e-3), "unit": "tokens/s", "n_gpus": world,
+                              "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+                              "higher_is_better": True, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                              "data": "synthetic", "config": cfg, "clocks": clocks,
+                              "mode": "context-sharded decode (eager calls, NCCL all-gathers between kernels)"}))
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return
     w, r = run_ours(args, rank, world, device)
     step_bytes, idx_bytes, score_bytes = algorithmic(w)
     tokens = w.B * w.T * w.steps * world

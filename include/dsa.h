@@ -244,6 +244,66 @@ dsa_status dsa_decode_step(const dsa_group_io *groups, int G, int L, int B, int 
                            void *workspace, size_t workspace_bytes, cudaStream_t stream, cudaStream_t side);
 
 /*
+ * Context-sharded decode ("Le contexte d'un million de tokens", Service efficace pour un
+ * million de contextes: a long context is spread over several GPUs; the pages give no
+ * algorithm).  Every GPU holds a contiguous range [offset, offset + N) of the cached tokens
+ * of every sequence (index keys and compressed rows).  One step, with the exchanges done
+ * by the caller (e.g. torch.distributed all-gathers over NCCL):
+ *   1. dsa_index_score and dsa_topk on the shard (q_pos0 = the query's global position
+ *      minus offset) give the shard's own top-k;
+ *   2. dsa_shard_candidates turns it into (score, global position) candidates;
+ *   3. the candidates of all shards are gathered, shard by shard in position order, and
+ *      dsa_merge_candidates keeps the k best: the row's index list, identical to the
+ *      unsharded top-k (a token in the row's top-k is in its shard's top-k);
+ *   4. per layer, dsa_sparse_attn_shard attends over the selected rows the shard holds and
+ *      returns the log-sum-exp of their logits beside the partial output;
+ *   5. the partials of all shards are gathered and dsa_merge_partials combines them:
+ *      out = sum_w exp(lse_w - LSE) out_w, LSE = ln sum_w exp(lse_w).
+ */
+
+/*
+ * Step 3 on one shard.
+ *   kv   [B, N, 576] bf16  the shard's compressed rows: global positions [offset, offset + N)
+ *   idx  [B, T, k]   i32   global positions (entries < 0 or outside the shard are skipped)
+ *   out  [B, T, H, 512] f32 out: softmax over the shard's selected rows only (0 if none)
+ *   lse  [B, T, H]   f32   out: ln sum_j exp(scale * q . kv[j]) over them (-inf if none)
+ * Otherwise as dsa_sparse_attn (workspace included).
+ */
+dsa_status dsa_sparse_attn_shard(const uint16_t *q, const uint16_t *kv, const int32_t *idx,
+                                 int B, int T, int N, long long offset, int H, int k, float scale,
+                                 float *out, float *lse, void *workspace, size_t workspace_bytes,
+                                 cudaStream_t stream);
+
+/*
+ *   scores     [B, T, N] f32   the shard's indexer scores (as dsa_index_score wrote them)
+ *   idx        [B, T, k] i32   the shard's top-k list (dsa_topk: shard-local positions)
+ *   cand_score [B, T, k] f32   out: score of each entry (-inf for padding)
+ *   cand_pos   [B, T, k] i32   out: its global position offset + idx (-1 for padding)
+ */
+dsa_status dsa_shard_candidates(const float *scores, const int32_t *idx, int B, int T, int N, int k,
+                                long long offset, float *cand_score, int32_t *cand_pos,
+                                cudaStream_t stream);
+
+/*
+ *   cand_score, cand_pos [W, B, T, kc]  the candidates of W shards, gathered shard-major
+ *                          (as an all-gather leaves them), shards in position order, so
+ *                          that the valid positions (>= 0) of a row increase from shard 0's
+ *                          list to shard W-1's; W * kc <= 8 * 2048
+ *   idx [B, T, k] i32 out: the k best by (score descending, position ascending; a NaN
+ *                          ranks below every number), ascending, -1 padding when fewer
+ *                          than k candidates are valid
+ */
+dsa_status dsa_merge_candidates(const float *cand_score, const int32_t *cand_pos, int W, int B,
+                                int T, int kc, int k, int32_t *idx, cudaStream_t stream);
+
+/*
+ *   outs [W, B, T, H, 512] f32, lses [W, B, T, H] f32  the shards' partials
+ *   out  [B, T, H, 512] f32 out: their log-sum-exp combination (0 where every lse is -inf)
+ */
+dsa_status dsa_merge_partials(const float *outs, const float *lses, int W, int B, int T, int H,
+                              float *out, cudaStream_t stream);
+
+/*
  * MTP verify step -- rejection sampling of the draft tokens ("GLM-5.2 MTP IndexShare
  * inference", Rejection Sampling: the acceptance rate is sum_v min(p_v, q_v); the MTP
  * pages verify the draft tokens in order and cut the sequence at the first rejection).

@@ -29,6 +29,7 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
 
 # every symbol include/dsa.h declares
 EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_index_score_e4m3",
+           "dsa_sparse_attn_shard", "dsa_shard_candidates", "dsa_merge_candidates", "dsa_merge_partials",
            "dsa_topk",
            "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error",
            "dsa_check_device_status", "dsa_last_cuda_error", "dsa_cuda_error_string", "dsa_verify",
@@ -67,6 +68,10 @@ def lib() -> ctypes.CDLL:
         L.dsa_workspace_size.restype = S
         L.dsa_index_score.argtypes = [P, P, P, I, I, I, LL, P, P]
         L.dsa_index_score_e4m3.argtypes = [P, P, P, I, I, I, LL, P, P]
+        L.dsa_sparse_attn_shard.argtypes = [P, P, P, I, I, I, LL, I, I, F, P, P, P, S, P]
+        L.dsa_shard_candidates.argtypes = [P, P, I, I, I, I, LL, P, P, P]
+        L.dsa_merge_candidates.argtypes = [P, P, I, I, I, I, I, P, P]
+        L.dsa_merge_partials.argtypes = [P, P, I, I, I, I, P, P]
         L.dsa_topk.argtypes = [P, I, I, I, LL, I, P, P, S, P]
         L.dsa_sparse_attn.argtypes = [P, P, P, I, I, I, I, I, F, P, P, S, P]
         L.dsa_group_forward.argtypes = [P, P, P, P, P, I, I, I, I, LL, I, I, F, I, P, P, P, S, P]
@@ -84,7 +89,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_decode_workspace_size.restype = S
         L.dsa_decode_step.argtypes = [P, I, I, I, I, I, I, F, P, S, P, P]
         L.dsa_decode_step.restype = I
-        for f in ("dsa_index_score", "dsa_index_score_e4m3", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc",
+        for f in ("dsa_index_score", "dsa_index_score_e4m3", "dsa_sparse_attn_shard", "dsa_shard_candidates",
+                  "dsa_merge_candidates", "dsa_merge_partials", "dsa_topk", "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc",
                   "dsa_verify"):
             getattr(L, f).restype = I
         _lib = L
@@ -223,6 +229,75 @@ def dsa_sparse_attn(q, kv, idx, scale: float, out=None, ws=None, stream=None):
                                _ptr(out, (torch.float32,), "out", (B, T, H, DV)),
                                _ptr(ws, (torch.uint8,), "workspace"), ws.numel(), _stream(stream))
     _check(rc, "dsa_sparse_attn")
+    return out
+
+
+def dsa_sparse_attn_shard(q, kv, idx, offset: int, scale: float, out=None, lse=None, ws=None, stream=None):
+    """Attention over the selected rows one context shard holds (kv: global positions
+    [offset, offset + N)): q [B,T,H,576] bf16, kv [B,N,576] bf16, idx [B,T,k] int32 global
+    positions -> (out [B,T,H,512] f32, lse [B,T,H] f32)."""
+    torch = _torch()
+    B, T, H, _ = q.shape
+    N = kv.shape[1]
+    k = idx.shape[2]
+    if out is None:
+        out = torch.empty((B, T, H, DV), dtype=torch.float32, device=q.device)
+    if lse is None:
+        lse = torch.empty((B, T, H), dtype=torch.float32, device=q.device)
+    if ws is None:
+        ws = workspace(B, T, N, k, H, 1, q.device)
+    rc = lib().dsa_sparse_attn_shard(_ptr(q, _bf16_types(), "q", (B, T, H, DQK)),
+                                     _ptr(kv, _bf16_types(), "kv", (B, N, DQK)),
+                                     _ptr(idx, (torch.int32,), "idx", (B, T, k)), B, T, N, int(offset), H, k,
+                                     float(scale), _ptr(out, (torch.float32,), "out", (B, T, H, DV)),
+                                     _ptr(lse, (torch.float32,), "lse", (B, T, H)),
+                                     _ptr(ws, (torch.uint8,), "workspace"), ws.numel(), _stream(stream))
+    _check(rc, "dsa_sparse_attn_shard")
+    return out, lse
+
+
+def dsa_shard_candidates(scores, idx, offset: int, cand_score=None, cand_pos=None, stream=None):
+    """scores [B,T,N] f32 and the shard's top-k idx [B,T,k] int32 -> (cand_score [B,T,k] f32,
+    cand_pos [B,T,k] int32 global positions)."""
+    torch = _torch()
+    B, T, N = scores.shape
+    k = idx.shape[2]
+    if cand_score is None:
+        cand_score = torch.empty((B, T, k), dtype=torch.float32, device=scores.device)
+    if cand_pos is None:
+        cand_pos = torch.empty((B, T, k), dtype=torch.int32, device=scores.device)
+    rc = lib().dsa_shard_candidates(_ptr(scores, (torch.float32,), "scores", (B, T, N)),
+                                    _ptr(idx, (torch.int32,), "idx", (B, T, k)), B, T, N, k, int(offset),
+                                    _ptr(cand_score, (torch.float32,), "cand_score", (B, T, k)),
+                                    _ptr(cand_pos, (torch.int32,), "cand_pos", (B, T, k)), _stream(stream))
+    _check(rc, "dsa_shard_candidates")
+    return cand_score, cand_pos
+
+
+def dsa_merge_candidates(cand_score, cand_pos, k: int, idx=None, stream=None):
+    """cand_score [W,B,T,kc] f32, cand_pos [W,B,T,kc] int32 (shard-major, shards in position
+    order) -> idx [B,T,k] int32: the k best, ascending, -1 padding."""
+    torch = _torch()
+    W, B, T, kc = cand_score.shape
+    if idx is None:
+        idx = torch.empty((B, T, k), dtype=torch.int32, device=cand_score.device)
+    rc = lib().dsa_merge_candidates(_ptr(cand_score, (torch.float32,), "cand_score", (W, B, T, kc)),
+                                    _ptr(cand_pos, (torch.int32,), "cand_pos", (W, B, T, kc)), W, B, T, kc, int(k),
+                                    _ptr(idx, (torch.int32,), "idx", (B, T, k)), _stream(stream))
+    _check(rc, "dsa_merge_candidates")
+    return idx
+
+
+def dsa_merge_partials(outs, lses, out=None, stream=None):
+    """outs [W,B,T,H,512] f32, lses [W,B,T,H] f32 -> out [B,T,H,512] f32."""
+    torch = _torch()
+    W, B, T, H, _ = outs.shape
+    if out is None:
+        out = torch.empty((B, T, H, DV), dtype=torch.float32, device=outs.device)
+    rc = lib().dsa_merge_partials(_ptr(outs, (torch.float32,), "outs", (W, B, T, H, DV)),
+                                  _ptr(lses, (torch.float32,), "lses", (W, B, T, H)), W, B, T, H,
+                                  _ptr(out, (torch.float32,), "out", (B, T, H, DV)), _stream(stream))
+    _check(rc, "dsa_merge_partials")
     return out
 
 

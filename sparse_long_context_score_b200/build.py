@@ -15,7 +15,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libdsa.so")
 BUILD_DIR = os.path.join(PKG, "_build")
-SOURCES = ["dsa_api.cu", "indexer_tc.cu", "topk.cu", "topk_cluster.cu", "attn_tc.cu", "dsa_noalloc.cu", "verify.cu"]
+SOURCES = ["dsa_api.cu", "indexer_tc.cu", "topk.cu", "topk_cluster.cu", "attn_tc.cu", "dsa_noalloc.cu", "verify.cu",
+           "shard.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I", INCLUDE, "-I", CSRC]

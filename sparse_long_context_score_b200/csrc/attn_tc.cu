@@ -114,7 +114,7 @@ struct AttnMaps {
 // 13 warps: one SM sub-partition hosts four of them, so 128 registers per thread at most
 __global__ void __launch_bounds__(kThreadsA, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const int32_t* __restrict__ idx, int T, int N,
-               int H, int k, int chunk, float scale_log2, int q_early, float* __restrict__ partials,
+               int H, int k, int chunk, float scale_log2, int q_early, long long idx_offset, float* __restrict__ partials,
                int* __restrict__ err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -200,7 +200,10 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const int key = tile * kKeys + r0 + 4 * g + rsub;
-        out[g] = (tile < ntiles && key < nkeys) ? __ldg(&sel[key]) : -1;
+        // a selected global position, as a row of this cache (which holds positions
+        // [idx_offset, idx_offset + N)); -1 when it is padding or outside
+        const long long gp = (tile < ntiles && key < nkeys) ? (long long)__ldg(&sel[key]) - idx_offset : -1;
+        out[g] = gp >= 0 && gp < N ? (int)gp : -1;
       }
     };
     int cur[4], nxt[4];
@@ -454,6 +457,9 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   if (threadIdx.x < 64) {
     const int h = threadIdx.x;
     s_coef[h] = split_mode ? 1.f : (s_l[h] > 0.f ? 1.f / s_l[h] : 0.f);
+    // natural log-sum-exp of the logits: m and l are in base 2 (sum_j 2^(z_j) = 2^m l)
+    if (!split_mode && layers.lse[layer] && h < H)
+      layers.lse[layer][(size_t)row * H + h] = s_l[h] > 0.f ? (s_m[h] + log2f(s_l[h])) * 0.69314718055994531f : -INFINITY;
   }
   __syncthreads();  // s_coef
   // Twelve warps, three per TMEM lane quarter, take the eight 32-column chunks of O^T (TMEM
@@ -534,6 +540,8 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
 #pragma unroll
       for (int sp = 0; sp < kMaxSplits; ++sp)
         if (sp < nsplit) s_cs[sp * 64 + h] = (den > 0.f && mr[sp] != -INFINITY) ? exp2f(mr[sp] - M) / den : 0.f;
+      if (split == 0 && layers.lse[layer] && h < H)
+        layers.lse[layer][(size_t)row * H + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
     }
     // this CTA has read the other splits' shared memory: they may exit once all have
     cluster_arrive();
@@ -682,8 +690,8 @@ size_t attn_workspace_bytes(long long rows, int L, int, int k, int sm_budget) {
 }
 
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                                  int k, float scale, void* ws, size_t ws_bytes, bool q_early, int sm_budget,
-                                  cudaStream_t stream) {
+                                  int k, float scale, long long idx_offset, void* ws, size_t ws_bytes, bool q_early,
+                                  int sm_budget, cudaStream_t stream) {
   const long long rows = (long long)B * T;
   AttnMaps maps;
   for (int l = 0; l < L; ++l)
@@ -712,7 +720,7 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f,
-                            q_early ? 1 : 0, static_cast<float*>(ws), err);
+                            q_early ? 1 : 0, idx_offset, static_cast<float*>(ws), err);
 }
 
 cudaError_t attn_error_word(int** p) { return g_err_addr.get(g_attn_tc_error, p); }

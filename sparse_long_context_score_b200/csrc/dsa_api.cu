@@ -138,7 +138,7 @@ cudaError_t enqueue_group(const GroupCall& c, unsigned char* base, const GroupLa
     if ((e = launch_topk(scores, c.B, c.T, c.N, c.q_pos0, c.k, c.idx, tws, fused_hist, tail_sms, stream)) != cudaSuccess)
       return e;
   }
-  return launch_sparse_attn_tc(c.layers, c.L, c.idx, c.B, c.T, c.N, c.H, c.k, c.scale, base + g.attn_off, g.attn_bytes,
+  return launch_sparse_attn_tc(c.layers, c.L, c.idx, c.B, c.T, c.N, c.H, c.k, c.scale, 0, base + g.attn_off, g.attn_bytes,
                                /*q_early=*/c.compute_indices != 0, tail_sms, stream);
 }
 
@@ -274,7 +274,7 @@ dsa_status dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const int32_t*
   layers.kv[0] = kv;
   layers.out[0] = out;
   return cuda_status(
-      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, workspace, workspace_bytes, false, 0, stream));
+      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, 0, workspace, workspace_bytes, false, 0, stream));
 }
 
 dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t* ik, const uint16_t* const* q,
@@ -373,6 +373,50 @@ dsa_status dsa_decode_step(const dsa_group_io* groups, int G, int L, int B, int 
   if ((e = cudaEventRecord(ev->join, side)) != cudaSuccess || (e = cudaStreamWaitEvent(stream, ev->join, 0)) != cudaSuccess)
     return cuda_status(e);
   return DSA_OK;
+}
+
+dsa_status dsa_sparse_attn_shard(const uint16_t* q, const uint16_t* kv, const int32_t* idx, int B, int T, int N,
+                                 long long offset, int H, int k, float scale, float* out, float* lse, void* workspace,
+                                 size_t workspace_bytes, cudaStream_t stream) {
+  if (!q || !kv || !idx || !out || !lse || !sizes_ok(B, T, N) || k <= 0 || H <= 0 || offset < 0)
+    return DSA_ERR_INVALID_ARG;
+  if (k > DSA_MAX_TOPK || !heads_supported(H)) return DSA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(kv, 16) || !aligned(idx, 4) || !aligned(out, 16) || !aligned(lse, 4))
+    return DSA_ERR_INVALID_ARG;
+  const size_t need = attn_workspace_bytes((long long)B * T, 1, H, k);
+  if (need && (!workspace || workspace_bytes < need || !aligned(workspace, 256))) return DSA_ERR_WORKSPACE;
+  AttnLayers layers{};
+  layers.q[0] = q;
+  layers.kv[0] = kv;
+  layers.out[0] = out;
+  layers.lse[0] = lse;
+  return cuda_status(
+      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, offset, workspace, workspace_bytes, false, 0, stream));
+}
+
+dsa_status dsa_shard_candidates(const float* scores, const int32_t* idx, int B, int T, int N, int k, long long offset,
+                                float* cand_score, int32_t* cand_pos, cudaStream_t stream) {
+  if (!scores || !idx || !cand_score || !cand_pos || !sizes_ok(B, T, N) || k <= 0 || offset < 0 ||
+      offset + N > 0x7FFFFFFFLL)
+    return DSA_ERR_INVALID_ARG;
+  return cuda_status(launch_shard_candidates(scores, idx, (long long)B * T, N, k, offset, cand_score, cand_pos, stream));
+}
+
+dsa_status dsa_merge_candidates(const float* cand_score, const int32_t* cand_pos, int W, int B, int T, int kc, int k,
+                                int32_t* idx, cudaStream_t stream) {
+  if (!cand_score || !cand_pos || !idx || W <= 0 || B < 0 || T < 0 || kc <= 0 || k <= 0) return DSA_ERR_INVALID_ARG;
+  if (k > DSA_MAX_TOPK || (long long)W * kc > 8 * DSA_MAX_TOPK) return DSA_ERR_UNSUPPORTED;
+  if ((long long)B * T == 0) return DSA_OK;
+  return cuda_status(launch_merge_candidates(cand_score, cand_pos, W, (long long)B * T, kc, k, idx, stream));
+}
+
+dsa_status dsa_merge_partials(const float* outs, const float* lses, int W, int B, int T, int H, float* out,
+                              cudaStream_t stream) {
+  if (!outs || !lses || !out || W <= 0 || B < 0 || T < 0 || H <= 0) return DSA_ERR_INVALID_ARG;
+  if (!aligned(outs, 16) || !aligned(out, 16) || !aligned(lses, 4)) return DSA_ERR_INVALID_ARG;
+  const long long R = (long long)B * T * H;
+  if (R == 0) return DSA_OK;
+  return cuda_status(launch_merge_partials(outs, lses, W, R, out, stream));
 }
 
 dsa_status dsa_verify(const float* p, const float* q, const int32_t* draft, const float* u, const float* u2, int B,

@@ -92,6 +92,7 @@ struct AttnLayers {
   const uint16_t* q[kMaxLayers];
   const uint16_t* kv[kMaxLayers];
   float* out[kMaxLayers];
+  float* lse[kMaxLayers];  // optional [rows][H] natural log-sum-exp of the logits (nullptr: none)
 };
 
 constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core attention (a split's granularity)
@@ -132,8 +133,18 @@ cudaError_t launch_topk_cluster(const float* scores, int B, int T, int N, long l
 
 // q_early: the kernel before it in the stream does not write the queries (it is the
 // group's own top-k), so they are loaded before that kernel completes
+// idx_offset: the cache holds global positions [idx_offset, idx_offset + N); selected
+// positions outside it are skipped (a context shard)
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
-                                  int k, float scale, void* ws, size_t ws_bytes, bool q_early, int sm_budget,
+                                  int k, float scale, long long idx_offset, void* ws, size_t ws_bytes, bool q_early,
+                                  int sm_budget, cudaStream_t stream);
+
+// context-sharded decode (shard.cu)
+cudaError_t launch_shard_candidates(const float* scores, const int32_t* idx, long long rows, int Ns, int k,
+                                    long long offset, float* cand_score, int32_t* cand_pos, cudaStream_t stream);
+cudaError_t launch_merge_candidates(const float* cand_score, const int32_t* cand_pos, int W, long long rows, int kc,
+                                    int k, int32_t* idx, cudaStream_t stream);
+cudaError_t launch_merge_partials(const float* outs, const float* lses, int W, long long R, float* out,
                                   cudaStream_t stream);
 
 }  // namespace dsa

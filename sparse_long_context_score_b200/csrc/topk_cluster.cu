@@ -290,9 +290,12 @@ topk_cluster_kernel(const float* __restrict__ scores, int T, int N, long long q_
       }
     }
     // this CTA's b* elements, compacted into its list (at most `count` <= kMergeCap)
-    uint32_t n_loc = 0, n_above = 0;
-    uint32_t j = cta_excl_scan((uint32_t)__popc(cand_bits), sm, n_loc);
-    (void)cta_excl_scan((uint32_t)__popc(above_bits), sm, n_above);
+    // one scan of both counts: candidates in the low 16 bits, elements above b* in the high
+    // 16 (at most 1024 x KPT <= 32768 of either per CTA)
+    uint32_t packed_total = 0;
+    uint32_t j = cta_excl_scan((uint32_t)__popc(cand_bits) | ((uint32_t)__popc(above_bits) << 16), sm,
+                               packed_total) & 0xFFFFu;
+    const uint32_t n_loc = packed_total & 0xFFFFu, n_above = packed_total >> 16;
     for (uint32_t m = cand_bits; m; m &= m - 1) {
       const int step = __ffs(m) - 1;
       if (j < (uint32_t)kMergeCap) sm.m.loc[j] = comp(seg0 + 32 * step + lane);
