@@ -114,3 +114,23 @@ def test_decode_step_matches_oracle(dsa, orc, B, G, in_order):
         assert np.array_equal(host(groups[g]["idx"]), ridx), f"group {g}"
         for l in range(w.L):
             assert_close(host(groups[g]["outs"][l]), routs[l], f"group {g} layer {l}")
+
+
+@pytest.mark.parametrize("case", ["flat_rows", "short_rows_padded", "mixed"])
+def test_decode_select_edge_rows(dsa, orc, case):
+    """Decode groups with degenerate rows: every score equal (all-zero keys: the threshold
+    bin is the whole row, ties to the lower positions), rows shorter than k (kept whole,
+    padded), and one flat row among ordinary ones.  The index lists equal the oracle's."""
+    N = {"flat_rows": 20000, "short_rows_padded": 1500, "mixed": 12000}[case]
+    w = C.scaled(C.WORKLOADS["decode128k"], B=3, N=N, q_pos0=N - 1)
+    iq, wt, ik, qs, kvs = C.host_group_inputs(w)
+    if case == "flat_rows":
+        ik = np.zeros_like(ik)
+    if case == "mixed":
+        ik[1] = 0                                     # one flat row among ordinary ones
+    idx, outs = dsa.dsa_group_forward(dev_bf16(iq), dev(wt), dev_bf16(ik), [dev_bf16(x) for x in qs],
+                                      [dev_bf16(x) for x in kvs], w.q_pos0, w.k, C.SCALE)
+    ridx, routs = orc.group_forward(iq, wt, ik, qs, kvs, w.q_pos0, w.k, C.SCALE)
+    assert np.array_equal(host(idx), ridx)
+    assert_close(host(outs[0]), routs[0], f"{case} layer 0")
+    assert dsa.dsa_check_device_status() == 0
