@@ -259,8 +259,10 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     dsa.lib()
     groups = make_inputs(w, device, rank)
     micro = args.schedule == "micro" and w.T == 1 and w.steps == 1 and w.B >= 2
-    # the E4M3 index format runs through dsa_decode_step (in order: side = stream)
-    use_step = micro or (w.index_fp8 and w.T == 1 and w.steps == 1)
+    # a decode step (one query per sequence, no draft steps) runs through dsa_decode_step, in
+    # order (side = stream) unless micro-batched; MTP drafting and prefill through
+    # dsa_group_forward
+    use_step = micro or (w.T == 1 and w.steps == 1)
     if w.index_fp8 and not use_step:
         raise ValueError("the E4M3 index format runs through the decode step only")
     ws = dsa.decode_workspace(w.B, w.N, w.k, w.H, w.L, device) if use_step else \

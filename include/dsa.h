@@ -221,7 +221,10 @@ dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t 
  * side == stream, the groups run in order over the whole batch on `stream`, exactly like
  * one dsa_group_forward per group (on B200 this in-order step is the faster of the two at
  * the decode shapes measured: the top-k and attention are latency-bound and take nearly
- * as long for half a batch as for all of it).
+ * as long for half a batch as for all of it).  A decode step reads each selected row once,
+ * so the attention gathers them under an L2 evict-first policy (dsa_group_forward keeps the
+ * default policy: its caller may re-read the rows, as MTP draft steps do); the results are
+ * the same either way.
  *   groups[g]   the group's tensors for all B sequences, in the layouts of
  *               dsa_group_forward with T = 1 (q, kv, out: L entries each)
  *   workspace   dsa_decode_workspace_size(B, N, k, H, L) bytes, 256-byte aligned

@@ -25,7 +25,8 @@
 //               own rows' indices, and one instruction moves four whole 128-byte lines),
 //               waits for its own copies, fences them to the async proxy and arrives on the
 //               stage barrier, so both stages gather at once; the row indices of the warp's
-//               next tile are loaded while the current one is copied.  (Random 1152-byte
+//               next tile are loaded while the current one is copied; a decode step's
+//               rows, read once, are copied under an L2 evict-first policy.  (Random 1152-byte
 //               rows are too small for TMA: measured on B200 with the same bytes in flight,
 //               a 128-byte box per row reached 0.57 TB/s, 4-row gather boxes 1.6 TB/s, one
 //               bulk copy per row 2.8 TB/s, 16-byte cp.async 4.9 TB/s.)
@@ -111,10 +112,14 @@ struct AttnMaps {
   CUtensorMap q[kMaxLayers];
 };
 
+// kernel flags
+constexpr int kAttnQEarly = 1;     // the queries may be loaded before the preceding kernel ends
+constexpr int kAttnRowsOnce = 2;   // gathered rows are read once: L2 evict-first policy
+
 // 13 warps: one SM sub-partition hosts four of them, so 128 registers per thread at most
 __global__ void __launch_bounds__(kThreadsA, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const int32_t* __restrict__ idx, int T, int N,
-               int H, int k, int chunk, float scale_log2, int q_early, long long idx_offset, float* __restrict__ partials,
+               int H, int k, int chunk, float scale_log2, int flags, long long idx_offset, float* __restrict__ partials,
                int* __restrict__ err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -206,6 +211,8 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         out[g] = gp >= 0 && gp < N ? (int)gp : -1;
       }
     };
+    const bool rows_once = (flags & kAttnRowsOnce) != 0;
+    const uint64_t row_policy = l2_evict_first_policy();
     int cur[4], nxt[4];
     load_index(ps, cur);
     for (int i = ps; i < ntiles; i += kStages) {
@@ -228,8 +235,13 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         const uint16_t* src = kvb + (size_t)(v ? cur[g] : 0) * kDqk + c8 * 8;
         const int r = r0 + 4 * g + rsub;
         const uint32_t dst = st + r * 128 + ((c8 ^ (r & 7)) << 4);
+        if (rows_once) {
 #pragma unroll
-        for (int m = 0; m < kBlocks; ++m) cp_async_16(dst + m * kBlockBytes, src + m * 64, v ? 16 : 0);
+          for (int m = 0; m < kBlocks; ++m) cp_async_16_hint(dst + m * kBlockBytes, src + m * 64, v ? 16 : 0, row_policy);
+        } else {
+#pragma unroll
+          for (int m = 0; m < kBlocks; ++m) cp_async_16(dst + m * kBlockBytes, src + m * 64, v ? 16 : 0);
+        }
       }
       cp_async_commit();
       cp_async_wait<0>();
@@ -248,7 +260,7 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
       // the queries may be read before the preceding kernel completes only when the caller
       // knows that kernel does not write them (the top-k of the same group)
       tma_prefetch(&maps.q[layer]);
-      if (!q_early) grid_dep_wait();
+      if (!(flags & kAttnQEarly)) grid_dep_wait();
       const CUtensorMap* qm = &maps.q[layer];
       mbar_arrive_expect_tx(qfull_bar, kQBytes);
       for (int kb = 0; kb < kBlocks; ++kb) tma_load_2d(sQ + kb * kQBlockBytes, qm, qfull_bar, 64 * kb, row * H);
@@ -691,7 +703,7 @@ size_t attn_workspace_bytes(long long rows, int L, int, int k, int sm_budget) {
 
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
                                   int k, float scale, long long idx_offset, void* ws, size_t ws_bytes, bool q_early,
-                                  int sm_budget, cudaStream_t stream) {
+                                  bool rows_once, int sm_budget, cudaStream_t stream) {
   const long long rows = (long long)B * T;
   AttnMaps maps;
   for (int l = 0; l < L; ++l)
@@ -719,8 +731,9 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  const int flags = (q_early ? kAttnQEarly : 0) | (rows_once ? kAttnRowsOnce : 0);
   return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f,
-                            q_early ? 1 : 0, idx_offset, static_cast<float*>(ws), err);
+                            flags, idx_offset, static_cast<float*>(ws), err);
 }
 
 cudaError_t attn_error_word(int** p) { return g_err_addr.get(g_attn_tc_error, p); }

@@ -81,6 +81,7 @@ struct GroupCall {
   long long q_pos0;
   float scale;
   int32_t* idx;
+  bool rows_once = false;  // the attention's rows are read once (a decode step)
 };
 
 dsa_status check_group(const void* iq, const float* w, const void* ik, bool f8, const uint16_t* const* q,
@@ -128,6 +129,11 @@ cudaError_t enqueue_group(const GroupCall& c, unsigned char* base, const GroupLa
     // in decode the indexer folds the first radix digit of the select into its epilogue
     const int sms = device_sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
+    // A bf16 decode indexer given all SMs is no faster than one on six sevenths of them
+    // (the key stream saturates HBM either way); the SMs it leaves free take the first
+    // CTAs of the top-k and the attention, launched behind it, before it ends (measured on
+    // B200 at 128K and 1M contexts: 2-3% off the step; the E4M3 indexer gains nothing).
+    if (idx_sms == 0 && c.T == 1 && !c.f8 && c.B <= sms * 6 / 7) idx_sms = sms * 6 / 7;
     const int cap = idx_sms > 0 && idx_sms < sms ? idx_sms : sms;
     const bool fused_hist = c.T == 1 && c.B <= cap;
     if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess) return e;
@@ -139,7 +145,7 @@ cudaError_t enqueue_group(const GroupCall& c, unsigned char* base, const GroupLa
       return e;
   }
   return launch_sparse_attn_tc(c.layers, c.L, c.idx, c.B, c.T, c.N, c.H, c.k, c.scale, 0, base + g.attn_off, g.attn_bytes,
-                               /*q_early=*/c.compute_indices != 0, tail_sms, stream);
+                               /*q_early=*/c.compute_indices != 0, c.rows_once, tail_sms, stream);
 }
 
 // Events of dsa_decode_step, created once per device and host thread.
@@ -274,7 +280,7 @@ dsa_status dsa_sparse_attn(const uint16_t* q, const uint16_t* kv, const int32_t*
   layers.kv[0] = kv;
   layers.out[0] = out;
   return cuda_status(
-      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, 0, workspace, workspace_bytes, false, 0, stream));
+      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, 0, workspace, workspace_bytes, false, false, 0, stream));
 }
 
 dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t* ik, const uint16_t* const* q,
@@ -339,6 +345,7 @@ dsa_status dsa_decode_step(const dsa_group_io* groups, int G, int L, int B, int 
       if (st != DSA_OK) return st;
       c.q_pos0 = N - 1;
       c.scale = scale;
+      c.rows_once = true;
     }
   }
   if (!workspace || workspace_bytes < need || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE;
@@ -391,7 +398,7 @@ dsa_status dsa_sparse_attn_shard(const uint16_t* q, const uint16_t* kv, const in
   layers.out[0] = out;
   layers.lse[0] = lse;
   return cuda_status(
-      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, offset, workspace, workspace_bytes, false, 0, stream));
+      launch_sparse_attn_tc(layers, 1, idx, B, T, N, H, k, scale, offset, workspace, workspace_bytes, false, false, 0, stream));
 }
 
 dsa_status dsa_shard_candidates(const float* scores, const int32_t* idx, int B, int T, int N, int k, long long offset,

@@ -102,7 +102,8 @@ int attn_split_chunk(int k, int nsplit);
 size_t attn_workspace_bytes(long long rows, int L, int H, int k, int sm_budget = 0);
 
 // tcgen05 indexer (T == 1: decode, one query per MMA; T > 1: 8 queries per MMA).  With a
-// histogram pointer (decode only, B <= 148) the first radix digit of the select is counted.
+// histogram pointer (decode only, B no more than the SMs of the budget; zeroed by the
+// caller) the first radix digit of the select is counted.
 // f8: q and k hold E4M3 bytes instead of bf16 (the same layouts, one byte per element).
 cudaError_t launch_index_score_tc(const void* q, const float* w, const void* k, int B, int T, int N, long long q_pos0,
                                   float* scores, uint32_t* hist, int sm_budget, bool f8, cudaStream_t stream);
@@ -135,9 +136,12 @@ cudaError_t launch_topk_cluster(const float* scores, int B, int T, int N, long l
 // group's own top-k), so they are loaded before that kernel completes
 // idx_offset: the cache holds global positions [idx_offset, idx_offset + N); selected
 // positions outside it are skipped (a context shard)
+// rows_once: the caller reads the selected rows once (a decode step), so they are gathered
+// under an L2 evict-first policy; otherwise (MTP draft steps, prefill) they may stay in L2
+// for the next call or the next query
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
                                   int k, float scale, long long idx_offset, void* ws, size_t ws_bytes, bool q_early,
-                                  int sm_budget, cudaStream_t stream);
+                                  bool rows_once, int sm_budget, cudaStream_t stream);
 
 // context-sharded decode (shard.cu)
 cudaError_t launch_shard_candidates(const float* scores, const int32_t* idx, long long rows, int Ns, int k,

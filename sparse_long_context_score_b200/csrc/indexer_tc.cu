@@ -11,8 +11,9 @@
 // Warp roles (one CTA per SM, persistent over a contiguous range of (query group, key
 // tile) items):
 //   warp 0      TMA producer: 128x128 key tiles (bf16: two 64-column boxes; E4M3: one
-//               128-column box; 128-byte swizzle) into a ring of shared-memory stages; the
-//               query group once per group change;
+//               128-column box; 128-byte swizzle) into a ring of shared-memory stages (in
+//               decode under an L2 evict-first policy: each tile is read once); the query
+//               group once per group change;
 //   warp 1      allocates TMEM; one thread issues tcgen05.mma into a ring of TMEM
 //               accumulators (decode: 4 x 32 columns; prefill: 2 x 256) and commits to the
 //               stage / accumulator barriers;
@@ -179,6 +180,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
     if (lane == 0) {
       Cursor cur;
       cur.start(it, begin, end);
+      const uint64_t key_policy = l2_evict_first_policy();
       int stage = 0;
       uint32_t phase = 0, qfree_phase = 0;
       int cur_qg = -1;
@@ -204,8 +206,13 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constan
         const int b = cur.qg / it.G;
         const uint32_t dst = sA + stage * C::kStageBytesA;
         mbar_arrive_expect_tx(full_bar(stage), C::kStageBytesA);
-        for (int hh = 0; hh < C::kHalves; ++hh)
-          tma_load_3d(dst + hh * kHalfBytesA, &kmap, full_bar(stage), 64 * hh, cur.tile * kTileKeys, b);
+        for (int hh = 0; hh < C::kHalves; ++hh) {
+          if (QG == 1)  // decode: every key tile is read once per launch
+            tma_load_3d_hint(dst + hh * kHalfBytesA, &kmap, full_bar(stage), 64 * hh, cur.tile * kTileKeys, b,
+                             key_policy);
+          else          // prefill: every query group re-reads the keys, which stay in L2
+            tma_load_3d(dst + hh * kHalfBytesA, &kmap, full_bar(stage), 64 * hh, cur.tile * kTileKeys, b);
+        }
         ++issued;
         if (++stage == C::kStages) {
           stage = 0;
@@ -447,10 +454,10 @@ cudaError_t launch_tc(const void* q, const float* w, const void* k, int B, int T
     const long long v = visible_count(N, q_pos0, tl);
     total += (v + kTileKeys - 1) / kTileKeys;
   }
-  if (total == 0) return cudaSuccess;
   // persistent: one CTA per SM of the budget (all SMs by default)
   const int sms = device_sm_count();
   if (sms <= 0) return cudaErrorInvalidDevice;
+  if (total == 0) return cudaSuccess;
   const int cap = sm_budget > 0 && sm_budget < sms ? sm_budget : sms;
   const int grid = (int)(total < cap ? total : cap);
   indexer_tc_kernel<QG, kHist, kF8><<<grid, C::kThreads, C::kSmem, stream>>>(kmap, qmap, w, B, T, N, q_pos0, total, scores,
