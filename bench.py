@@ -516,8 +516,8 @@ def workload_config(w, world: int) -> dict:
 
 
 def launches_per_group(w, sms: int = 148, long_per_sm: int = 4) -> int:
-    """libdsa kernels one dsa_group_forward launches: the indexer, the top-k and one
-    attention launch for all layers.  The top-k is one kernel for rows a cluster holds
+    """libdsa kernels one dsa_group_forward launches: the indexer, the top-k and the
+    attention of all layers (one launch, plus the split combine when it splits keys).  The top-k is one kernel for rows a cluster holds
     (decode shapes) and for long rows whose CTAs (one per 8192 scores) all fit the GPU at
     once (a cooperative launch: `long_per_sm` of them per SM); otherwise a select and a
     compact kernel, plus a histogram kernel when the indexer does not count the first
@@ -536,16 +536,24 @@ def launches_per_group(w, sms: int = 148, long_per_sm: int = 4) -> int:
     long_rows = nchunks <= 512 and rows * nchunks <= long_per_sm * sms
     fused_hist = w.T == 1 and w.B <= sms
     topk = 1 if (cluster or long_rows) else (2 if fused_hist else 3)
-    return 1 + topk + 1
+    return 1 + topk + attn_launches(w, sms)
+
+
+def attn_launches(w, sms: int = 148) -> int:
+    """Launches of one attention call over the group's L layers: the attention kernel, and
+    the split combine when the (row, layer) units are few enough for their keys to be split
+    over several CTAs (mirrors attn_num_splits: at most one CTA per SM in all)."""
+    units = w.B * w.T * w.L
+    return 2 if (w.k > 64 and 2 * units <= sms) else 1
 
 
 def step_launches(w, micro: bool) -> int:
     """libdsa kernels of one step: per group, per micro-batch (two halves of the batch when
     the step is micro-batched), launches_per_group of that micro-batch; every MTP draft
-    step after the first adds one attention launch."""
+    step after the first adds one attention call (L = 1)."""
     from synth import configs as C
     if not micro:
-        return (launches_per_group(w) + (w.steps - 1)) * w.groups
+        return (launches_per_group(w) + (w.steps - 1) * attn_launches(C.scaled(w, L=1))) * w.groups
     b0 = (w.B + 1) // 2
     halves = [C.scaled(w, B=b0), C.scaled(w, B=w.B - b0)]
     return sum(launches_per_group(h, sms=148 // 3) for h in halves if h.B > 0) * w.groups

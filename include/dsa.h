@@ -179,10 +179,11 @@ dsa_status dsa_topk_noalloc(const float *scores, int B, int T, int N, long long 
  *   out  [B, T, H, 512] f32    softmax_j(scale * q . kv[idx_j]) weighted sum of values;
  *                              zero when a row selects nothing
  * bf16 operands, f32 accumulation and softmax.  H in {16, 32, 48, 64}.
- * When few (row, layer) units are launched, each one's keys are split over up to 8 CTAs
- * whose partial outputs meet in `workspace` (one [64][512] f32 block per split, 128 KB);
- * dsa_workspace_size(B, T, N, k, H, 1) covers it.  Otherwise (e.g. long prefill chunks)
- * no workspace is read and it may be NULL.
+ * When few (row, layer) units are launched, each one's keys are split over up to 32 CTAs
+ * (one per SM of the GPU in all) whose partial outputs meet in `workspace` (per split a
+ * [64][512] f32 block and 64 (max, sum) pairs, 128.5 KB) and are merged by a second kernel
+ * launched behind the first; dsa_workspace_size(B, T, N, k, H, 1) covers it.  Otherwise
+ * (e.g. long prefill chunks) no workspace is read and it may be NULL.
  */
 dsa_status dsa_sparse_attn(const uint16_t *q, const uint16_t *kv, const int32_t *idx,
                            int B, int T, int N, int H, int k, float scale, float *out,

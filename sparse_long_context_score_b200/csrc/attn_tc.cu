@@ -39,13 +39,12 @@
 //               of its own it does not wait behind the next S, whose MMAs its own
 //               interleave with in the tensor pipe, and a stage is released as soon as its
 //               PV completes.
-// The key splits of one (row, layer) run as one thread-block cluster.  After the main
-// loop the splits exchange their running max and sum per head through distributed shared
-// memory; each split scales its unnormalised O by its share of the normaliser and writes it
-// from TMEM to a global partial buffer (L2-resident); after one more cluster barrier split
-// r sums slice r of the [H][512] output over the partials.  A single split writes the
-// normalised output directly.  The launch waits for the preceding kernel (programmatic
-// dependent launch) only where it reads that kernel's results.
+// A (row, layer) whose keys are split over several CTAs: each split writes its unnormalised
+// O (straight from TMEM, 32 consecutive value dims of a head per warp store) and its
+// running max and sum per head to a global partial block (L2-resident), and the combine
+// kernel launched behind it (programmatic dependent launch: its CTAs wait on the device
+// for this grid) merges the splits.  A single split writes the normalised output directly.
+// The launch waits for the preceding kernel only where it reads that kernel's results.
 // All mbarrier waits are bounded (sm100.cuh).
 #include <cudaTypedefs.h>
 
@@ -83,7 +82,7 @@ constexpr int kThreadsA = (kPvWarp + 1) * 32;      // 448
 static_assert(kThreadsA == 448, "8 gather, 1 S, 4 softmax and 1 PV warp");
 static_assert(kRowsPerWarp == 16, "a gather warp copies 4 x 4 rows");
 constexpr float kRescaleLog2 = 8.f;
-constexpr int kMaxSplits = 8;                    // key splits of one (row, layer): one portable cluster
+constexpr int kMaxSplits = 32;                   // key splits of one (row, layer): a combine warp's lanes
 
 constexpr int kOffQ = 0;
 constexpr int kOffStage = kOffQ + kQBytes;
@@ -93,7 +92,7 @@ constexpr int kOffM = kOffL + 64 * 4;            // [64] f32
 constexpr int kOffCoef = kOffM + 64 * 4;         // [64] f32: this split's share of the normaliser
 constexpr int kOffMask = kOffCoef + 64 * 4;      // [kStages] u64: valid rows of the tile in the stage
 constexpr int kOffVote = kOffMask + kStages * 8;  // [2] u32 (tile parity): one byte per softmax warp
-constexpr int kNumBars = 2 * kStages + 12;
+constexpr int kNumBars = 2 * kStages + 11;
 constexpr int kOffBar = kOffVote + 8;
 constexpr int kOffTmem = kOffBar + kNumBars * 8;
 constexpr int kSmemA = kOffTmem + 16 + 1024;     // + alignment slack
@@ -105,8 +104,7 @@ constexpr int kTmemS = 256;    // S: 2 buffers x 64 columns, lanes 0..15 of each
 constexpr int kTmemCols = 512;
 
 constexpr int kPartialFloats = 64 * kDv;         // one split's [64][512] partial output
-constexpr int kCsOffset = kPartialFloats + 4 * kMaxSplits;  // floats from the staging buffer to c_s
-static_assert((kCsOffset + kMaxSplits * 64) * 4 <= kStages * kStageBytes, "staged O, received slices and c_s fit");
+constexpr int kPartialMl = 64 * 2;               // ... and its (m, l) per head
 
 struct AttnMaps {
   CUtensorMap q[kMaxLayers];
@@ -120,7 +118,7 @@ constexpr int kAttnRowsOnce = 2;   // gathered rows are read once: L2 evict-firs
 __global__ void __launch_bounds__(kThreadsA, 1)
 attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const int32_t* __restrict__ idx, int T, int N,
                int H, int k, int chunk, float scale_log2, int flags, long long idx_offset, float* __restrict__ partials,
-               int* __restrict__ err) {
+               float2* __restrict__ partial_ml, int* __restrict__ err) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
   const uint32_t sbase = smem_u32(smem);
@@ -144,7 +142,6 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   const uint32_t qfull_bar = bar0 + 8u * (2 * kStages + 8);
   const uint32_t grp_bar = bar0 + 8u * (2 * kStages + 9);
   const uint32_t sdone_bar = bar0 + 8u * (2 * kStages + 10);
-  const uint32_t rbar = bar0 + 8u * (2 * kStages + 11);  // split reduction: the slices landed
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + kOffTmem);
 
   const int split = blockIdx.x, row = blockIdx.y, layer = blockIdx.z;
@@ -154,6 +151,9 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
   const int j0 = split * chunk;
   const int nkeys = max(min(j0 + chunk, k) - j0, 0);
   const int ntiles = (nkeys + kKeys - 1) / kKeys;
+  // the split combine behind this grid may be scheduled once every CTA of it has started;
+  // it waits on the device for this grid to complete
+  grid_dep_launch();
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -170,7 +170,6 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     mbar_init(qfull_bar, 1);
     mbar_init(grp_bar, 128);
     mbar_init(sdone_bar, 1);
-    mbar_init(rbar, 1);
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -190,8 +189,8 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     const int ps = warp / kWarpsPerStage, wq = warp % kWarpsPerStage;
     const int r0 = kRowsPerWarp * wq;
     // the index list comes from the preceding kernel.  (Every other warp waits on the
-    // gather through the pipeline barriers, and the output is written only after the
-    // cluster barriers that follow this wait.)
+    // gather through the pipeline barriers, and the output is written only after the CTA
+    // barrier that follows this wait.)
     grid_dep_wait();
     const int32_t* sel = idx + (size_t)row * k + j0;
     const uint16_t* kvb = layers.kv[layer] + (size_t)b * N * kDqk;
@@ -453,31 +452,30 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
     }
   }
 
-  // ------------------------------------------------------------------ split reduction
-  //   out[h] = sum_s c_s[h] O_s[h],  c_s[h] = 2^(m_s[h] - M[h]) / sum_r 2^(m_r[h] - M[h]) l_r[h],
-  // M[h] = max_r m_r[h].  Every split stages its O (unnormalised; a single split: O / l) from
-  // TMEM as [H][512] f32 in its consumed stages and writes it with one bulk copy: to its
-  // partial block (L2-resident), or, for a single split, to the output.  After one cluster
-  // barrier split r reads every split's (m, l) through distributed shared memory, bulk-loads
-  // slice r of every split's partial, and writes slice r of the output.  Every thread passes
-  // the cluster barriers on every path (a failed wait above only skips work), so none of
-  // them can be left waiting.
+  // ------------------------------------------------------------------ epilogue
+  // A single split writes O / l; a split of several writes its unnormalised O to its
+  // [64][512] partial block and its (m, l) per head, which the combine kernel merges.
   tc_fence_before();
   __syncthreads();  // (m, l) of this split published; its MMAs have completed
   tc_fence_after();
   const bool split_mode = nsplit > 1;
+  const size_t unit = (size_t)layer * gridDim.y + row;
   if (threadIdx.x < 64) {
     const int h = threadIdx.x;
     s_coef[h] = split_mode ? 1.f : (s_l[h] > 0.f ? 1.f / s_l[h] : 0.f);
-    // natural log-sum-exp of the logits: m and l are in base 2 (sum_j 2^(z_j) = 2^m l)
-    if (!split_mode && layers.lse[layer] && h < H)
+    if (split_mode) {
+      partial_ml[(unit * nsplit + split) * 64 + h] = make_float2(s_m[h], s_l[h]);
+    } else if (layers.lse[layer] && h < H) {
+      // natural log-sum-exp of the logits: m and l are in base 2 (sum_j 2^(z_j) = 2^m l)
       layers.lse[layer][(size_t)row * H + h] = s_l[h] > 0.f ? (s_m[h] + log2f(s_l[h])) * 0.69314718055994531f : -INFINITY;
+    }
   }
   __syncthreads();  // s_coef
   // Twelve warps, three per TMEM lane quarter, take the eight 32-column chunks of O^T (TMEM
   // lane = value dim, column = head); for each head a warp stores 32 consecutive value dims
-  // (128 bytes, conflict-free) of the staging buffer.
-  float* obuf = reinterpret_cast<float*>(smem + kOffStage);
+  // (128 bytes) from its registers.  The output holds H heads, a partial block all 64.
+  float* dst = split_mode ? partials + (unit * nsplit + split) * kPartialFloats : layers.out[layer] + (size_t)row * H * kDv;
+  const int hmax = split_mode ? 64 : H;
   if (warp != kMmaWarp && warp != kPvWarp) {
     const int quarter = warp & 3;
     const int jw = warp < kProducerWarps ? warp >> 2 : 2;
@@ -496,92 +494,22 @@ attn_tc_kernel(const __grid_constant__ AttnMaps maps, AttnLayers layers, const i
         for (int c2 = 0; c2 < 32; ++c2) o0[c2] = o1[c2] = 0u;
       }
       {
-        const int hh = 32 * (c0 & 1), dim = 128 * (c0 >> 1) + 32 * quarter + lane;
+        const int hh = 32 * (c0 & 1), lim = hmax - hh;
+        float* d = dst + hh * kDv + 128 * (c0 >> 1) + 32 * quarter + lane;
+        const float* cf = s_coef + hh;
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) obuf[(hh + c2) * kDv + dim] = __uint_as_float(o0[c2]) * s_coef[hh + c2];
+        for (int c2 = 0; c2 < 32; ++c2)
+          if (c2 < lim) d[c2 * kDv] = __uint_as_float(o0[c2]) * cf[c2];
       }
       if (two) {
-        const int hh = 32 * (c1 & 1), dim = 128 * (c1 >> 1) + 32 * quarter + lane;
+        const int hh = 32 * (c1 & 1), lim = hmax - hh;
+        float* d = dst + hh * kDv + 128 * (c1 >> 1) + 32 * quarter + lane;
+        const float* cf = s_coef + hh;
 #pragma unroll
-        for (int c2 = 0; c2 < 32; ++c2) obuf[(hh + c2) * kDv + dim] = __uint_as_float(o1[c2]) * s_coef[hh + c2];
+        for (int c2 = 0; c2 < 32; ++c2)
+          if (c2 < lim) d[c2 * kDv] = __uint_as_float(o1[c2]) * cf[c2];
       }
     }
-    fence_proxy_async();  // the staged O is visible to the bulk copy (async proxy)
-  }
-  __syncthreads();
-  float* dst = split_mode ? partials + (((size_t)layer * gridDim.y + row) * nsplit + split) * kPartialFloats
-                          : layers.out[layer] + (size_t)row * H * kDv;
-  if (threadIdx.x == 0) {
-    bulk_store(dst, smem_u32(obuf), (uint32_t)(H * kDv * 4));
-    bulk_commit();
-    bulk_wait_all();  // written (and the staging buffer read)
-    fence_proxy_async_global();
-  }
-  if (split_mode) {
-    cluster_sync();  // every split's partial is in global memory and its (m, l) in shared memory
-    // this split's slice of the output: float4 e = h * 128 + d / 4 of the [H][512] block,
-    // a contiguous range of every split's partial, bulk-loaded into the staging buffer
-    const int total = H * (kDv / 4);
-    const int e0 = (int)((long long)split * total / nsplit), e1 = (int)((long long)(split + 1) * total / nsplit);
-    const uint32_t slice_bytes = (uint32_t)(e1 - e0) * 16u;
-    const float* part = partials + ((size_t)layer * gridDim.y + row) * nsplit * kPartialFloats;
-    if (threadIdx.x == 0 && slice_bytes > 0) {
-      fence_proxy_async_global();
-      mbar_arrive_expect_tx(rbar, slice_bytes * (uint32_t)nsplit);
-      for (int sp = 0; sp < nsplit; ++sp)
-        bulk_load(smem_u32(obuf) + (uint32_t)sp * slice_bytes, part + (size_t)sp * kPartialFloats + 4 * (size_t)e0,
-                  slice_bytes, rbar);
-    }
-    // c_s[h] of every split while the slices land; s_cs[s][h] sits past the received
-    // slices (nsplit slices of at most ceil(H * 128 / nsplit) float4: up to kMaxSplits - 1
-    // float4 more than the [H][512] block)
-    float* s_cs = obuf + kCsOffset;
-    if (threadIdx.x < 64) {
-      const int h = threadIdx.x;
-      float mr[kMaxSplits], lr[kMaxSplits];
-      float M = -INFINITY;
-#pragma unroll
-      for (int sp = 0; sp < kMaxSplits; ++sp) {
-        mr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_m + h), sp)) : -INFINITY;
-        lr[sp] = sp < nsplit ? ld_cluster_f32(cluster_map(smem_u32(s_l + h), sp)) : 0.f;
-        M = fmaxf(M, mr[sp]);
-      }
-      float den = 0.f;
-#pragma unroll
-      for (int sp = 0; sp < kMaxSplits; ++sp) den += (mr[sp] == -INFINITY ? 0.f : exp2f(mr[sp] - M)) * lr[sp];
-#pragma unroll
-      for (int sp = 0; sp < kMaxSplits; ++sp)
-        if (sp < nsplit) s_cs[sp * 64 + h] = (den > 0.f && mr[sp] != -INFINITY) ? exp2f(mr[sp] - M) / den : 0.f;
-      if (split == 0 && layers.lse[layer] && h < H)
-        layers.lse[layer][(size_t)row * H + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
-    }
-    // this CTA has read the other splits' shared memory: they may exit once all have
-    cluster_arrive();
-    __syncthreads();  // s_cs
-    bool landed = slice_bytes == 0 || mbar_wait(rbar, 0, err, 31);
-    if (!landed && slice_bytes > 0) landed = mbar_wait_drain(rbar, 0);  // the copies end before the CTA does
-    if (landed) {
-      const float4* recv = reinterpret_cast<const float4*>(obuf);
-      const int n4 = e1 - e0;
-      float4* out4 = reinterpret_cast<float4*>(layers.out[layer] + (size_t)row * H * kDv) + e0;
-      for (int e = (int)threadIdx.x; e < n4; e += kThreadsA) {
-        const int h = (e0 + e) >> 7;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int sp = 0; sp < kMaxSplits; ++sp) {
-          if (sp < nsplit) {
-            const float c = s_cs[sp * 64 + h];
-            const float4 v = recv[sp * n4 + e];
-            acc.x += c * v.x;
-            acc.y += c * v.y;
-            acc.z += c * v.z;
-            acc.w += c * v.w;
-          }
-        }
-        out4[e] = acc;
-      }
-    }
-    cluster_wait();
   }
   tc_fence_before();
   __syncthreads();
@@ -618,47 +546,61 @@ bool make_map_576(CUtensorMap* map, const void* base, long long rows, int box_ro
 
 SymbolAddress g_err_addr;
 
-// How many clusters of each size (1..kMaxSplits) of this kernel fit on the GPU at once,
-// per device; filled on the first launch on a device (before any stream capture).
-int g_cluster_fit[64][kMaxSplits + 1];
-
-cudaError_t query_cluster_fit() {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  for (int c = 1; c <= kMaxSplits; ++c) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(c, 1, 1);
-    cfg.blockDim = dim3(kThreadsA);
-    cfg.dynamicSmemBytes = kSmemA;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = c;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    int n = 0;
-    if ((e = cudaOccupancyMaxActiveClusters(&n, attn_tc_kernel, &cfg)) != cudaSuccess) return e;
-    g_cluster_fit[dev][c] = n;
+// Merges the key splits of every (row, layer):
+//   out[h] = sum_s 2^(m_s[h] - M[h]) O_s[h] / sum_s 2^(m_s[h] - M[h]) l_s[h],  M[h] = max_s m_s[h],
+// and the natural log-sum-exp (M[h] + log2 of the denominator) * ln 2 when asked.  One CTA
+// per (8 heads, row, layer); warp w takes head 8 x + w: lane s < nsplit reads split s's
+// (m, l) and forms its coefficient, then every lane sums four float4 of the head's 512
+// values over the splits.  Launched behind the attention as its programmatic dependent.
+__global__ void __launch_bounds__(256) attn_combine_kernel(const float* __restrict__ partials,
+                                                           const float2* __restrict__ partial_ml, AttnLayers layers,
+                                                           int H, int nsplit) {
+  grid_dep_wait();  // the attention's partials
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x * 8 + warp, row = blockIdx.y, layer = blockIdx.z;
+  if (h >= H) return;
+  const size_t unit = (size_t)layer * gridDim.y + row;
+  float m = -INFINITY, l = 0.f;
+  if (lane < nsplit) {
+    const float2 v = partial_ml[(unit * nsplit + lane) * 64 + h];
+    m = v.x;
+    l = v.y;
   }
-  return cudaSuccess;
+  float M = m;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+  float c = m == -INFINITY ? 0.f : exp2f(m - M);  // (M is finite when m is)
+  float den = c * l;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xFFFFFFFFu, den, o);
+  c = den > 0.f ? c / den : 0.f;
+  if (lane == 0 && layers.lse[layer])
+    layers.lse[layer][(size_t)row * H + h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+  const float4* p = reinterpret_cast<const float4*>(partials + unit * nsplit * kPartialFloats) + h * (kDv / 4) + lane;
+  float4 acc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+  for (int sp = 0; sp < nsplit; ++sp) {
+    const float cs = __shfl_sync(0xFFFFFFFFu, c, sp);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldcg(p + (size_t)sp * (kPartialFloats / 4) + 32 * i);
+      acc[i].x += cs * v.x;
+      acc[i].y += cs * v.y;
+      acc[i].z += cs * v.z;
+      acc[i].w += cs * v.w;
+    }
+  }
+  float4* out = reinterpret_cast<float4*>(layers.out[layer] + ((size_t)row * H + h) * kDv) + lane;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) out[32 * i] = acc[i];
 }
 
-// kernel attribute and cluster-fit table, once per device
+// kernel attributes, once per device
 cudaError_t attn_setup() {
   static DeviceOnce once;
-  return once.run([] {
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA);
-    return e != cudaSuccess ? e : query_cluster_fit();
-  });
-}
-
-const int* cluster_fit_of_device() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  return g_cluster_fit[dev];
+  return once.run([] { return cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemA); });
 }
 
 // splits of the launch on the current device, within an SM budget (0: all SMs); 0 when
@@ -666,7 +608,7 @@ const int* cluster_fit_of_device() {
 int launch_splits(long long rows, int L, int k, int sm_budget) {
   const int sms = device_sm_count();
   if (sms <= 0 || attn_setup() != cudaSuccess) return 0;
-  return attn_num_splits(rows, L, k, sm_budget > 0 && sm_budget < sms ? sm_budget : sms, cluster_fit_of_device());
+  return attn_num_splits(rows, L, k, sm_budget > 0 && sm_budget < sms ? sm_budget : sms);
 }
 
 }  // namespace
@@ -677,28 +619,27 @@ int attn_split_chunk(int k, int nsplit) {
   return (chunk + kAttnTile - 1) / kAttnTile * kAttnTile;
 }
 
-// Splits per (query row, layer): the most (<= kMaxSplits, at most one CTA per SM of the
-// budget in total) whose clusters all fit on the GPU at once -- a second wave of clusters
-// would double the time.  Without the device's figures (fit == nullptr) the SM budget
-// alone decides.
-int attn_num_splits(long long rows, int L, int k, int sm_budget, const int* fit) {
+// Splits per (query row, layer): the most (<= kMaxSplits, one per 64-row tile at most)
+// with at most one CTA per SM of the budget in total -- a second wave of CTAs would double
+// the time.
+int attn_num_splits(long long rows, int L, int k, int sm_budget) {
   const long long units = rows * L > 0 ? rows * L : 1;
   const long long max_ns = (k + kAttnTile - 1) / kAttnTile;
   int best = 1;
   for (int ns = 1; ns <= kMaxSplits && ns <= max_ns; ++ns) {
     if (units * ns > sm_budget) break;
-    if (fit && ns > 1 && units > fit[ns]) continue;  // (a size that cannot run at all reports 0)
     best = ns;
   }
   const int chunk = attn_split_chunk(k, best);
   return (k + chunk - 1) / chunk;
 }
 
-// The split partials: one [64][512] f32 block per (layer, row, split) when a (row, layer)
-// is split, none otherwise; sized for the splits of the launch on the current device.
+// The split partials: one [64][512] f32 block and 64 (m, l) pairs per (layer, row, split)
+// when a (row, layer) is split, none otherwise; sized for the splits of the launch on the
+// current device.
 size_t attn_workspace_bytes(long long rows, int L, int, int k, int sm_budget) {
   const int ns = launch_splits(rows, L, k, sm_budget);
-  return ns > 1 ? (size_t)rows * L * ns * kPartialFloats * sizeof(float) : 0;
+  return ns > 1 ? (size_t)rows * L * ns * (kPartialFloats + kPartialMl) * sizeof(float) : 0;
 }
 
 cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t* idx, int B, int T, int N, int H,
@@ -714,26 +655,34 @@ cudaError_t launch_sparse_attn_tc(const AttnLayers& layers, int L, const int32_t
   const int nsplit = launch_splits(rows, L, k, sm_budget);
   if (nsplit <= 0) return cudaErrorInvalidDevice;
   const int chunk = attn_split_chunk(k, nsplit);
-  if (nsplit > 1 && (!ws || ws_bytes < (size_t)rows * L * nsplit * kPartialFloats * sizeof(float)))
+  const size_t part_floats = (size_t)rows * L * nsplit * kPartialFloats;
+  if (nsplit > 1 && (!ws || ws_bytes < (size_t)rows * L * nsplit * (kPartialFloats + kPartialMl) * sizeof(float)))
     return cudaErrorInvalidValue;
-  // the splits of one (row, layer) are one cluster along x
+  float* partials = static_cast<float*>(ws);
+  float2* partial_ml = nsplit > 1 ? reinterpret_cast<float2*>(partials + part_floats) : nullptr;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(nsplit, (unsigned)rows, L);
   cfg.blockDim = dim3(kThreadsA);
   cfg.dynamicSmemBytes = kSmemA;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = nsplit;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // waits in-kernel
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // waits in-kernel
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cfg.numAttrs = 1;
   const int flags = (q_early ? kAttnQEarly : 0) | (rows_once ? kAttnRowsOnce : 0);
-  return cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f,
-                            flags, idx_offset, static_cast<float*>(ws), err);
+  e = cudaLaunchKernelEx(&cfg, attn_tc_kernel, maps, layers, idx, T, N, H, k, chunk, scale * 1.4426950408889634f, flags,
+                         idx_offset, partials, partial_ml, err);
+  if (e != cudaSuccess || nsplit == 1) return e;
+  // the split combine, as the attention's programmatic dependent
+  cudaLaunchConfig_t ccfg = {};
+  ccfg.gridDim = dim3((unsigned)((H + 7) / 8), (unsigned)rows, L);
+  ccfg.blockDim = dim3(256);
+  ccfg.stream = stream;
+  ccfg.attrs = attr;
+  ccfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&ccfg, attn_combine_kernel, static_cast<const float*>(partials),
+                            static_cast<const float2*>(partial_ml), layers, H, nsplit);
 }
 
 cudaError_t attn_error_word(int** p) { return g_err_addr.get(g_attn_tc_error, p); }

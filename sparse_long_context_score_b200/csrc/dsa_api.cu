@@ -129,11 +129,6 @@ cudaError_t enqueue_group(const GroupCall& c, unsigned char* base, const GroupLa
     // in decode the indexer folds the first radix digit of the select into its epilogue
     const int sms = device_sm_count();
     if (sms <= 0) return cudaErrorInvalidDevice;
-    // A bf16 decode indexer given all SMs is no faster than one on six sevenths of them
-    // (the key stream saturates HBM either way); the SMs it leaves free take the first
-    // CTAs of the top-k and the attention, launched behind it, before it ends (measured on
-    // B200 at 128K and 1M contexts: 2-3% off the step; the E4M3 indexer gains nothing).
-    if (idx_sms == 0 && c.T == 1 && !c.f8 && c.B <= sms * 6 / 7) idx_sms = sms * 6 / 7;
     const int cap = idx_sms > 0 && idx_sms < sms ? idx_sms : sms;
     const bool fused_hist = c.T == 1 && c.B <= cap;
     if (fused_hist && (e = cudaMemsetAsync(tws.hist, 0, tws.zero_bytes, stream)) != cudaSuccess) return e;

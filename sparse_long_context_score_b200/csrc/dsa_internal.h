@@ -97,7 +97,7 @@ struct AttnLayers {
 
 constexpr int kAttnTile = 64;  // selected rows per tile of the tensor-core attention (a split's granularity)
 
-int attn_num_splits(long long rows, int L, int k, int sm_budget, const int* cluster_fit);
+int attn_num_splits(long long rows, int L, int k, int sm_budget);
 int attn_split_chunk(int k, int nsplit);
 size_t attn_workspace_bytes(long long rows, int L, int H, int k, int sm_budget = 0);
 

@@ -55,9 +55,11 @@ struct TcCfg {
   static constexpr int kN = 32 * QG;                  // MMA N
   static constexpr int kHalves = kF8 ? 1 : 2;         // 128-byte column boxes per 128-wide row
   static constexpr int kStageBytesA = kHalves * kHalfBytesA;
-  // 160 KB of keys in flight per SM in decode (measured on B200: a deeper ring is no
-  // faster); prefill: a shallower ring beside the larger B
-  static constexpr int kStages = kF8 ? (QG == 1 ? 10 : 8) : (QG == 1 ? 5 : 4);
+  // decode: 96 KB of keys in flight per SM (three bf16 or six E4M3 stages).  Measured on
+  // B200 over the 268 MB decode128k key stream on 148 SMs: 3 stages 46.0 us, 4 47.1, 5
+  // 49.2, 6 50.5 -- more requests in flight than the HBM needs only slow it down (E4M3, 134
+  // MB: 6 stages 30.7 us, 10 31.6).  Prefill: a ring of 4 (8 E4M3) beside the larger B.
+  static constexpr int kStages = kF8 ? (QG == 1 ? 6 : 8) : (QG == 1 ? 3 : 4);
   static constexpr int kHalfBytesB = kN * 128;
   static constexpr int kBytesB = kHalves * kHalfBytesB;
   static constexpr int kTmemCols = kAccBufs * kN;  // 128 or 512: a power of two >= 32

@@ -30,19 +30,22 @@ def test_packed_views_are_aligned_disjoint_and_typed():
     assert float(views[3].float().abs().sum()) == 0.0
 
 
-@pytest.mark.parametrize("name,expected", [("decode128k", 3), ("mtp", 3), ("tiny", 3), ("decode1m", 3), ("prefill", 5)])
+@pytest.mark.parametrize("name,expected", [("decode128k", 4), ("mtp", 4), ("tiny", 4), ("decode1m", 4), ("prefill", 5)])
 def test_launches_per_group(name, expected):
     # indexer + top-k (one kernel for decode-shaped rows and for long rows that fit the GPU
     # at once; else select + compact, plus a histogram kernel when the indexer does not
-    # count the first digit) + one attention launch
+    # count the first digit) + the attention (and its split combine when few (row, layer)
+    # units split their keys over several CTAs: every decode shape, not the prefill)
     assert bench.launches_per_group(C.WORKLOADS[name]) == expected
 
 
 def test_step_launches():
-    # decode128k micro-batched: two halves of 4 sequences, each indexer + cluster top-k + attention
-    assert bench.step_launches(C.WORKLOADS["decode128k"], True) == 6
-    assert bench.step_launches(C.WORKLOADS["decode128k"], False) == 3
-    # decode1m: two halves of one 1M-token sequence, 8 groups: indexer + one-launch top-k + attention
-    assert bench.step_launches(C.WORKLOADS["decode1m"], True) == 48
-    # MTP: one group, 7 draft steps: indexer + top-k + 7 attention launches
-    assert bench.step_launches(C.WORKLOADS["mtp"], False) == 9
+    # decode128k micro-batched: two halves of 4 sequences, each indexer + cluster top-k +
+    # attention + split combine
+    assert bench.step_launches(C.WORKLOADS["decode128k"], True) == 8
+    assert bench.step_launches(C.WORKLOADS["decode128k"], False) == 4
+    # decode1m: two halves of one 1M-token sequence, 8 groups: indexer + one-launch top-k +
+    # attention + split combine
+    assert bench.step_launches(C.WORKLOADS["decode1m"], True) == 64
+    # MTP: one group, 7 draft steps: indexer + top-k + 7 x (attention + split combine)
+    assert bench.step_launches(C.WORKLOADS["mtp"], False) == 16
