@@ -45,9 +45,11 @@ def parse():
     p.add_argument("--shard", default="batch", choices=["batch", "context"],
                    help="multi-GPU: each rank its own batch (weak scaling), or every sequence's context "
                         "spread over the ranks (strong scaling; sparse_long_context_score_b200.sharded)")
-    p.add_argument("--schedule", default="sequential", choices=["micro", "sequential"],
-                   help="decode workloads: one dsa_group_forward per group in order on one stream (the "
-                        "faster on B200), or dsa_decode_step (two micro-batches on two streams)")
+    p.add_argument("--schedule", default="auto", choices=["auto", "micro", "sequential"],
+                   help="decode workloads through dsa_decode_step: the groups in order on one stream, or "
+                        "two micro-batches on two streams (the indexer of one beside the top-k and "
+                        "attention of the other); auto: micro-batches when the rows are longer than a "
+                        "cluster's select holds (N > 262144, as at 1M contexts), in order otherwise")
     p.add_argument("--ncu-case", choices=["indexer", "topk", "attn", "indexer_prefill", "attn_mtp", "topk_1m",
                                           "indexer_fp8"],
                    help="run one kernel of the decode step a few times on a profiler-sized case and exit "
@@ -246,6 +248,19 @@ def make_inputs(w, device, rank):
     return groups
 
 
+# Rows longer than this take the long-row select (one cooperative launch with row barriers),
+# whose latency two micro-batches hide behind the other half's indexer (measured on B200:
+# 1M contexts 1056 -> 894 us per step, 512K 725 -> 654 us; at 128K-256K in order is faster).
+CLUSTER_MAX_ROW = 8 * 1024 * 32
+
+
+def use_micro(schedule: str, w) -> bool:
+    """Whether the decode step of workload w runs as two micro-batches."""
+    if not (w.T == 1 and w.steps == 1 and w.B >= 2):
+        return False
+    return schedule == "micro" or (schedule == "auto" and min(w.N, w.q_pos0 + 1) > CLUSTER_MAX_ROW)
+
+
 def run_ours(args, rank, world, device, w=None, e2e=True):
     """Times the workload's step on this rank's GPU.  Returns a dict: the step time (graph
     replay, inputs resident in HBM), the indexer launch time, the end-to-end times (eager
@@ -258,7 +273,7 @@ def run_ours(args, rank, world, device, w=None, e2e=True):
     torch.cuda.set_device(device)
     dsa.lib()
     groups = make_inputs(w, device, rank)
-    micro = args.schedule == "micro" and w.T == 1 and w.steps == 1 and w.B >= 2
+    micro = use_micro(args.schedule, w)
     # a decode step (one query per sequence, no draft steps) runs through dsa_decode_step, in
     # order (side = stream) unless micro-batched; MTP drafting and prefill through
     # dsa_group_forward

@@ -220,9 +220,12 @@ dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t 
  * previous one) on about two thirds of the SMs, and each micro-batch's top-k and
  * attention run beside the other's indexer on the remaining third.  With B = 1, or with
  * side == stream, the groups run in order over the whole batch on `stream`, exactly like
- * one dsa_group_forward per group (on B200 this in-order step is the faster of the two at
- * the decode shapes measured: the top-k and attention are latency-bound and take nearly
- * as long for half a batch as for all of it).  A decode step reads each selected row once,
+ * one dsa_group_forward per group.  Which is faster depends on the row length (measured on
+ * B200): with rows longer than a thread-block cluster's select holds (N > 262,144: the
+ * long-row select, latency-bound) the two micro-batches hide it behind the other half's
+ * indexer (1M contexts, B = 2: 894 against 1056 us per step of 8 groups; 512K: 654 against
+ * 725 us); at 128K-256K the in-order step is faster (decode128k, B = 8: 97 against 138 us),
+ * since the top-k and attention take nearly as long for half a batch as for all of it.  A decode step reads each selected row once,
  * so the attention gathers them under an L2 evict-first policy (dsa_group_forward keeps the
  * default policy: its caller may re-read the rows, as MTP draft steps do); the results are
  * the same either way.

@@ -49,3 +49,15 @@ def test_step_launches():
     assert bench.step_launches(C.WORKLOADS["decode1m"], True) == 64
     # MTP: one group, 7 draft steps: indexer + top-k + 7 x (attention + split combine)
     assert bench.step_launches(C.WORKLOADS["mtp"], False) == 16
+
+
+def test_auto_schedule():
+    # two micro-batches only for decode steps whose rows take the long-row select
+    W = C.WORKLOADS
+    assert bench.use_micro("auto", W["decode1m"])
+    assert not bench.use_micro("auto", W["decode128k"])
+    assert not bench.use_micro("auto", W["decode128k_fp8"])
+    assert not bench.use_micro("auto", W["mtp"])        # draft steps: not a plain decode step
+    assert not bench.use_micro("auto", W["prefill"])
+    assert not bench.use_micro("auto", C.scaled(W["decode1m"], B=1))
+    assert bench.use_micro("micro", W["decode128k"]) and not bench.use_micro("sequential", W["decode1m"])
