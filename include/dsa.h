@@ -161,7 +161,7 @@ dsa_status dsa_topk(const float *scores, int B, int T, int N, long long q_pos0, 
  *     array: at most 21 query rows (B*T) for N up to 1,048,576 (fewer for longer rows);
  *     beyond that the call returns DSA_ERR_WORKSPACE -- use dsa_topk.
  *   - The first call on a device looks up the array's device address (a runtime call,
- *     not an allocation); make that first call before any stream capture.
+ *     not an allocation).
  *   - All calls share the array and it keeps the last call's contents; the parts that
  *     must start at zero are cleared on `stream` by every call that uses them.  Calls that
  *     overlap on the GPU (unordered streams) race on the array and must not be issued.

@@ -92,10 +92,13 @@ def test_topk_special_values(dsa, orc):
 
 
 def test_topk_candidate_overflow_path(dsa, orc):
-    # more than 8192 elements share the threshold bin: resolved from the row itself
-    N, k = 60000, 2048
-    sc = np.full((2, 1, N), 1.5, np.float32)
-    sc[1, 0, 123::3] = 1.75
+    # the scan kernels (20 rows of 300000: too long for a cluster, too many chunks for one
+    # cooperative launch), with more than 8192 elements in the threshold bin: resolved
+    # from the row itself
+    B, N, k = 20, 300000, 2048
+    sc = np.full((B, 1, N), 1.5, np.float32)
+    for b in range(1, B):
+        sc[b, 0, 100 * b::2 + b % 3] = 1.75 + 0.25 * (b % 2)
     got = host(dsa.dsa_topk(dev(sc), N - 1, k))
     assert np.array_equal(got, orc.topk(sc, N - 1, k))
 
