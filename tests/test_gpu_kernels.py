@@ -65,6 +65,8 @@ def _score_rows(seed, B, T, N, levels):
     (1, 1, 50000, 49999, 2048, 1),
     # one cluster of 8 CTAs with 32 keys per thread; equal keys down to the index digits
     (1, 1, 200000, 199999, 2048, 1 << 18), (2, 1, 150000, 149999, 2048, 3),
+    # decode128k rows: one cluster of 8 CTAs per row (merge path; heavy ties: digit path)
+    (8, 1, 131072, 131071, 2048, 1 << 20), (8, 1, 131072, 131071, 2048, 5),
     # shapes for the scan kernels: more rows than one wave of clusters, rows too long
     (1, 160, 3000, 2900, 256, 1000), (1, 1, 300000, 299999, 2048, 1 << 20), (1, 1, 300000, 299999, 2048, 7),
 ])
