@@ -14,10 +14,12 @@
 //
 // One CTA per draft position (16 warps).  Warp w streams its contiguous segment of the
 // vocabulary once (coalesced 16-byte loads of p and q), accumulating the acceptance rate
-// and its residual weight; the CTA then knows the totals, and only on a rejection does the
-// warp whose segment holds the target re-read that segment to find the token.  A second,
-// one-thread-per-sequence kernel counts the leading accepted positions.  HBM-bound: 8 B
-// read per vocabulary entry and draft position.
+// and its residual weight, and keeps the residual weight of every chunk it reads (128
+// entries per warp step) in shared memory.  On a rejection the chunk sums locate the
+// target to one chunk, and only that chunk is read again: the token is found a memory round
+// trip after the stream, not a whole segment later.  A second, one-thread-per-sequence
+// kernel counts the leading accepted positions.  HBM-bound: 8 B read per vocabulary entry
+// and draft position.
 #include "dsa_common.cuh"
 #include "dsa_internal.h"
 #include "sm100.cuh"
@@ -30,10 +32,38 @@ using namespace sm100;
 
 constexpr int kVThreads = 512;
 constexpr int kVWarps = kVThreads / 32;
+// the chunk sums' shared memory: 16 warps x 8 B per chunk, at most kVMaxChunks chunks per
+// warp (a chunk is one warp step of 128 or 32 entries, or several for vocabularies beyond
+// 3,145,728 entries with 16-byte loads, 786,432 without)
+constexpr int kVMaxChunks = 1536;
+constexpr int kVerifyMaxSmem = kVWarps * kVMaxChunks * 8;
 
 __device__ __forceinline__ uint64_t residual_weight(float p, float q) {
   const float r = p - q;
   return r > 0.f ? (uint64_t)(r * 1099511627776.0f) : 0ull;  // 2^40, truncated
+}
+
+// sum of v over the warp
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// A warp's segment (a multiple of 4 entries), its steps (128 entries with 16-byte loads,
+// else 32), the steps per chunk and the chunks (the shared memory holds one weight per chunk
+// and warp).
+__host__ __device__ inline int verify_seg(int V) { return ((V + kVWarps - 1) / kVWarps + 3) & ~3; }
+__host__ __device__ inline int verify_steps(int V, int vec) {
+  const int cw = vec ? 128 : 32;
+  return (verify_seg(V) + cw - 1) / cw;
+}
+__host__ __device__ inline int verify_spc(int V, int vec) {
+  return (verify_steps(V, vec) + kVMaxChunks - 1) / kVMaxChunks;
+}
+__host__ __device__ inline int verify_chunks(int V, int vec) {
+  const int spc = verify_spc(V, vec);
+  return (verify_steps(V, vec) + spc - 1) / spc;
 }
 
 __global__ void __launch_bounds__(kVThreads)
@@ -43,30 +73,56 @@ verify_kernel(const float* __restrict__ p, const float* __restrict__ q, const in
   __shared__ float s_alpha[kVWarps];
   __shared__ unsigned long long s_w[kVWarps];
   __shared__ int s_token;
+  extern __shared__ unsigned long long s_cw[];  // [kVWarps][nchunk]: residual weight per chunk
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const long long r = blockIdx.x;
   const float* pr = p + r * V;
   const float* qr = q + r * V;
-  // contiguous segment of this warp, a multiple of 4 entries long
-  const int seg = ((V + kVWarps - 1) / kVWarps + 3) & ~3;
+  // contiguous segment of this warp, a multiple of 4 entries long, read in chunks of cw
+  // entries (one per warp step)
+  const int seg = verify_seg(V);
   const int s0 = min(V, warp * seg), s1 = min(V, s0 + seg);
+  const int cw = vec ? 128 : 32, nsteps = verify_steps(V, vec), spc = verify_spc(V, vec);
+  const int nchunk = verify_chunks(V, vec);
+  unsigned long long* cwarp = s_cw + (size_t)warp * nchunk;
   grid_dep_wait();
   float a = 0.f;
   unsigned long long w = 0ull;
+  unsigned long long wc = 0ull;  // the current chunk's weight (lane 0)
   if (vec) {
 #pragma unroll 4
-    for (int i = s0 + 4 * lane; i < s1; i += 128) {
-      const float4 pv = __ldcs(reinterpret_cast<const float4*>(pr + i));
-      const float4 qv = __ldcs(reinterpret_cast<const float4*>(qr + i));
-      a += fminf(pv.x, qv.x) + fminf(pv.y, qv.y) + fminf(pv.z, qv.z) + fminf(pv.w, qv.w);
-      w += residual_weight(pv.x, qv.x) + residual_weight(pv.y, qv.y) + residual_weight(pv.z, qv.z) +
-           residual_weight(pv.w, qv.w);
+    for (int c = 0; c < nsteps; ++c) {
+      const int i = s0 + c * 128 + 4 * lane;
+      unsigned long long wl = 0ull;
+      if (i < s1) {
+        const float4 pv = __ldcs(reinterpret_cast<const float4*>(pr + i));
+        const float4 qv = __ldcs(reinterpret_cast<const float4*>(qr + i));
+        a += fminf(pv.x, qv.x) + fminf(pv.y, qv.y) + fminf(pv.z, qv.z) + fminf(pv.w, qv.w);
+        wl = residual_weight(pv.x, qv.x) + residual_weight(pv.y, qv.y) + residual_weight(pv.z, qv.z) +
+             residual_weight(pv.w, qv.w);
+      }
+      w += wl;
+      wc += warp_sum_u64(wl);
+      if ((c + 1) % spc == 0 || c + 1 == nsteps) {
+        if (lane == 0) cwarp[c / spc] = wc;
+        wc = 0ull;
+      }
     }
   } else {
-    for (int i = s0 + lane; i < s1; i += 32) {
-      const float pv = __ldcs(pr + i), qv = __ldcs(qr + i);
-      a += fminf(pv, qv);
-      w += residual_weight(pv, qv);
+    for (int c = 0; c < nsteps; ++c) {
+      const int i = s0 + c * 32 + lane;
+      unsigned long long wl = 0ull;
+      if (i < s1) {
+        const float pv = __ldcs(pr + i), qv = __ldcs(qr + i);
+        a += fminf(pv, qv);
+        wl = residual_weight(pv, qv);
+      }
+      w += wl;
+      wc += warp_sum_u64(wl);
+      if ((c + 1) % spc == 0 || c + 1 == nsteps) {
+        if (lane == 0) cwarp[c / spc] = wc;
+        wc = 0ull;
+      }
     }
   }
 #pragma unroll
@@ -105,36 +161,59 @@ verify_kernel(const float* __restrict__ p, const float* __restrict__ q, const in
       base += s_w[i];
     }
     if (warp == ws) {
-      // this warp's segment holds the target: find the entry, 128 at a time
-      for (int i0 = s0; i0 < s1; i0 += 128) {
-        const int i = i0 + 4 * lane;
-        unsigned long long w4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) w4[e] = i + e < s1 ? residual_weight(pr[i + e], qr[i + e]) : 0ull;
-        const unsigned long long lsum = w4[0] + w4[1] + w4[2] + w4[3];
-        unsigned long long incl = lsum;
+      // this warp's segment holds the target: its chunk from the chunk sums (32 at a time),
+      // then the entry from that chunk, read again
+      const unsigned long long* cs = s_cw + (size_t)ws * nchunk;
+      int chunk = -1;
+      for (int c0 = 0; c0 < nchunk && chunk < 0; c0 += 32) {
+        const unsigned long long v = c0 + lane < nchunk ? cs[c0 + lane] : 0ull;
+        unsigned long long incl = v;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
           const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
           if (lane >= o) incl += y;
         }
-        const unsigned int hit = __ballot_sync(0xFFFFFFFFu, base + incl > T);
+        const unsigned int hit = __ballot_sync(0xFFFFFFFFu, c0 + lane < nchunk && base + incl > T);
         if (hit) {
-          if (lane == __ffs(hit) - 1) {
-            unsigned long long run = base + incl - lsum;
-            int t = i + 3;
-            for (int e = 0; e < 4; ++e) {
-              run += w4[e];
-              if (run > T) {
-                t = i + e;
-                break;
-              }
-            }
-            s_token = t;
-          }
-          break;
+          const int h = __ffs(hit) - 1;
+          chunk = c0 + h;
+          base += __shfl_sync(0xFFFFFFFFu, incl - v, h);  // weight before the chunk
+        } else {
+          base += __shfl_sync(0xFFFFFFFFu, incl, 31);
         }
-        base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      }
+      if (chunk >= 0) {
+        // the chunk's steps, read again in order until the target is passed
+        const int per = cw / 32;  // entries per lane and step: 4 (vec) or 1
+        for (int c = chunk * spc; c < min(nsteps, (chunk + 1) * spc); ++c) {
+          const int i = s0 + c * cw + per * lane;
+          unsigned long long w4[4] = {0ull, 0ull, 0ull, 0ull};
+          for (int e = 0; e < per; ++e) w4[e] = i + e < s1 ? residual_weight(pr[i + e], qr[i + e]) : 0ull;
+          const unsigned long long lsum = w4[0] + w4[1] + w4[2] + w4[3];
+          unsigned long long incl = lsum;
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const unsigned long long y = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+            if (lane >= o) incl += y;
+          }
+          const unsigned int hit = __ballot_sync(0xFFFFFFFFu, base + incl > T);
+          if (hit) {
+            if (lane == __ffs(hit) - 1) {
+              unsigned long long run = base + incl - lsum;
+              int t = i + per - 1;
+              for (int e = 0; e < per; ++e) {
+                run += w4[e];
+                if (run > T) {
+                  t = i + e;
+                  break;
+                }
+              }
+              s_token = t;
+            }
+            break;
+          }
+          base += __shfl_sync(0xFFFFFFFFu, incl, 31);
+        }
       }
     }
   }
@@ -163,8 +242,13 @@ cudaError_t launch_verify(const float* p, const float* q, const int32_t* draft, 
                           cudaStream_t stream) {
   const long long rows = (long long)B * S;
   const int vec = (V % 4 == 0) && ((reinterpret_cast<uintptr_t>(p) | reinterpret_cast<uintptr_t>(q)) % 16 == 0);
-  verify_kernel<<<(unsigned)rows, kVThreads, 0, stream>>>(p, q, draft, u, u2, V, vec, alpha, accept, token);
-  cudaError_t e = cudaGetLastError();
+  const size_t smem = (size_t)kVWarps * verify_chunks(V, vec) * sizeof(unsigned long long);  // <= kVerifyMaxSmem
+  static DeviceOnce once;
+  cudaError_t e = once.run(
+      [] { return cudaFuncSetAttribute(verify_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kVerifyMaxSmem); });
+  if (e != cudaSuccess) return e;
+  verify_kernel<<<(unsigned)rows, kVThreads, smem, stream>>>(p, q, draft, u, u2, V, vec, alpha, accept, token);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)((B + 127) / 128));

@@ -95,3 +95,11 @@ def test_verify_rejects_out_of_range_draft(dsa):
     draft = np.array([[512, -3]], np.int32)
     _, acc, tok, alen = dsa.dsa_verify(dev(p), dev(q), dev(draft), dev(u), dev(u2))
     assert host(acc).tolist() == [[0, 0]] and host(tok).tolist() == [[-1, -1]] and host(alen).tolist() == [0]
+
+
+def test_verify_vocab_beyond_one_step_per_chunk(dsa, orc):
+    """Vocabularies whose warp segments hold more steps than the kernel keeps chunk sums
+    for: a chunk spans two steps (scalar loads at 800001 entries, 16-byte loads at
+    3200000), so the resample re-reads two steps of the target's chunk."""
+    _compare(dsa, orc, *_case(74, 2, 2, 800001, temp_q=2.0))
+    _compare(dsa, orc, *_case(75, 1, 2, 3200000, temp_q=2.0))
