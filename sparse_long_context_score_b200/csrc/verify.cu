@@ -12,10 +12,10 @@
 // 2^40), their exact 64-bit sum S and target floor(floor(u2 * 2^24) * S / 2^24), and picks
 // the first token whose inclusive prefix sum exceeds the target.
 //
-// One CTA per draft position (16 warps).  Warp w streams its contiguous segment of the
-// vocabulary once (coalesced 16-byte loads of p and q), accumulating the acceptance rate
-// and its residual weight, and keeps the residual weight of every chunk it reads (128
-// entries per warp step) in shared memory.  On a rejection the chunk sums locate the
+// One CTA per draft position (32 warps).  Warp w streams its contiguous segment of the
+// vocabulary once (coalesced 16-byte loads of p and q, four steps' loads in flight per
+// thread), accumulating the acceptance rate and its residual weight, and keeps the
+// residual weight of every chunk it reads (128 entries per warp step) in shared memory.  On a rejection the chunk sums locate the
 // target to one chunk, and only that chunk is read again: the token is found a memory round
 // trip after the stream, not a whole segment later.  A second, one-thread-per-sequence
 // kernel counts the leading accepted positions.  HBM-bound: 8 B read per vocabulary entry
@@ -30,13 +30,13 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kVThreads = 512;
+constexpr int kVThreads = 1024;
 constexpr int kVWarps = kVThreads / 32;
-// the chunk sums' shared memory: 16 warps x 8 B per chunk, at most kVMaxChunks chunks per
-// warp (a chunk is one warp step of 128 or 32 entries, or several for vocabularies beyond
-// 3,145,728 entries with 16-byte loads, 786,432 without)
-constexpr int kVMaxChunks = 1536;
-constexpr int kVerifyMaxSmem = kVWarps * kVMaxChunks * 8;
+// the chunk sums' shared memory: 8 B per chunk and warp, at most kVMaxChunks chunks per
+// warp (192 KB in all); a chunk is one warp step of 128 entries (16-byte loads) or 32, or
+// several steps for the largest vocabularies
+constexpr int kVerifyMaxSmem = 196608;
+constexpr int kVMaxChunks = kVerifyMaxSmem / (kVWarps * 8);
 
 __device__ __forceinline__ uint64_t residual_weight(float p, float q) {
   const float r = p - q;
@@ -90,22 +90,33 @@ verify_kernel(const float* __restrict__ p, const float* __restrict__ q, const in
   unsigned long long w = 0ull;
   unsigned long long wc = 0ull;  // the current chunk's weight (lane 0)
   if (vec) {
-#pragma unroll 4
-    for (int c = 0; c < nsteps; ++c) {
-      const int i = s0 + c * 128 + 4 * lane;
-      unsigned long long wl = 0ull;
-      if (i < s1) {
-        const float4 pv = __ldcs(reinterpret_cast<const float4*>(pr + i));
-        const float4 qv = __ldcs(reinterpret_cast<const float4*>(qr + i));
-        a += fminf(pv.x, qv.x) + fminf(pv.y, qv.y) + fminf(pv.z, qv.z) + fminf(pv.w, qv.w);
-        wl = residual_weight(pv.x, qv.x) + residual_weight(pv.y, qv.y) + residual_weight(pv.z, qv.z) +
-             residual_weight(pv.w, qv.w);
+    // four steps' loads issued together, then their arithmetic
+    for (int c0 = 0; c0 < nsteps; c0 += 4) {
+      float4 pv[4], qv[4];
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int i = s0 + (c0 + u4) * 128 + 4 * lane;
+        if (c0 + u4 < nsteps && i < s1) {
+          pv[u4] = __ldcs(reinterpret_cast<const float4*>(pr + i));
+          qv[u4] = __ldcs(reinterpret_cast<const float4*>(qr + i));
+        } else {
+          pv[u4] = qv[u4] = make_float4(0.f, 0.f, 0.f, 0.f);
+        }
       }
-      w += wl;
-      wc += warp_sum_u64(wl);
-      if ((c + 1) % spc == 0 || c + 1 == nsteps) {
-        if (lane == 0) cwarp[c / spc] = wc;
-        wc = 0ull;
+#pragma unroll
+      for (int u4 = 0; u4 < 4; ++u4) {
+        const int c = c0 + u4;
+        if (c >= nsteps) break;
+        a += fminf(pv[u4].x, qv[u4].x) + fminf(pv[u4].y, qv[u4].y) + fminf(pv[u4].z, qv[u4].z) +
+             fminf(pv[u4].w, qv[u4].w);
+        const unsigned long long wl = residual_weight(pv[u4].x, qv[u4].x) + residual_weight(pv[u4].y, qv[u4].y) +
+                                      residual_weight(pv[u4].z, qv[u4].z) + residual_weight(pv[u4].w, qv[u4].w);
+        w += wl;
+        wc += warp_sum_u64(wl);
+        if ((c + 1) % spc == 0 || c + 1 == nsteps) {
+          if (lane == 0) cwarp[c / spc] = wc;
+          wc = 0ull;
+        }
       }
     }
   } else {
