@@ -51,7 +51,7 @@ def parse():
                         "attention of the other); auto: micro-batches when the rows are longer than a "
                         "cluster's select holds (N > 262144, as at 1M contexts), in order otherwise")
     p.add_argument("--ncu-case", choices=["indexer", "topk", "attn", "indexer_prefill", "attn_mtp", "topk_1m",
-                                          "indexer_fp8"],
+                                          "indexer_fp8", "verify"],
                    help="run one kernel of the decode step a few times on a profiler-sized case and exit "
                         "(for ncu captures; prints no benchmark line)")
     return p.parse_args()
@@ -585,7 +585,9 @@ def ncu_case(kind: str) -> None:
       indexer_prefill 512 prefill queries (causal, after 126976 cached tokens) over the
                       131072-token key cache, QG = 8 tensor-core tiles;
       topk_1m         the decode1m select: 2 rows of 1,048,576 scores, first digit counted
-                      by the indexer as in the step."""
+                      by the indexer as in the step;
+      verify          the MTP verify step: 16 x 7 draft positions over a 151552-token
+                      vocabulary (136 MB of p and q)."""
     import torch
     import synth
     import synth.device as sd
@@ -633,6 +635,18 @@ def ncu_case(kind: str) -> None:
         ws = dsa.workspace(w1.B, 1, w1.N, w1.k, w1.H, 1)
         for _ in range(launches):  # the group call: indexer (with the first digit) -> top-k -> attention
             dsa.dsa_group_forward(iq, wt, ik, [q], [kv], w1.q_pos0, w1.k, C.SCALE, ws=ws)
+    elif kind == "verify":
+        wm = C.WORKLOADS["mtp"]
+        B, S, V = wm.B, wm.steps, VERIFY_VOCAB
+        zp = sd.normal_bf16(torch.empty(B, S, V, dtype=bf, device="cuda"), wm.key(synth.KIND_Q, 1, 0))
+        zq = sd.normal_bf16(torch.empty(B, S, V, dtype=bf, device="cuda"), wm.key(synth.KIND_Q, 1, 1))
+        pr = torch.softmax(zp.float() * 2.0, dim=-1).contiguous()
+        qr = torch.softmax(zq.float() * 2.6 + zp.float(), dim=-1).contiguous()
+        draft = torch.argmax(qr, dim=-1).to(torch.int32).contiguous()
+        u = sd.unit_f32(torch.empty(B, S, dtype=torch.float32, device="cuda"), wm.key(synth.KIND_SCORES, 1, 0)) + 0.5
+        u2 = sd.unit_f32(torch.empty(B, S, dtype=torch.float32, device="cuda"), wm.key(synth.KIND_SCORES, 1, 1)) + 0.5
+        for _ in range(launches):
+            dsa.dsa_verify(pr, qr, draft, u, u2)
     else:
         rows, n = (32, 65536) if kind == "attn" else (16, 262151)
         q = sd.normal_bf16(torch.empty(rows, 1, w.H, 576, dtype=bf, device="cuda"), w.key(synth.KIND_Q))
