@@ -315,7 +315,8 @@ dsa_status dsa_merge_partials(const float *outs, const float *lses, int W, int B
  * inference", Rejection Sampling: the acceptance rate is sum_v min(p_v, q_v); the MTP
  * pages verify the draft tokens in order and cut the sequence at the first rejection).
  *   p, q    [B, S, V] f32  target and draft probabilities of each draft position
- *                          (row b*S + j is position j of sequence b); V < 2^24
+ *                          (row b*S + j is position j of sequence b; values in [0, 1]);
+ *                          V < 2^24
  *   draft   [B, S] i32     the draft tokens
  *   u, u2   [B, S] f32     uniform numbers in [0, 1): the accept test and the resample
  *   alpha   [B, S] f32 out the acceptance rate sum_v min(p_v, q_v)

@@ -43,11 +43,12 @@ __device__ __forceinline__ uint64_t residual_weight(float p, float q) {
   return r > 0.f ? (uint64_t)(r * 1099511627776.0f) : 0ull;  // 2^40, truncated
 }
 
-// sum of v over the warp
+// sum over the warp of v < 2^42 (four residual weights of a lane): two 32-bit warp
+// reductions of its 24-bit halves, each sum below 2^29
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-  return v;
+  const uint32_t lo = __reduce_add_sync(0xFFFFFFFFu, (uint32_t)(v & 0xFFFFFFull));
+  const uint32_t hi = __reduce_add_sync(0xFFFFFFFFu, (uint32_t)(v >> 24));
+  return ((unsigned long long)hi << 24) + lo;
 }
 
 // A warp's segment (a multiple of 4 entries), its steps (128 entries with 16-byte loads,
