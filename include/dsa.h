@@ -49,7 +49,8 @@ typedef enum {
     DSA_OK = 0,
     DSA_ERR_INVALID_ARG = -1,  /* null pointer, bad size, misaligned pointer          */
     DSA_ERR_UNSUPPORTED = -2,  /* a shape the kernels do not implement                */
-    DSA_ERR_WORKSPACE = -3,    /* workspace missing or smaller than dsa_workspace_size */
+    DSA_ERR_WORKSPACE = -3,    /* workspace missing or too small (dsa_workspace_size;
+                                  dsa_workspace_size_min for dsa_group_forward) */
     DSA_ERR_CUDA = -4,         /* a CUDA launch or runtime call failed                 */
     DSA_ERR_TIMEOUT = -5,      /* a bounded device-side wait gave up (see status word) */
     DSA_ERR_DEVICE = -6        /* a kernel recorded a device-side error                */
@@ -102,6 +103,17 @@ dsa_status dsa_device_error(int *code, int clear);
  * query it with the device that will run the calls current.  Returns 0 for invalid sizes.
  */
 size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L);
+
+/*
+ * The smallest workspace dsa_group_forward accepts for these sizes.  With fewer bytes than
+ * dsa_workspace_size (the whole [B, T, N] score plane), a group call with T > 1 scores and
+ * selects the query rows in chunks (of one sequence, a multiple of 8 rows, as many as the
+ * workspace holds), each chunk's score plane reusing the same space -- the prefill's plane
+ * is then never held whole (4096 x 131072 queries x keys: 2 GiB whole, 4.2 MB per 8-row
+ * chunk).  The results are the same; a chunk whose plane fits L2 is read back from it.
+ * Decode (T = 1) has no smaller form: the same as dsa_workspace_size.
+ */
+size_t dsa_workspace_size_min(int B, int T, int N, int k, int H, int L);
 
 /*
  * Step 1 -- indexer score.
@@ -199,6 +211,8 @@ dsa_status dsa_sparse_attn(const uint16_t *q, const uint16_t *kv, const int32_t 
  *                          MTP draft steps 2..7); iq, w, ik may then be NULL
  *   idx_shared [B,T,k]  the shared index list; never written when compute_indices = 0,
  *                       and read unchanged by all L layers
+ *   workspace           dsa_workspace_size bytes, or fewer down to dsa_workspace_size_min
+ *                       (the score plane in chunks of query rows, see there)
  * 1 <= L <= DSA_MAX_LAYERS.
  */
 dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t *ik,

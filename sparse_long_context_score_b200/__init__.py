@@ -28,7 +28,8 @@ STATUS = {0: "DSA_OK", -1: "DSA_ERR_INVALID_ARG", -2: "DSA_ERR_UNSUPPORTED", -3:
           -4: "DSA_ERR_CUDA", -5: "DSA_ERR_TIMEOUT", -6: "DSA_ERR_DEVICE"}
 
 # every symbol include/dsa.h declares
-EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_index_score", "dsa_index_score_e4m3",
+EXPORTS = ("dsa_status_string", "dsa_version", "dsa_workspace_size", "dsa_workspace_size_min", "dsa_index_score",
+           "dsa_index_score_e4m3",
            "dsa_sparse_attn_shard", "dsa_shard_candidates", "dsa_merge_candidates", "dsa_merge_partials",
            "dsa_topk",
            "dsa_sparse_attn", "dsa_group_forward", "dsa_topk_noalloc", "dsa_device_error",
@@ -66,6 +67,8 @@ def lib() -> ctypes.CDLL:
         L.dsa_version.restype = I
         L.dsa_workspace_size.argtypes = [I, I, I, I, I, I]
         L.dsa_workspace_size.restype = S
+        L.dsa_workspace_size_min.argtypes = [I, I, I, I, I, I]
+        L.dsa_workspace_size_min.restype = S
         L.dsa_index_score.argtypes = [P, P, P, I, I, I, LL, P, P]
         L.dsa_index_score_e4m3.argtypes = [P, P, P, I, I, I, LL, P, P]
         L.dsa_sparse_attn_shard.argtypes = [P, P, P, I, I, I, LL, I, I, F, P, P, P, S, P]
@@ -158,10 +161,16 @@ def dsa_workspace_size(B: int, T: int, N: int, k: int, H: int, L: int) -> int:
     return int(lib().dsa_workspace_size(B, T, N, k, H, L))
 
 
-def workspace(B: int, T: int, N: int, k: int, H: int, L: int, device=None):
-    """Allocate a workspace tensor of dsa_workspace_size bytes (torch allocation)."""
+def dsa_workspace_size_min(B: int, T: int, N: int, k: int, H: int, L: int) -> int:
+    return int(lib().dsa_workspace_size_min(B, T, N, k, H, L))
+
+
+def workspace(B: int, T: int, N: int, k: int, H: int, L: int, device=None, nbytes=None):
+    """Allocate a workspace tensor (torch allocation): dsa_workspace_size bytes, or
+    `nbytes` (down to dsa_workspace_size_min: a group call then scores and selects the query
+    rows in chunks)."""
     torch = _torch()
-    n = dsa_workspace_size(B, T, N, k, H, L)
+    n = dsa_workspace_size(B, T, N, k, H, L) if nbytes is None else int(nbytes)
     if n == 0:
         raise ValueError("invalid sizes for dsa_workspace_size")
     return torch.empty(n, dtype=torch.uint8, device=device or "cuda")

@@ -53,19 +53,55 @@ bool sizes_ok(int B, int T, int N) {
 
 struct GroupLayout {
   size_t topk_off, topk_bytes, scores_off, scores_bytes, attn_off, attn_bytes, total;
+  int chunk;  // query rows (of one sequence) per indexer + select pass; T: the whole plane at once
 };
 
-GroupLayout group_layout(int B, int T, int N, int k, int H, int L) {
-  const long long rows = (long long)B * T;
+// Workspace of a group call: the select's workspace and the score plane for `chunk` query
+// rows of one sequence at a time (chunk == T: all B x T rows in one pass), and the
+// attention's split partials for all rows.
+GroupLayout group_layout(int B, int T, int N, int k, int H, int L, int chunk) {
+  const long long rows = chunk >= T ? (long long)B * T : (long long)chunk;
   GroupLayout g;
+  g.chunk = chunk >= T ? T : chunk;
   g.topk_off = 0;
   g.topk_bytes = round256(topk_workspace_bytes(rows, N));
   g.scores_off = g.topk_off + g.topk_bytes;
   g.scores_bytes = round256((size_t)rows * N * sizeof(float));
   g.attn_off = g.scores_off + g.scores_bytes;
-  g.attn_bytes = round256(attn_workspace_bytes(rows, L, H, k));
+  g.attn_bytes = round256(attn_workspace_bytes((long long)B * T, L, H, k));
   g.total = g.attn_off + g.attn_bytes;
   return g;
+}
+GroupLayout group_layout(int B, int T, int N, int k, int H, int L) { return group_layout(B, T, N, k, H, L, T); }
+
+// Query rows per pass when the score plane is processed in chunks: a multiple of 8 (the
+// prefill indexer's query group), and no fewer than 8 unless T is.
+constexpr int kChunkQuantum = 8;
+int min_chunk(int T) { return T < kChunkQuantum ? T : kChunkQuantum; }
+
+// The layout a workspace of `bytes` allows: the whole plane when it fits, else the largest
+// chunk that does (chunk == 0: not even the smallest).  Decode (T == 1) never chunks.
+GroupLayout layout_for(int B, int T, int N, int k, int H, int L, size_t bytes) {
+  GroupLayout g = group_layout(B, T, N, k, H, L);
+  if (bytes >= g.total || T == 1) return g;
+  int lo = min_chunk(T), hi = T - 1;
+  GroupLayout best = group_layout(B, T, N, k, H, L, lo);
+  if (best.total > bytes) {
+    best.chunk = 0;
+    return best;
+  }
+  while (lo < hi) {  // the largest multiple of 8 below T that fits (the total grows with the chunk)
+    const int mid = ((lo + hi + 1) / 2) / kChunkQuantum * kChunkQuantum;
+    if (mid <= lo) break;
+    const GroupLayout m = group_layout(B, T, N, k, H, L, mid);
+    if (m.total <= bytes) {
+      lo = mid;
+      best = m;
+    } else {
+      hi = mid - 1;
+    }
+  }
+  return best;
 }
 
 bool heads_supported(int H) { return H == 16 || H == 32 || H == 48 || H == 64; }
@@ -123,7 +159,27 @@ cudaError_t enqueue_group(const GroupCall& c, unsigned char* base, const GroupLa
   const long long rows = (long long)c.B * c.T;
   cudaError_t e;
   if (before && (e = cudaStreamWaitEvent(stream, before, 0)) != cudaSuccess) return e;
-  if (c.compute_indices) {
+  if (c.compute_indices && g.chunk < c.T) {
+    // the score plane in chunks of query rows of one sequence, each scored and selected
+    // before the next (the chunk's plane is reused, and stays in L2 when it fits)
+    float* scores = reinterpret_cast<float*>(base + g.scores_off);
+    const size_t esz = c.f8 ? 1 : 2;
+    for (int b = 0; b < c.B; ++b)
+      for (int t0 = 0; t0 < c.T; t0 += g.chunk) {
+        const int tn = c.T - t0 < g.chunk ? c.T - t0 : g.chunk;
+        const size_t r0 = (size_t)b * c.T + t0;
+        TopkWorkspace tws = topk_workspace(base + g.topk_off, tn, c.N);
+        if ((e = launch_index_score_tc(static_cast<const unsigned char*>(c.iq) + r0 * kIndexHeads * kIndexDim * esz,
+                                       c.w + r0 * kIndexHeads,
+                                       static_cast<const unsigned char*>(c.ik) + (size_t)b * c.N * kIndexDim * esz, 1,
+                                       tn, c.N, c.q_pos0 + t0, scores, nullptr, idx_sms, c.f8, stream)) != cudaSuccess)
+          return e;
+        if ((e = launch_topk(scores, 1, tn, c.N, c.q_pos0 + t0, c.k, c.idx + r0 * c.k, tws, false, tail_sms, stream)) !=
+            cudaSuccess)
+          return e;
+      }
+    if (after_idx && (e = cudaEventRecord(after_idx, stream)) != cudaSuccess) return e;
+  } else if (c.compute_indices) {
     TopkWorkspace tws = topk_workspace(base + g.topk_off, rows, c.N);
     float* scores = reinterpret_cast<float*>(base + g.scores_off);
     // in decode the indexer folds the first radix digit of the select into its epilogue
@@ -236,6 +292,13 @@ size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L) {
   return group_layout(B, T, N, k, H, L).total;
 }
 
+size_t dsa_workspace_size_min(int B, int T, int N, int k, int H, int L) {
+  if (!sizes_ok(B, T, N) || k <= 0 || k > DSA_MAX_TOPK || H <= 0 || L <= 0 || L > DSA_MAX_LAYERS) return 0;
+  if (T == 1) return group_layout(B, T, N, k, H, L).total;
+  const size_t whole = group_layout(B, T, N, k, H, L).total, chunked = group_layout(B, T, N, k, H, L, min_chunk(T)).total;
+  return chunked < whole ? chunked : whole;
+}
+
 dsa_status dsa_index_score(const uint16_t* q, const float* w, const uint16_t* k, int B, int T, int N,
                            long long q_pos0, float* scores, cudaStream_t stream) {
   if (!q || !w || !k || !scores || !sizes_ok(B, T, N)) return DSA_ERR_INVALID_ARG;
@@ -287,8 +350,10 @@ dsa_status dsa_group_forward(const uint16_t* iq, const float* w, const uint16_t*
   if (st != DSA_OK) return st;
   c.q_pos0 = q_pos0;
   c.scale = scale;
-  const GroupLayout g = group_layout(B, T, N, k, H, L);
-  if (!workspace || workspace_bytes < g.total || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE;
+  // a workspace smaller than dsa_workspace_size (down to dsa_workspace_size_min) scores and
+  // selects the query rows in chunks
+  const GroupLayout g = layout_for(B, T, N, k, H, L, workspace_bytes);
+  if (!workspace || g.chunk == 0 || workspace_bytes < g.total || !aligned(workspace, 256)) return DSA_ERR_WORKSPACE;
   return cuda_status(enqueue_group(c, static_cast<unsigned char*>(workspace), g, 0, 0, nullptr, nullptr, stream));
 }
 

@@ -46,6 +46,13 @@ def test_workspace_size(L):
     assert L.dsa_workspace_size(1, 1, 10, 16, 64, 9) == 0        # too many layers
     big = L.dsa_workspace_size(1, 4096, 131072, 2048, 64, 4)
     assert big >= 4096 * 131072 * 4                                 # the prefill score plane
+    # the smallest workspace: the prefill's plane in chunks of 8 query rows; decode has no
+    # smaller form
+    small = L.dsa_workspace_size_min(1, 4096, 131072, 2048, 64, 4)
+    assert 8 * 131072 * 4 <= small < big // 100
+    assert L.dsa_workspace_size_min(8, 1, 131072, 2048, 64, 4) == L.dsa_workspace_size(8, 1, 131072, 2048, 64, 4)
+    assert L.dsa_workspace_size_min(1, 5, 1000, 64, 64, 1) == L.dsa_workspace_size(1, 5, 1000, 64, 64, 1)  # T < 8
+    assert L.dsa_workspace_size_min(0, 8, 10, 10, 64, 4) == 0
 
 
 FAKE = ctypes.c_void_p(1 << 20)  # aligned, never dereferenced: every call below fails validation

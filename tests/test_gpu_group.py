@@ -42,6 +42,30 @@ def test_group_matches_oracle(dsa, orc, name, kw):
         assert np.all(idx[:, t][idx[:, t] >= 0] <= w.q_pos0 + t)
 
 
+@pytest.mark.parametrize("kw", [dict(T=48, N=6000, q_pos0=6000 - 48), dict(B=2, T=45, N=5000, q_pos0=5000 - 45)])
+def test_prefill_chunked_score_plane_matches_oracle(dsa, orc, kw):
+    """A workspace smaller than dsa_workspace_size: the query rows are scored and selected
+    in chunks (8 rows at dsa_workspace_size_min, more with more bytes; ragged last chunks,
+    two sequences), with the same index lists and outputs as the oracle."""
+    w = C.scaled(C.WORKLOADS["prefill"], **kw)
+    iq, wt, ik, qs, kvs = C.host_group_inputs(w)
+    ridx, routs = orc.group_forward(iq, wt, ik, qs, kvs, w.q_pos0, w.k, C.SCALE)
+    n_min = dsa.dsa_workspace_size_min(w.B, w.T, w.N, w.k, w.H, w.L)
+    n_all = dsa.dsa_workspace_size(w.B, w.T, w.N, w.k, w.H, w.L)
+    assert n_min < n_all
+    dq, dkv = [dev_bf16(x) for x in qs], [dev_bf16(x) for x in kvs]
+    for nbytes in (n_min, n_min + 24 * w.N * 4 + 65536):
+        ws = dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, nbytes=nbytes)
+        idx, outs = dsa.dsa_group_forward(dev_bf16(iq), dev(wt), dev_bf16(ik), dq, dkv, w.q_pos0, w.k, C.SCALE, ws=ws)
+        assert np.array_equal(host(idx), ridx), f"workspace {nbytes}"
+        for l in range(w.L):
+            assert_close(host(outs[l]), routs[l], f"chunked layer {l}, workspace {nbytes}")
+    with pytest.raises(dsa.DsaError):
+        ws = dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, nbytes=n_min - 256)
+        dsa.dsa_group_forward(dev_bf16(iq), dev(wt), dev_bf16(ik), dq, dkv, w.q_pos0, w.k, C.SCALE, ws=ws)
+    assert dsa.dsa_check_device_status() == 0
+
+
 def test_index_list_is_shared_and_unchanged(dsa):
     """compute_indices=0 reads idx_shared without writing it, and gives the same outputs
     as the computing call for every layer."""
