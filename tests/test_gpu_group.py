@@ -42,7 +42,7 @@ def test_group_matches_oracle(dsa, orc, name, kw):
         assert np.all(idx[:, t][idx[:, t] >= 0] <= w.q_pos0 + t)
 
 
-@pytest.mark.parametrize("kw", [dict(T=48, N=6000, q_pos0=6000 - 48), dict(B=2, T=45, N=5000, q_pos0=5000 - 45)])
+@pytest.mark.parametrize("kw", [dict(T=24, N=4000, q_pos0=4000 - 24), dict(B=2, T=19, N=3000, q_pos0=3000 - 19)])
 def test_prefill_chunked_score_plane_matches_oracle(dsa, orc, kw):
     """A workspace smaller than dsa_workspace_size: the query rows are scored and selected
     in chunks (8 rows at dsa_workspace_size_min, more with more bytes; ragged last chunks,
@@ -54,7 +54,7 @@ def test_prefill_chunked_score_plane_matches_oracle(dsa, orc, kw):
     n_all = dsa.dsa_workspace_size(w.B, w.T, w.N, w.k, w.H, w.L)
     assert n_min < n_all
     dq, dkv = [dev_bf16(x) for x in qs], [dev_bf16(x) for x in kvs]
-    for nbytes in (n_min, n_min + 24 * w.N * 4 + 65536):
+    for nbytes in (n_min, n_min + 8 * w.N * 4 + 65536):
         ws = dsa.workspace(w.B, w.T, w.N, w.k, w.H, w.L, nbytes=nbytes)
         idx, outs = dsa.dsa_group_forward(dev_bf16(iq), dev(wt), dev_bf16(ik), dq, dkv, w.q_pos0, w.k, C.SCALE, ws=ws)
         assert np.array_equal(host(idx), ridx), f"workspace {nbytes}"
