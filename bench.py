@@ -250,7 +250,7 @@ def make_inputs(w, device, rank):
 
 # Rows longer than this take the long-row select (one cooperative launch with row barriers),
 # whose latency two micro-batches hide behind the other half's indexer (measured on B200:
-# 1M contexts 1056 -> 894 us per step, 512K 725 -> 654 us; at 128K-256K in order is faster).
+# 1M contexts 1056 -> 871 us per step, 512K 725 -> 654 us; at 128K-256K in order is faster).
 CLUSTER_MAX_ROW = 8 * 1024 * 32
 
 
@@ -571,7 +571,7 @@ def step_launches(w, micro: bool) -> int:
         return (launches_per_group(w) + (w.steps - 1) * attn_launches(C.scaled(w, L=1))) * w.groups
     b0 = (w.B + 1) // 2
     halves = [C.scaled(w, B=b0), C.scaled(w, B=w.B - b0)]
-    return sum(launches_per_group(h, sms=148 // 3) for h in halves if h.B > 0) * w.groups
+    return sum(launches_per_group(h, sms=148 // 4) for h in halves if h.B > 0) * w.groups
 
 
 def ncu_case(kind: str) -> None:

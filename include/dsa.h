@@ -231,13 +231,13 @@ dsa_status dsa_group_forward(const uint16_t *iq, const float *w, const uint16_t 
  * returns, so the call completes on `stream` like any other).  Each micro-batch runs its
  * groups in order (group g+1's indexer after group g's attention, as in a model).  The
  * HBM-bound indexers of the two micro-batches take turns (each waits for the other's
- * previous one) on about two thirds of the SMs, and each micro-batch's top-k and
- * attention run beside the other's indexer on the remaining third.  With B = 1, or with
+ * previous one) on three quarters of the SMs, and each micro-batch's top-k and attention
+ * run beside the other's indexer on the remaining quarter.  With B = 1, or with
  * side == stream, the groups run in order over the whole batch on `stream`, exactly like
  * one dsa_group_forward per group.  Which is faster depends on the row length (measured on
  * B200): with rows longer than a thread-block cluster's select holds (N > 262,144: the
  * long-row select, latency-bound) the two micro-batches hide it behind the other half's
- * indexer (1M contexts, B = 2: 894 against 1056 us per step of 8 groups; 512K: 654 against
+ * indexer (1M contexts, B = 2: 871 against 1056 us per step of 8 groups; 512K: 654 against
  * 725 us); at 128K-256K the in-order step is faster (decode128k, B = 8: 97 against 138 us),
  * since the top-k and attention take nearly as long for half a batch as for all of it.  A decode step reads each selected row once,
  * so the attention gathers them under an L2 evict-first policy (dsa_group_forward keeps the

@@ -419,10 +419,11 @@ dsa_status dsa_decode_step(const dsa_group_io* groups, int G, int L, int B, int 
   }
   const int sms = device_sm_count();
   if (sms <= 0) return cuda_status(cudaErrorInvalidDevice);
-  // The indexer keeps HBM near its peak on about two thirds of the SMs; the other
-  // micro-batch's top-k and attention run beside it on the rest (measured on B200: a
-  // 7/16 share for them was slower).
-  const int tail_sms = sms / 3, idx_sms = sms - tail_sms;
+  // The indexer keeps HBM near its peak on three quarters of the SMs; the other
+  // micro-batch's top-k and attention run beside it on the rest (measured on B200 at 1M
+  // contexts: a quarter of the SMs for them 871 us per step, a third 893, a fifth 886-893,
+  // two fifths 934).
+  const int tail_sms = sms / 4, idx_sms = sms - tail_sms;
   DecodeEvents* ev = decode_events();
   if (!ev) return cuda_status(cudaErrorInvalidDevice);
   if ((e = cudaEventRecord(ev->fork, stream)) != cudaSuccess || (e = cudaStreamWaitEvent(side, ev->fork, 0)) != cudaSuccess)
