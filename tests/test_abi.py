@@ -96,6 +96,12 @@ def test_group_forward_rejects(L):
     assert L.dsa_group_forward(None, None, None, a, a, 2, 1, 1, 64, 63, 24, 8, 0.1, 0, FAKE, a, FAKE, 1 << 30, None) == -2
     # workspace too small
     assert L.dsa_group_forward(FAKE, FAKE, FAKE, a, a, 2, 1, 1, 64, 63, 64, 8, 0.1, 1, FAKE, a, FAKE, 16, None) == -3
+    # a prefill-shaped call (T = 64 queries over 100000 keys): one byte short of the smallest
+    # chunked workspace is refused before anything is enqueued
+    n_min = L.dsa_workspace_size_min(1, 64, 100000, 2048, 64, 2)
+    assert 0 < n_min < L.dsa_workspace_size(1, 64, 100000, 2048, 64, 2)
+    assert L.dsa_group_forward(FAKE, FAKE, FAKE, a, a, 2, 1, 64, 100000, 99936, 64, 2048, 0.1, 1, FAKE, a, FAKE,
+                               n_min - 1, None) == -3
 
 
 def test_binding_refuses_cpu_tensors():
