@@ -27,7 +27,8 @@
  *     256-byte); scores and index lists 4-byte.
  *   - Calls are asynchronous: work is enqueued on `stream` and the call returns.  The
  *     library allocates no memory and keeps no per-call state; scratch memory is the
- *     caller's `workspace` (size from dsa_workspace_size).
+ *     caller's `workspace` (size from dsa_workspace_size; dsa_group_forward also takes
+ *     less, down to dsa_workspace_size_min).
  *   - Invalid arguments return an error before anything is enqueued.  DSA_ERR_CUDA
  *     reports a launch failure (cudaGetLastError after the launch).
  *   - Query t of a sequence sits at position q_pos0 + t and sees cached positions
