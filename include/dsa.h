@@ -112,6 +112,8 @@ size_t dsa_workspace_size(int B, int T, int N, int k, int H, int L);
  * workspace holds), each chunk's score plane reusing the same space -- the prefill's plane
  * is then never held whole (4096 x 131072 queries x keys: 2 GiB whole, 4.2 MB per 8-row
  * chunk).  The results are the same; a chunk whose plane fits L2 is read back from it.
+ * The cost is time (measured on B200, 4096 queries, 4 layers: 14.9 ms with the whole
+ * plane, 16.3 ms with 64 MiB of workspace, 25.1 ms with the minimum, 4.7 MiB).
  * Decode (T = 1) has no smaller form: the same as dsa_workspace_size.
  */
 size_t dsa_workspace_size_min(int B, int T, int N, int k, int H, int L);
